@@ -1,0 +1,14 @@
+"""Test infrastructure only: the plain fp64 CPU oracle for trellis-coded quantization.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never does: the product
+path fails loudly when its extension is missing instead of falling back here.
+"""
+from .tcq_oracle import (  # noqa: F401
+    build_oracle,
+    oracle_decode,
+    oracle_encode,
+    oracle_greedy,
+    oracle_path_cost,
+    oracle_words_per_block,
+)

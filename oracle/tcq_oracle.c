@@ -1,0 +1,268 @@
+/*
+ * tcq_oracle.c -- TEST INFRASTRUCTURE ONLY.
+ *
+ * A plain, slow, single-threaded CPU oracle for trellis-coded quantization
+ * (TCQ) of weight blocks over the bitshift trellis, computed in fp64.  Only
+ * the test suite, the smoke check and the CPU-baseline leg of the benchmark
+ * may load this file's library; the CUDA library never does, and the two share
+ * no code, header, table or helper.
+ *
+ * What it computes, and where the sources state it:
+ *   - Trellis-coded quantization with a stateful decoder and a "bitshift"
+ *     trellis: "QTIP: Quantization with Trellises and Incoherence Processing"
+ *     (abstract).  The state is the last L bits written, k new bits are shifted
+ *     in per weight, and the reconstruction is a codebook lookup by state.
+ *   - The search is the Viterbi dynamic program that keeps the cheapest path
+ *     into every state, linear in length: "How do you fit a 4B LLM in 1.24 GB:
+ *     trellis-coded 2-bit" (section on trellis memory and the Viterbi search).
+ *   - The branch metric is the per-coordinate weighted error d_j (x_j - c)^2,
+ *     with d_j the diagonal of the Hessian's LDL factor, and a start state is
+ *     stored per coding block: CurveTQ abstract (aggregator page, paper
+ *     2610.09212).
+ *
+ * Notation (one block): T weights x_1..x_T, weights d_1..d_T (d == NULL means
+ * d_t = 1), codebook c[0 .. 2^L).  With mask = 2^L - 1,
+ *     s_t = ((s_{t-1} << k) | b_t) & mask,      y_t = c[s_t],
+ *     J(s_0, b) = sum_t d_t (x_t - c[s_t])^2.
+ * The oracle returns the minimiser of J over every start state s_0 and every
+ * bitstream b (or over b alone for a fixed start), J_min, and the packed bits.
+ *
+ * The dynamic program is written per STATE on purpose (the plain textbook
+ * form), in double precision:
+ *   C_1[s]  = d_1 (x_1 - c[s])^2                 (every s_1 reachable: free start)
+ *   C_t[s]  = min_h C_{t-1}[(h << (L-k)) | (s >> k)] + d_t (x_t - c[s])^2
+ *   bp_t[s] = the smallest h reaching that minimum
+ *   s_T     = the smallest s minimising C_T; trace back through bp.
+ *   b_t = s_t & (2^k - 1); stored start = s_1 >> k (its low L-k bits are all
+ *   the decoder can see).
+ *
+ * Bit packing (the pages are silent; this reading is fixed here): symbol t
+ * (1-based) occupies stream bits [(t-1)k, tk), most significant bit first;
+ * stream bit p is bit 31 - (p mod 32) of 32-bit word p / 32; unused bits of the
+ * last word are zero.  Words per block W = ceil(T k / 32).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_OK 0
+#define ORACLE_EINVAL (-1)
+#define ORACLE_ENOMEM (-2)
+
+static int valid_shape(int L, int k, int T)
+{
+    if (L < 1 || L > 20) return 0;
+    if (k < 1 || k > L || k > 8) return 0;
+    if (T < 1) return 0;
+    return 1;
+}
+
+int oracle_words_per_block(int k, int T)
+{
+    if (k < 1 || T < 1) return -1;
+    return (int)(((int64_t)T * k + 31) / 32);
+}
+
+/* Write the k-bit symbol b_t (1-based t) into a block's word array, one bit at
+ * a time, most significant bit first. */
+static void put_symbol(uint32_t* words, int k, int t, uint32_t sym)
+{
+    for (int i = 0; i < k; ++i) {
+        uint32_t bit = (sym >> (k - 1 - i)) & 1u;
+        int64_t p = (int64_t)(t - 1) * k + i;
+        if (bit) words[p / 32] |= 1u << (31 - (int)(p % 32));
+    }
+}
+
+/* Read the k-bit symbol b_t back, one bit at a time. */
+static uint32_t get_symbol(const uint32_t* words, int k, int t)
+{
+    uint32_t sym = 0;
+    for (int i = 0; i < k; ++i) {
+        int64_t p = (int64_t)(t - 1) * k + i;
+        uint32_t bit = (words[p / 32] >> (31 - (int)(p % 32))) & 1u;
+        sym = (sym << 1) | bit;
+    }
+    return sym;
+}
+
+static double weight_at(const double* d, int64_t i)
+{
+    return d ? d[i] : 1.0;
+}
+
+/*
+ * Viterbi encode of n_blocks independent blocks.
+ *   x, d        : [n_blocks, T] row-major (d may be NULL: d_t = 1)
+ *   cb          : codebook, 2^L values (the exact widening of the caller's
+ *                 fp32 / fp16 entries)
+ *   fixed_start : < 0 for a free start state; otherwise s_0 is fixed to it
+ *   start_state : [n_blocks] canonical stored start, s_1 >> k
+ *   bits        : [n_blocks, W] packed symbols
+ *   cost        : [n_blocks] J_min
+ */
+int oracle_encode(const double* x, const double* d, const double* cb, int L, int k,
+                  int T, int64_t n_blocks, int64_t fixed_start, uint32_t* start_state,
+                  uint32_t* bits, double* cost)
+{
+    if (!valid_shape(L, k, T) || n_blocks < 0) return ORACLE_EINVAL;
+    if (n_blocks == 0) return ORACLE_OK;
+    if (!x || !cb || !start_state || !bits || !cost) return ORACLE_EINVAL;
+
+    const int64_t S = (int64_t)1 << L;
+    const uint32_t mask = (uint32_t)(S - 1);
+    const uint32_t low_mask = (uint32_t)(((uint64_t)1 << (L - k)) - 1); /* low L-k bits */
+    const int H = 1 << k;
+    const int W = oracle_words_per_block(k, T);
+
+    double* prev = (double*)malloc(sizeof(double) * S);
+    double* cur = (double*)malloc(sizeof(double) * S);
+    uint8_t* bp = (uint8_t*)malloc((size_t)T * (size_t)S); /* bp[t-1][s], t = 1..T */
+    uint32_t* path = (uint32_t*)malloc(sizeof(uint32_t) * (size_t)T);
+    if (!prev || !cur || !bp || !path) {
+        free(prev); free(cur); free(bp); free(path);
+        return ORACLE_ENOMEM;
+    }
+
+    for (int64_t blk = 0; blk < n_blocks; ++blk) {
+        const double* xb = x + blk * T;
+        const double* db = d ? d + blk * T : NULL;
+
+        /* t = 1 */
+        for (int64_t s = 0; s < S; ++s) {
+            int reachable = 1;
+            if (fixed_start >= 0)
+                reachable = (((uint32_t)s >> k) == ((uint32_t)fixed_start & low_mask));
+            double e = xb[0] - cb[s];
+            prev[s] = reachable ? weight_at(db, 0) * e * e : INFINITY;
+            bp[s] = 0;
+        }
+
+        /* t = 2 .. T */
+        for (int t = 2; t <= T; ++t) {
+            const double xt = xb[t - 1];
+            const double dt = weight_at(db, t - 1);
+            uint8_t* bpt = bp + (size_t)(t - 1) * (size_t)S;
+            for (int64_t s = 0; s < S; ++s) {
+                double best = INFINITY;
+                int best_h = 0;
+                for (int h = 0; h < H; ++h) {
+                    uint32_t pred = (((uint32_t)h << (L - k)) | ((uint32_t)s >> k)) & mask;
+                    if (prev[pred] < best) { /* strict: the smallest h wins a tie */
+                        best = prev[pred];
+                        best_h = h;
+                    }
+                }
+                double e = xt - cb[s];
+                cur[s] = best + dt * e * e;
+                bpt[s] = (uint8_t)best_h;
+            }
+            double* tmp = prev; prev = cur; cur = tmp;
+        }
+
+        /* final state: the smallest s on ties */
+        int64_t s_best = 0;
+        for (int64_t s = 1; s < S; ++s)
+            if (prev[s] < prev[s_best]) s_best = s;
+        cost[blk] = prev[s_best];
+
+        /* trace back */
+        uint32_t s = (uint32_t)s_best;
+        path[T - 1] = s;
+        for (int t = T; t >= 2; --t) {
+            uint32_t h = bp[(size_t)(t - 1) * (size_t)S + s];
+            s = ((h << (L - k)) | (s >> k)) & mask;
+            path[t - 2] = s;
+        }
+
+        uint32_t* wb = bits + blk * W;
+        memset(wb, 0, sizeof(uint32_t) * (size_t)W);
+        for (int t = 1; t <= T; ++t)
+            put_symbol(wb, k, t, path[t - 1] & (uint32_t)(H - 1));
+        start_state[blk] = path[0] >> k;
+    }
+
+    free(prev); free(cur); free(bp); free(path);
+    return ORACLE_OK;
+}
+
+/*
+ * Decode: s_t = ((s_{t-1} << k) | b_t) & mask starting from the stored start
+ * state as given (its bits above L-k fall out of the mask), y_t = c[s_t].
+ */
+int oracle_decode(const uint32_t* bits, const uint32_t* start_state, const double* cb, int L,
+                  int k, int T, int64_t n_blocks, double* y)
+{
+    if (!valid_shape(L, k, T) || n_blocks < 0) return ORACLE_EINVAL;
+    if (n_blocks == 0) return ORACLE_OK;
+    if (!bits || !start_state || !cb || !y) return ORACLE_EINVAL;
+    const uint64_t mask = ((uint64_t)1 << L) - 1;
+    const int W = oracle_words_per_block(k, T);
+    for (int64_t blk = 0; blk < n_blocks; ++blk) {
+        uint64_t s = start_state[blk];
+        for (int t = 1; t <= T; ++t) {
+            uint32_t b = get_symbol(bits + blk * W, k, t);
+            s = ((s << k) | b) & mask;
+            y[blk * T + t - 1] = cb[s];
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* J = sum_t d_t (x_t - y_t)^2 per block, in fp64. */
+int oracle_path_cost(const double* x, const double* d, const double* y, int T, int64_t n_blocks,
+                     double* cost)
+{
+    if (T < 1 || n_blocks < 0) return ORACLE_EINVAL;
+    if (n_blocks == 0) return ORACLE_OK;
+    if (!x || !y || !cost) return ORACLE_EINVAL;
+    for (int64_t blk = 0; blk < n_blocks; ++blk) {
+        double acc = 0.0;
+        for (int t = 0; t < T; ++t) {
+            double e = x[blk * T + t] - y[blk * T + t];
+            acc += weight_at(d, blk * T + t) * e * e;
+        }
+        cost[blk] = acc;
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * Greedy trellis rounding, the baseline the Pingala-8 post shows losing to the
+ * searched path: from the given start state, at each step take the symbol whose
+ * codeword (within the current coset) is nearest, the smallest symbol on ties.
+ */
+int oracle_greedy(const double* x, const double* d, const double* cb, int L, int k, int T,
+                  int64_t n_blocks, const uint32_t* start_in, uint32_t* bits, double* cost)
+{
+    if (!valid_shape(L, k, T) || n_blocks < 0) return ORACLE_EINVAL;
+    if (n_blocks == 0) return ORACLE_OK;
+    if (!x || !cb || !start_in || !bits || !cost) return ORACLE_EINVAL;
+    const uint64_t mask = ((uint64_t)1 << L) - 1;
+    const int H = 1 << k;
+    const int W = oracle_words_per_block(k, T);
+    for (int64_t blk = 0; blk < n_blocks; ++blk) {
+        uint64_t s = start_in[blk];
+        double acc = 0.0;
+        uint32_t* wb = bits + blk * W;
+        memset(wb, 0, sizeof(uint32_t) * (size_t)W);
+        for (int t = 1; t <= T; ++t) {
+            double xt = x[blk * T + t - 1];
+            double dt = weight_at(d, blk * T + t - 1);
+            double best = INFINITY;
+            int best_b = 0;
+            for (int b = 0; b < H; ++b) {
+                uint64_t sn = ((s << k) | (uint64_t)b) & mask;
+                double e = xt - cb[sn];
+                double m = dt * e * e;
+                if (m < best) { best = m; best_b = b; }
+            }
+            s = ((s << k) | (uint64_t)best_b) & mask;
+            acc += best;
+            put_symbol(wb, k, t, (uint32_t)best_b);
+        }
+        cost[blk] = acc;
+    }
+    return ORACLE_OK;
+}

@@ -1,0 +1,162 @@
+"""ctypes wrapper of the plain C oracle (``tcq_oracle.c``).  Test infrastructure only.
+
+Everything is converted to fp64 before the call: the codebook is the exact
+widening of the caller's fp32 or fp16 entries, and x, d are the exact widening
+of their fp32 values.  See ``tcq_oracle.c`` for the definition it computes and
+the passages it follows.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "tcq_oracle.c")
+_LIB = os.path.join(_HERE, "libtcq_oracle.so")
+_lib = None
+
+
+def build_oracle(force: bool = False) -> str:
+    """Compile the oracle with plain gcc -O2 (IEEE arithmetic, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"]
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build_oracle())
+        dp = ctypes.POINTER(ctypes.c_double)
+        up = ctypes.POINTER(ctypes.c_uint32)
+        i64 = ctypes.c_int64
+        ci = ctypes.c_int
+        lib.oracle_words_per_block.argtypes = [ci, ci]
+        lib.oracle_words_per_block.restype = ci
+        lib.oracle_encode.argtypes = [dp, dp, dp, ci, ci, ci, i64, i64, up, up, dp]
+        lib.oracle_encode.restype = ci
+        lib.oracle_decode.argtypes = [up, up, dp, ci, ci, ci, i64, dp]
+        lib.oracle_decode.restype = ci
+        lib.oracle_path_cost.argtypes = [dp, dp, dp, ci, i64, dp]
+        lib.oracle_path_cost.restype = ci
+        lib.oracle_greedy.argtypes = [dp, dp, dp, ci, ci, ci, i64, up, up, dp]
+        lib.oracle_greedy.restype = ci
+        _lib = lib
+    return _lib
+
+
+def _f64(a):
+    return None if a is None else np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _u32(a):
+    return np.ascontiguousarray(np.asarray(a, dtype=np.uint32))
+
+
+def _ptr(a, ctype):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def oracle_words_per_block(k: int, T: int) -> int:
+    return int(_load().oracle_words_per_block(k, T))
+
+
+def oracle_encode(x, d, codebook, L: int, k: int, fixed_start: int | None = None):
+    """Viterbi-optimal TCQ of every row of ``x`` ([n_blocks, T]).
+
+    Returns ``(start_state uint32[n], bits uint32[n, W], cost float64[n])``.
+    ``d`` may be None (d_t = 1).  ``fixed_start`` None means a free start state.
+    """
+    x = _f64(x)
+    if x.ndim == 1:
+        x = x[None, :]
+    n, T = x.shape
+    d = _f64(d)
+    if d is not None:
+        d = np.ascontiguousarray(np.broadcast_to(d.reshape(-1, T) if d.ndim > 1 else d, (n, T)))
+    cb = _f64(codebook).reshape(-1)
+    if cb.size != (1 << L):
+        raise ValueError(f"codebook must hold 2^L = {1 << L} entries, got {cb.size}")
+    W = oracle_words_per_block(k, T)
+    start = np.zeros(n, dtype=np.uint32)
+    bits = np.zeros((n, W), dtype=np.uint32)
+    cost = np.zeros(n, dtype=np.float64)
+    rc = _load().oracle_encode(
+        _ptr(x, ctypes.c_double), _ptr(d, ctypes.c_double), _ptr(cb, ctypes.c_double),
+        L, k, T, n, -1 if fixed_start is None else int(fixed_start),
+        _ptr(start, ctypes.c_uint32), _ptr(bits, ctypes.c_uint32), _ptr(cost, ctypes.c_double),
+    )
+    if rc != 0:
+        raise ValueError(f"oracle_encode failed with code {rc}")
+    return start, bits, cost
+
+
+def oracle_decode(bits, start_state, codebook, L: int, k: int, T: int):
+    """Decode ``bits`` ([n, W]) from ``start_state`` ([n]) to fp64 values [n, T]."""
+    bits = _u32(bits)
+    if bits.ndim == 1:
+        bits = bits[None, :]
+    start = _u32(start_state).reshape(-1)
+    n = start.size
+    cb = _f64(codebook).reshape(-1)
+    y = np.zeros((n, T), dtype=np.float64)
+    rc = _load().oracle_decode(
+        _ptr(bits, ctypes.c_uint32), _ptr(start, ctypes.c_uint32), _ptr(cb, ctypes.c_double),
+        L, k, T, n, _ptr(y, ctypes.c_double),
+    )
+    if rc != 0:
+        raise ValueError(f"oracle_decode failed with code {rc}")
+    return y
+
+
+def oracle_path_cost(x, d, y):
+    """sum_t d_t (x_t - y_t)^2 per row, in fp64."""
+    x = _f64(x)
+    if x.ndim == 1:
+        x = x[None, :]
+    n, T = x.shape
+    y = _f64(y).reshape(n, T)
+    d = _f64(d)
+    if d is not None:
+        d = np.ascontiguousarray(np.broadcast_to(d.reshape(-1, T) if d.ndim > 1 else d, (n, T)))
+    cost = np.zeros(n, dtype=np.float64)
+    rc = _load().oracle_path_cost(
+        _ptr(x, ctypes.c_double), _ptr(d, ctypes.c_double), _ptr(y, ctypes.c_double),
+        T, n, _ptr(cost, ctypes.c_double),
+    )
+    if rc != 0:
+        raise ValueError(f"oracle_path_cost failed with code {rc}")
+    return cost
+
+
+def oracle_greedy(x, d, codebook, L: int, k: int, start_state):
+    """Greedy trellis rounding from the given start states; returns (bits, cost)."""
+    x = _f64(x)
+    if x.ndim == 1:
+        x = x[None, :]
+    n, T = x.shape
+    d = _f64(d)
+    if d is not None:
+        d = np.ascontiguousarray(np.broadcast_to(d.reshape(-1, T) if d.ndim > 1 else d, (n, T)))
+    cb = _f64(codebook).reshape(-1)
+    start = np.ascontiguousarray(np.broadcast_to(_u32(start_state).reshape(-1), (n,)))
+    W = oracle_words_per_block(k, T)
+    bits = np.zeros((n, W), dtype=np.uint32)
+    cost = np.zeros(n, dtype=np.float64)
+    rc = _load().oracle_greedy(
+        _ptr(x, ctypes.c_double), _ptr(d, ctypes.c_double), _ptr(cb, ctypes.c_double),
+        L, k, T, n, _ptr(start, ctypes.c_uint32), _ptr(bits, ctypes.c_uint32),
+        _ptr(cost, ctypes.c_double),
+    )
+    if rc != 0:
+        raise ValueError(f"oracle_greedy failed with code {rc}")
+    return bits, cost

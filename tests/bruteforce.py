@@ -1,0 +1,76 @@
+"""Exhaustive reference for tiny trellises, written independently of the oracle.
+
+It shares nothing with ``oracle/``: no recurrence, no traceback.  Every start
+state s_0 in [0, 2^L) and every bitstream b in [0, 2^k)^T is enumerated, and the
+state at step t is read straight off the bit window: with the stream as one
+integer n of T*k bits (b_1 in the most significant bits),
+
+    s_t = ((s_0 << t*k) | (n >> (T - t)*k)) mod 2^L,
+
+which is the "last L bits written" reading of the bitshift trellis.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def states_for(L: int, k: int, T: int, s0: np.ndarray, n: np.ndarray) -> np.ndarray:
+    """s_t for every (s0, n) pair given as broadcastable int64 arrays; shape [..., T]."""
+    mask = (1 << L) - 1
+    out = []
+    for t in range(1, T + 1):
+        out.append(((s0 << (t * k)) | (n >> ((T - t) * k))) & mask)
+    return np.stack(out, axis=-1)
+
+
+def brute_force(x, d, codebook, L: int, k: int, fixed_start: int | None = None):
+    """Minimum of J(s_0, b) over all start states and bitstreams for one block.
+
+    Returns (J_min, s0_min, n_min) with the first minimiser in (s0, n) order.
+    """
+    x = np.asarray(x, dtype=np.float64).reshape(-1)
+    T = x.size
+    d = np.ones(T) if d is None else np.asarray(d, dtype=np.float64).reshape(-1)
+    c = np.asarray(codebook, dtype=np.float64).reshape(-1)
+    assert c.size == 1 << L
+    assert T * k <= 16, "keep the enumeration small"
+    s0 = np.arange(1 << L, dtype=np.int64) if fixed_start is None else np.array([fixed_start])
+    n = np.arange(1 << (T * k), dtype=np.int64)
+    st = states_for(L, k, T, s0[:, None], n[None, :])  # [S0, N, T]
+    err = d * (x - c[st]) ** 2
+    J = err.sum(axis=-1)
+    flat = int(np.argmin(J))
+    i0, i1 = np.unravel_index(flat, J.shape)
+    return float(J[i0, i1]), int(s0[i0]), int(n[i1])
+
+
+def unpack_symbols(words, k: int, T: int) -> np.ndarray:
+    """Symbols b_1..b_T of one block from its packed words.
+
+    Stream bit p is bit 31 - (p mod 32) of word p // 32, so the words written
+    big-endian are the stream in order; numpy's unpackbits reads each byte
+    most significant bit first.
+    """
+    w = np.asarray(words, dtype=np.uint32).reshape(-1)
+    stream = np.unpackbits(w.astype(">u4").view(np.uint8))
+    sym = np.zeros(T, dtype=np.int64)
+    for i in range(k):
+        sym = (sym << 1) | stream[np.arange(T) * k + i].astype(np.int64)
+    return sym
+
+
+def stream_value(symbols, k: int) -> int:
+    n = 0
+    for b in symbols:
+        n = (n << k) | int(b)
+    return n
+
+
+def decode_window(words, start: int, codebook, L: int, k: int, T: int) -> np.ndarray:
+    """Values y_t = c[s_t] of one block from its words and start, by the bit window."""
+    sym = unpack_symbols(words, k, T)
+    n = stream_value(sym, k)  # Python int: T*k may exceed 64 bits
+    s0 = int(start) & 0xFFFFFFFF
+    mask = (1 << L) - 1
+    st = [((s0 << (t * k)) | (n >> ((T - t) * k))) & mask for t in range(1, T + 1)]
+    return np.asarray(codebook, dtype=np.float64)[np.array(st, dtype=np.int64)]
