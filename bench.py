@@ -1,0 +1,347 @@
+"""Benchmark: Viterbi TCQ encode (+ decode round trip) of the 14336x4096 MLP-shape
+matrix at L=16, k=2, T=256 on B200, one process per GPU.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...
+
+A step is one pass of the whole hot path over the workload: the encode
+(add-compare-select forward pass, backpointers, traceback, bit packing and the
+path cost, all inside the encoder kernel) and the decode of the result.  Inputs
+(x and d: 470 MB) are larger than the 126 MB L2, so no flush is needed between
+steps.  Each rank encodes its own matrix of that shape (weak scaling); there is
+no data-path collective.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import multiprocessing as mp
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Viterbi trellis nodes/sec (blocks·T·2^L) and weights encoded/sec at L=16,k=2"
+ALGO_OPS_PER_NODE = 3  # error, square-accumulate, compare-select
+SMS, LANES_PER_SM = 148, 128
+ROOFLINE_SRC = ["trellis_coded_weight_tcq_b200/csrc/acs_grouped.cuh",
+                "trellis_coded_weight_tcq_b200/csrc/acs_grouped.cu",
+                "trellis_coded_weight_tcq_b200/csrc/common.cuh"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "acs_grouped_L16k2_traffic.json")
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0}, "fallback"
+
+
+def _kernel_hash() -> str:
+    h = hashlib.sha256()
+    for p in ROOFLINE_SRC:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic_per_launch(n_blocks: int):
+    """DRAM bytes per launch from the committed ncu capture, scaled by blocks;
+    null when the kernel source changed since the capture."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except OSError:
+        return None
+    if rec.get("kernel_sha256_16") != _kernel_hash():
+        return None
+    return rec["dram_bytes_per_block"] * n_blocks
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=10)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        rows = []
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v == "Active"})
+        load = [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(r[1] for r in rows),
+                "samples": len(rows), "reasons": reasons}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline only)
+# ---------------------------------------------------------------------------
+def _oracle_job(args):
+    from oracle import oracle_encode
+
+    x, d, cb, L, k = args
+    t0 = time.perf_counter()
+    oracle_encode(x, d, cb, L, k)
+    return time.perf_counter() - t0
+
+
+def time_oracle(pool, cores, wl, blocks_per_core: int):
+    """Wall time of the oracle on cores x blocks_per_core blocks spread over the pool."""
+    n = min(wl.n_blocks, cores * blocks_per_core)
+    jobs = [(wl.x[i:i + 1], None if wl.d is None else wl.d[i:i + 1], wl.codebook, wl.L, wl.k)
+            for i in range(n)]
+    t0 = time.perf_counter()
+    pool.map(_oracle_job, jobs, chunksize=max(1, blocks_per_core))
+    wall = time.perf_counter() - t0
+    return n, wall
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    from oracle import build_oracle
+    from trellis_coded_weight_tcq_b200 import workloads
+
+    build_oracle()
+    cores = os.cpu_count() or 1
+    pool = mp.get_context("spawn").Pool(cores)
+    wl = workloads.mlp(0)
+    per_block = wl.T * (1 << wl.L)
+    for _ in range(args.warmup):
+        time_oracle(pool, cores, wl, 1)
+    times, blocks = [], 0
+    for _ in range(args.steps):
+        n, wall = time_oracle(pool, cores, wl, 1)
+        times.append(wall)
+        blocks = n
+    pool.close()
+    ms = 1e3 * sum(times) / len(times)
+    value = blocks * per_block / (ms / 1e3)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "nodes/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "L": wl.L, "k": wl.k, "T": wl.T, "n_blocks": wl.n_blocks},
+        "weights_per_s": blocks * wl.T / (ms / 1e3),
+        "cpu_baseline": {"value": value, "unit": "nodes/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{blocks} blocks of the workload per step, one block per "
+                                   f"process, {cores} spawn processes"},
+        "e2e": {"value": value, "unit": "nodes/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    cores = os.cpu_count() or 1
+    pool = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import build_oracle
+
+        build_oracle()
+        pool = mp.get_context("spawn").Pool(cores)  # started before any CUDA work
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from trellis_coded_weight_tcq_b200 import tcq, workloads
+
+    tcq.load_library()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev,
+                                timeout=__import__("datetime").timedelta(seconds=300))
+
+    wl = workloads.NAMED[args.workload](rank)
+    L, k, T, n = wl.L, wl.k, wl.T, wl.n_blocks
+    x = torch.from_numpy(wl.x).to(dev)
+    d = None if wl.d is None else torch.from_numpy(wl.d).to(dev)
+    cb = torch.from_numpy(wl.codebook).to(dev)
+    ws = tcq.Workspace(L, k, T, n, tcq.cb_dtype_of(cb), dev)
+    W = tcq.tcq_words_per_block(k, T)
+    out = tcq.Encoded(torch.empty(n, dtype=torch.int32, device=dev),
+                      torch.empty((n, W), dtype=torch.int32, device=dev),
+                      torch.empty(n, dtype=torch.float32, device=dev))
+    y = torch.empty((n, T), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    enc_ev = []
+
+    def step(record=False):
+        if record:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+        tcq.encode(x, d, cb, L, k, ws, out)
+        if record:
+            b.record(stream)
+            enc_ev.append((a, b))
+        tcq.decode(out.bits, out.start_state, cb, L, k, T, y)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clocks:
+        t_start.record(stream)
+        for _ in range(args.steps):
+            step(record=True)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = t_start.elapsed_time(t_end) / args.steps
+    acs_ms = sum(a.elapsed_time(b) for a, b in enc_ev) / len(enc_ev)
+    if world > 1:
+        t = torch.tensor([ms, acs_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, acs_ms = t.tolist()
+    gpu_launches = 2 * args.steps  # one encoder kernel + one decoder kernel per step
+
+    # ---- end to end through the C ABI from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        pipe = tcq.HostPipeline(n, T, L, k, d is not None, torch.from_numpy(wl.codebook), dev)
+        x_h = torch.from_numpy(wl.x).pin_memory()
+        d_h = None if wl.d is None else torch.from_numpy(wl.d).pin_memory()
+        for _ in range(args.warmup):
+            pipe.run(x_h, d_h)
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            pipe.run(x_h, d_h)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = e0.elapsed_time(e1) / args.steps
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = t.item()
+        e2e = {"value": world * wl.nodes / (e2e_ms / 1e3), "unit": "nodes/s",
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": pipe.h2d_bytes(),
+               "d2h_bytes_per_step": pipe.d2h_bytes()}
+        del pipe
+
+    # sanity: the last step's result is a valid encode of the workload (cheap host check)
+    cost_h = out.path_cost.cpu().numpy()
+    assert np.all(np.isfinite(cost_h)) and np.all(cost_h >= 0)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_kind = _peaks()
+    peak_ops = SMS * LANES_PER_SM * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
+    achieved_ops = wl.nodes * ALGO_OPS_PER_NODE / (acs_ms / 1e3)
+    roofline = {
+        "bound": "alu", "kernel": tcq.tcq_encode_path(L, k, tcq.cb_dtype_of(cb)),
+        "achieved": achieved_ops / 1e12, "peak": peak_ops / 1e12, "unit": "TOP/s",
+        "frac": achieved_ops / peak_ops,
+        "traffic": _traffic_per_launch(n),
+        "peak_basis": f"{SMS} SMs x {LANES_PER_SM} lanes x {peaks.get('sm_max_mhz', 1965.0)} MHz "
+                      f"({peak_kind} max SM clock); {ALGO_OPS_PER_NODE} ops per trellis node",
+        "acs_ms_per_launch": acs_ms,
+    }
+    cpu_baseline = None
+    if pool is not None:
+        nb, wall = time_oracle(pool, cores, wl, args.cpu_blocks_per_core)
+        pool.close()
+        v = nb * T * (1 << L) / wall
+        cpu_baseline = {"value": v, "unit": "nodes/s", "cores": cores, "kind": "oracle",
+                        "sample": f"{nb} blocks of {wl.name}, {args.cpu_blocks_per_core} per "
+                                  f"process on {cores} spawn processes, {wall:.1f} s wall"}
+    line = {
+        "metric": METRIC, "value": world * wl.nodes / (ms / 1e3), "unit": "nodes/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "L": L, "k": k, "T": T, "n_blocks": n,
+                   "codebook": str(wl.codebook.dtype), "weighted": d is not None,
+                   "l2": "inputs larger than L2 (x and d are 470 MB per GPU), no flush",
+                   "parallelism": f"blocks sharded per GPU (dp{world})"},
+        "weights_per_s": world * wl.weights / (ms / 1e3),
+        "encode_ms_per_step": acs_ms, "decode_ms_per_step": ms - acs_ms,
+        "roofline": roofline, "cpu_baseline": cpu_baseline, "e2e": e2e,
+        "clocks": clocks.summary(), "gpu_launches": gpu_launches,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["mlp", "qtip", "heavy", "l12", "tiny"], default="mlp")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-blocks-per-core", type=int, default=2)
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,149 @@
+/*
+ * tcq.h -- C ABI of the B200 (sm_100a) trellis-coded quantization library.
+ *
+ * Trellis-coded quantization (TCQ) of weight blocks over the bitshift trellis
+ * with a per-coordinate weighted branch metric, and the matching decoder.
+ *
+ * The operation, and where the sources define it:
+ *   - "QTIP: Quantization with Trellises and Incoherence Processing" (abstract):
+ *     TCQ with a stateful decoder over a hardware-efficient "bitshift" trellis,
+ *     lookup codes (one codeword per state).
+ *   - "How do you fit a 4B LLM in 1.24 GB? Trellis-coded 2-bit" (sections on
+ *     trellis-coded quantization and the Viterbi search): the state picks the
+ *     coset for the next weight, the written bits pick the value and set the
+ *     next state; the encoder is the Viterbi dynamic program, linear in length;
+ *     decoding is "read bits, update state, look up values".
+ *   - CurveTQ abstract (aggregator page for paper 2610.09212): the Viterbi
+ *     branch metric weighted per coordinate by the diagonal d_j of the
+ *     Hessian's LDL factor, and a start state stored per coding block.
+ *
+ * Notation for one block of T weights: state bits L, bits per weight k,
+ * mask = 2^L - 1, codebook c[0 .. 2^L).
+ *     s_t = ((s_{t-1} << k) | b_t) & mask,   y_t = c[s_t],   t = 1..T
+ *     J   = sum_t d_t (x_t - y_t)^2
+ * tcq_encode returns, per block, a start state and bitstream b_1..b_T that
+ * minimise J over every start state and every bitstream (a free start).
+ *
+ * Storage format:
+ *   - start_state: one uint32 per block, the canonical value s_1 >> k
+ *     (< 2^(L-k)).  Decoders ignore its bits above L-k.
+ *   - bits: W = ceil(T*k/32) uint32 words per block.  Symbol t occupies stream
+ *     bits [(t-1)k, tk), most significant bit first; stream bit p is bit
+ *     31 - (p mod 32) of word p/32; unused bits of the last word are zero.
+ *     s_t is therefore the last L bits of (start_state || stream[0, tk)).
+ *
+ * Conventions for every entry point:
+ *   - All array pointers are DEVICE pointers owned by the caller.  The library
+ *     never allocates, never frees and keeps no global state (thread-safe).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *     default stream) and never synchronise.  Device-side failures surface on
+ *     the stream like any kernel failure.
+ *   - Arguments are validated on the host before anything is launched; a
+ *     rejected call launches nothing and writes nothing.
+ *   - No C++ exception crosses the ABI.
+ *   - Preconditions the host cannot check (values in device memory): x, d and
+ *     the codebook are finite and d_t >= 0.  Outside them the returned path
+ *     and cost are unspecified, but every memory access stays in bounds.
+ */
+#ifndef TCQ_H_
+#define TCQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* tcq_stream_t;
+
+typedef enum {
+    TCQ_OK = 0,
+    TCQ_ERR_INVALID_ARG = 1, /* null pointer, misaligned pointer, bad size      */
+    TCQ_ERR_UNSUPPORTED = 2, /* L, k or T outside the supported ranges          */
+    TCQ_ERR_WORKSPACE = 3,   /* workspace smaller than one resident CTA needs   */
+    TCQ_ERR_CUDA = 4,        /* a CUDA runtime call or a launch failed          */
+    TCQ_ERR_INTERNAL = 5     /* a library invariant broke (report it)           */
+} tcq_status;
+
+typedef enum {
+    TCQ_F32 = 0, /* codebook entries are IEEE binary32 */
+    TCQ_F16 = 1  /* codebook entries are IEEE binary16 */
+} tcq_dtype;
+
+/* Supported ranges: 1 <= k <= TCQ_MAX_K, k <= L <= TCQ_MAX_L, 1 <= T <= TCQ_MAX_T. */
+#define TCQ_MAX_L 16
+#define TCQ_MAX_K 4
+#define TCQ_MAX_T (1 << 20)
+
+/* Words of packed bits per block, ceil(T*k/32); -1 if k or T is out of range. */
+int tcq_words_per_block(int k, int T);
+
+/*
+ * Workspace bytes tcq_encode wants for this problem on the CURRENT device
+ * (enough for every persistent CTA the encoder would keep resident; it holds
+ * the Viterbi backpointers, k bits per group of 2^k states per step, double
+ * buffered per CTA).  Returns 0 for arguments tcq_encode would reject and for
+ * n_blocks == 0.  A smaller workspace is accepted down to one CTA's share: the
+ * encoder then runs fewer CTAs, and slower.
+ */
+size_t tcq_encode_workspace_bytes(int L, int k, int T, int64_t n_blocks, tcq_dtype cb_dtype);
+
+/*
+ * Viterbi TCQ encode of n_blocks independent blocks (the sources above: QTIP
+ * abstract for the bitshift trellis, the Viterbi section of the 2-bit post,
+ * the CurveTQ abstract for the weighted metric and the free start state).
+ *
+ *   x           fp32 [n_blocks, T] row-major, 4-byte aligned.
+ *   d           fp32 [n_blocks, T] row-major, 4-byte aligned; NULL means d_t = 1
+ *               (plain Euclidean search).
+ *   codebook    2^L entries of cb_dtype, aligned to the entry size.
+ *   start_state out: uint32 [n_blocks], canonical start s_1 >> k.
+ *   bits        out: uint32 [n_blocks, W], W = tcq_words_per_block(k, T).
+ *   path_cost   out: fp32 [n_blocks], J of the returned path (accumulated in
+ *               fp64 along the path, rounded once to fp32).
+ *   workspace   device scratch of workspace_bytes, 256-byte aligned; its
+ *               contents on entry do not matter and are garbage on return.
+ *
+ * Every returned path is optimal up to fp32 rounding of the search: J of the
+ * returned path exceeds the exact minimum by at most a few fp32 rounding
+ * errors of the path metrics.  Ties may be broken either way.
+ * n_blocks == 0 is a no-op (pointers may then be NULL).
+ */
+tcq_status tcq_encode(const float* x, const float* d, const void* codebook, tcq_dtype cb_dtype,
+                      int L, int k, int T, int64_t n_blocks, uint32_t* start_state,
+                      uint32_t* bits, float* path_cost, void* workspace, size_t workspace_bytes,
+                      tcq_stream_t stream);
+
+/*
+ * Decode (the 2-bit post's "read bits, update state, look up values"; QTIP's
+ * stateful bitshift decoder): y[b, t-1] = c[s_t] with s_t the last L bits of
+ * (start_state[b] || stream[0, tk)).  Bit-exact: y is the exact fp32 widening
+ * of the codebook entry.
+ *
+ *   bits        uint32 [n_blocks, W], 4-byte aligned.
+ *   start_state uint32 [n_blocks]; only its low L-k bits are read.
+ *   codebook    2^L entries of cb_dtype, aligned to the entry size.
+ *   y           out: fp32 [n_blocks, T] row-major, 4-byte aligned.
+ * n_blocks == 0 is a no-op.
+ */
+tcq_status tcq_decode(const uint32_t* bits, const uint32_t* start_state, const void* codebook,
+                      tcq_dtype cb_dtype, int L, int k, int T, int64_t n_blocks, float* y,
+                      tcq_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char* tcq_status_string(tcq_status status);
+
+/*
+ * Static name of the encoder kernel tcq_encode would launch for this shape
+ * ("grouped<L,k,...>" for the specialised add-compare-select kernels,
+ * "generic" for the runtime-(L,k) kernel), or "unsupported".
+ */
+const char* tcq_encode_path(int L, int k, tcq_dtype cb_dtype);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TCQ_H_ */

@@ -1,0 +1,103 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function the header declares, sizes things as documented, and rejects
+bad arguments before touching CUDA."""
+import ctypes
+
+import pytest
+
+from trellis_coded_weight_tcq_b200 import tcq
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from trellis_coded_weight_tcq_b200 import build
+
+    build.build()
+    return tcq.load_library()
+
+
+def test_every_declared_function_is_exported(lib):
+    names = tcq.header_functions()
+    assert set(names) >= {"tcq_encode", "tcq_decode", "tcq_encode_workspace_bytes",
+                          "tcq_words_per_block", "tcq_status_string", "tcq_encode_path"}
+    for name in names:
+        assert hasattr(lib, name), f"{name} declared in include/tcq.h but not exported"
+
+
+def test_words_per_block(lib):
+    assert tcq.tcq_words_per_block(2, 256) == 16
+    assert tcq.tcq_words_per_block(3, 256) == 24
+    assert tcq.tcq_words_per_block(2, 64) == 4
+    assert tcq.tcq_words_per_block(3, 11) == 2
+    assert tcq.tcq_words_per_block(1, 1) == 1
+    assert tcq.tcq_words_per_block(0, 5) == -1
+    assert tcq.tcq_words_per_block(5, 5) == -1
+    assert tcq.tcq_words_per_block(2, 0) == -1
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert tcq.tcq_status_string(s).startswith("TCQ_")
+    assert "unknown" in tcq.tcq_status_string(99)
+
+
+def test_encode_path_names(lib):
+    assert tcq.tcq_encode_path(16, 2, tcq.TCQ_F16).startswith("grouped<16,2")
+    assert tcq.tcq_encode_path(16, 3, tcq.TCQ_F16).startswith("grouped<16,3")
+    assert tcq.tcq_encode_path(12, 2, tcq.TCQ_F32).startswith("grouped<12,2")
+    assert tcq.tcq_encode_path(8, 2, tcq.TCQ_F32).startswith("grouped<8,2")
+    assert tcq.tcq_encode_path(16, 2, tcq.TCQ_F32) == "generic"
+    assert tcq.tcq_encode_path(3, 2, tcq.TCQ_F16) == "generic"
+    assert tcq.tcq_encode_path(17, 2, tcq.TCQ_F32) == "unsupported"
+    assert tcq.tcq_encode_path(8, 0, tcq.TCQ_F32) == "unsupported"
+    assert tcq.tcq_encode_path(8, 2, 7) == "unsupported"
+
+
+def test_workspace_query(lib):
+    F16, F32 = tcq.TCQ_F16, tcq.TCQ_F32
+    assert tcq.tcq_encode_workspace_bytes(16, 2, 256, 0, F16) == 0
+    assert tcq.tcq_encode_workspace_bytes(17, 2, 256, 10, F16) == 0
+    assert tcq.tcq_encode_workspace_bytes(8, 9, 256, 10, F32) == 0
+    assert tcq.tcq_encode_workspace_bytes(8, 2, 256, 10, 5) == 0
+    one = tcq.tcq_encode_workspace_bytes(16, 2, 256, 1, F16)
+    # one CTA, two round buffers of (T-1) steps x 512 threads x 8 bytes of backpointers
+    assert one == 2 * ((255 * 512 * 8 + 255) // 256 * 256)
+    many = tcq.tcq_encode_workspace_bytes(16, 2, 256, 10**6, F16)
+    assert many >= one and many % one == 0
+    # the generic kernel (fp32 codebook at L=16): one byte per (step, u) plus
+    # path metrics in global memory
+    assert tcq.tcq_encode_workspace_bytes(16, 2, 256, 1, F32) == 255 * 16384 + 2 * 4 * 16384
+    assert tcq.tcq_encode_workspace_bytes(4, 4, 1, 3, F32) == 0  # T = 1 needs no backpointers
+
+
+def test_rejections_happen_before_cuda(lib):
+    fake = ctypes.c_void_p(0x10000)  # never dereferenced: every call below is rejected on the host
+    vals = dict(x=fake, d=None, cb=fake, dt=tcq.TCQ_F32, L=8, k=2, T=16, n=4, st=fake, bits=fake,
+                cost=fake, ws=fake, wsb=1 << 20, stream=None)
+
+    def call(**over):
+        v = dict(vals, **over)
+        return tcq.tcq_encode(v["x"], v["d"], v["cb"], v["dt"], v["L"], v["k"], v["T"], v["n"],
+                              v["st"], v["bits"], v["cost"], v["ws"], v["wsb"], v["stream"])
+
+    assert call(n=0, x=None, cb=None, st=None, bits=None, cost=None, ws=None) == tcq.TCQ_OK
+    assert call(n=-1) == tcq.TCQ_ERR_INVALID_ARG
+    assert call(x=None) == tcq.TCQ_ERR_INVALID_ARG
+    assert call(ws=None) == tcq.TCQ_ERR_INVALID_ARG
+    assert call(x=ctypes.c_void_p(0x10002)) == tcq.TCQ_ERR_INVALID_ARG
+    assert call(ws=ctypes.c_void_p(0x10010)) == tcq.TCQ_ERR_INVALID_ARG
+    assert call(dt=3) == tcq.TCQ_ERR_INVALID_ARG
+    assert call(L=17) == tcq.TCQ_ERR_UNSUPPORTED
+    assert call(L=1, k=2) == tcq.TCQ_ERR_UNSUPPORTED
+    assert call(k=5, L=8) == tcq.TCQ_ERR_UNSUPPORTED
+    assert call(T=0) == tcq.TCQ_ERR_UNSUPPORTED
+    assert call(T=(1 << 20) + 1) == tcq.TCQ_ERR_UNSUPPORTED
+    dec = lambda **o: tcq.tcq_decode(o.get("bits", fake), o.get("st", fake), o.get("cb", fake),  # noqa: E731
+                                     o.get("dt", 0), o.get("L", 8), o.get("k", 2), o.get("T", 16),
+                                     o.get("n", 4), o.get("y", fake), None)
+    assert dec(n=0, bits=None, st=None, cb=None, y=None) == tcq.TCQ_OK
+    assert dec(y=None) == tcq.TCQ_ERR_INVALID_ARG
+    assert dec(bits=ctypes.c_void_p(0x10001)) == tcq.TCQ_ERR_INVALID_ARG
+    assert dec(dt=1, cb=ctypes.c_void_p(0x10001)) == tcq.TCQ_ERR_INVALID_ARG
+    assert dec(L=0) == tcq.TCQ_ERR_UNSUPPORTED
+    assert dec(n=-5) == tcq.TCQ_ERR_INVALID_ARG

@@ -1,0 +1,21 @@
+"""B200 (sm_100a) trellis-coded quantization: Viterbi encode and bitshift decode.
+
+The compute lives in the CUDA library ``libtcq.so`` (C ABI: ``include/tcq.h``);
+``tcq`` is its Python binding and ``workloads`` holds the seeded synthetic
+inputs.
+"""
+from .tcq import (  # noqa: F401
+    Encoded,
+    HostPipeline,
+    TCQError,
+    Workspace,
+    decode,
+    encode,
+    load_library,
+    tcq_decode,
+    tcq_encode,
+    tcq_encode_path,
+    tcq_encode_workspace_bytes,
+    tcq_status_string,
+    tcq_words_per_block,
+)

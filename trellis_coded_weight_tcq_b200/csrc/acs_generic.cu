@@ -1,0 +1,163 @@
+// acs_generic.cu -- Viterbi TCQ encoder for any supported (L, k) at run time.
+//
+// Same search and the same fp32 arithmetic as the grouped kernels (the
+// u-formulation of the recurrence, e = fma(-sqrt(d), c, sqrt(d) x),
+// cand = fma(e, e, M), strict compares so the smallest predecessor wins a tie),
+// without their compile-time layout: one thread per u per step, codewords read
+// through the L1 cache, one byte of backpointer per (step, u) in the workspace,
+// and the traceback done by thread 0 after each block's forward pass.  It
+// covers shapes the grouped kernels do not (L < 2k, odd sizes) and serves as a
+// second, independent GPU path in the tests; it is not tuned.
+#include "common.cuh"
+
+namespace tcq {
+
+namespace {
+
+constexpr int kGenericThreads = 256;
+// path metrics stay in shared memory up to this many bytes of ping-pong, else
+// they go to the workspace slot (global memory, L2 resident)
+constexpr size_t kGenericSmemMetricBytes = 96 * 1024;
+
+__host__ __device__ inline size_t round256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+__host__ __device__ inline size_t generic_metric_bytes(int L, int K)
+{
+    return 2 * sizeof(float) * ((size_t)1 << (L - K));
+}
+
+__host__ __device__ inline bool generic_metrics_in_smem(int L, int K)
+{
+    return generic_metric_bytes(L, K) <= kGenericSmemMetricBytes;
+}
+
+__host__ __device__ inline size_t generic_bp_bytes(int L, int K, int T)
+{
+    return round256((size_t)(T - 1) * ((size_t)1 << (L - K)));
+}
+
+__global__ void __launch_bounds__(kGenericThreads) acs_generic_kernel(EncodeArgs a)
+{
+    extern __shared__ __align__(16) float gsm[];
+    __shared__ float redv[kGenericThreads / 32];
+    __shared__ uint32_t reds[kGenericThreads / 32];
+    __shared__ uint32_t fin;
+
+    const int L = a.L, K = a.K, T = a.T;
+    const int LK = L - K;
+    const uint32_t NU = 1u << LK;
+    const int H = 1 << K;
+    unsigned char* slot = a.ws + (size_t)blockIdx.x * a.slot_bytes;
+    uint8_t* bp = slot;
+    float* Mbase = generic_metrics_in_smem(L, K)
+                       ? gsm
+                       : reinterpret_cast<float*>(slot + generic_bp_bytes(L, K, T));
+
+    for (long long b = blockIdx.x; b < a.n_blocks; b += gridDim.x) {
+        const float* xb = a.x + b * T;
+        const float* db = a.d ? a.d + b * T : nullptr;
+        float bestv = __int_as_float(0x7f800000);
+        uint32_t bests = 0xffffffffu;
+        for (int t = 1; t <= T; ++t) {
+            const float sd = db ? sqrtf(db[t - 1]) : 1.f;
+            const float ca = -sd, cx = sd * xb[t - 1];
+            const float* Mp = Mbase + ((t - 1) & 1) * NU;
+            float* Mn = Mbase + (t & 1) * NU;
+            for (uint32_t u = threadIdx.x; u < NU; u += blockDim.x) {
+                float best = __int_as_float(0x7f800000);
+                uint32_t bh = 0;
+                for (int h = 0; h < H; ++h) {
+                    const uint32_t s = ((uint32_t)h << LK) | u;
+                    const float e = fmaf(ca, load_codeword(a.cb, a.cb_f16, s), cx);
+                    const float v = fmaf(e, e, t == 1 ? 0.f : Mp[s >> K]);
+                    if (v < best) {
+                        best = v;
+                        bh = (uint32_t)h;
+                    }
+                }
+                if (t < T) {
+                    Mn[u] = best;
+                    bp[(size_t)(t - 1) * NU + u] = (uint8_t)bh;
+                } else {
+                    keep_best(best, (bh << LK) | u, bestv, bests);
+                }
+            }
+            __syncthreads();
+        }
+        // final state: lexicographic (cost, state) minimum over the CTA
+        for (int o = 16; o >= 1; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bestv, o);
+            const uint32_t os = __shfl_xor_sync(0xffffffffu, bests, o);
+            keep_best(ov, os, bestv, bests);
+        }
+        if ((threadIdx.x & 31) == 0) {
+            redv[threadIdx.x >> 5] = bestv;
+            reds[threadIdx.x >> 5] = bests;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float bv = redv[0];
+            uint32_t bs = reds[0];
+            for (int w = 1; w < (int)(blockDim.x >> 5); ++w) keep_best(redv[w], reds[w], bv, bs);
+            fin = bs;
+            // traceback, bit packing and the fp64 cost along the path
+            BackwardBitWriter bw(a.bits + b * a.W, a.W);
+            uint32_t s = fin;
+            double cost = 0.0;
+            for (int t = T; t >= 1; --t) {
+                const float dv = db ? db[t - 1] : 1.f;
+                const double e = (double)xb[t - 1] - (double)load_codeword(a.cb, a.cb_f16, s);
+                cost += (double)dv * e * e;
+                bw.put(t, K, s & (uint32_t)(H - 1));
+                if (t > 1) {
+                    const uint32_t u = s >> K;
+                    const uint32_t h = bp[(size_t)(t - 2) * NU + u];
+                    s = (h << LK) | u;
+                }
+            }
+            bw.finish();
+            a.start_state[b] = s >> K;
+            a.path_cost[b] = (float)cost;
+        }
+        __syncthreads();
+    }
+}
+
+size_t generic_slot_bytes(int L, int K, int T)
+{
+    size_t v = generic_bp_bytes(L, K, T);
+    if (!generic_metrics_in_smem(L, K)) v += round256(generic_metric_bytes(L, K));
+    return v;
+}
+
+size_t generic_smem_bytes(int L, int K, int)
+{
+    return generic_metrics_in_smem(L, K) ? generic_metric_bytes(L, K) : 0;
+}
+
+cudaError_t launch_generic(const EncodeArgs& a, int grid, cudaStream_t stream)
+{
+    const size_t smem = generic_smem_bytes(a.L, a.K, a.T);
+    cudaError_t e = cudaFuncSetAttribute(acs_generic_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    acs_generic_kernel<<<grid, kGenericThreads, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
+// two CTAs per SM: enough to overlap one CTA's serial traceback; more would only
+// multiply the workspace
+const EncodeKernelInfo kGenericInfo = {"generic", 1, kGenericThreads, 2, &generic_slot_bytes,
+                                       &generic_smem_bytes,
+                                       reinterpret_cast<const void*>(&acs_generic_kernel),
+                                       &launch_generic};
+
+}  // namespace
+
+const EncodeKernelInfo* generic_kernel_info(int L, int K)
+{
+    if (L < 1 || L > TCQ_MAX_L || K < 1 || K > TCQ_MAX_K || K > L) return nullptr;
+    return &kGenericInfo;
+}
+
+}  // namespace tcq

@@ -1,0 +1,116 @@
+// common.cuh -- device helpers and the internal launch interface shared by the
+// encoder and decoder kernels of the TCQ library.  Nothing here is visible
+// through the C ABI.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/tcq.h"
+
+namespace tcq {
+
+// Arguments of one encode launch (validated on the host before launch).
+struct EncodeArgs {
+    const float* x;        // [n_blocks, T]
+    const float* d;        // [n_blocks, T] or nullptr (d_t = 1)
+    const void* cb;        // 2^L entries
+    int cb_f16;            // 1: binary16 entries, 0: binary32
+    int L, K, T, W;        // state bits, bits per weight, block length, words per block
+    long long n_blocks;
+    uint32_t* start_state; // [n_blocks]
+    uint32_t* bits;        // [n_blocks, W]
+    float* path_cost;      // [n_blocks]
+    unsigned char* ws;     // workspace base: gridDim.x slots of slot_bytes
+    size_t slot_bytes;
+};
+
+struct DecodeArgs {
+    const uint32_t* bits;
+    const uint32_t* start_state;
+    const void* cb;
+    int cb_f16;
+    int L, K, T, W;
+    long long n_blocks;
+    float* y;
+};
+
+// One codebook entry, widened exactly to fp32.
+__device__ __forceinline__ float load_codeword(const void* cb, int f16, uint32_t s)
+{
+    if (f16) return __half2float(reinterpret_cast<const __half*>(cb)[s]);
+    return reinterpret_cast<const float*>(cb)[s];
+}
+
+// Named barrier over `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_barrier(int id, int count)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Writes one block's packed symbols from the last symbol back to the first.
+// Stream bit p is bit 31 - (p mod 32) of word p / 32; symbol t (1-based)
+// occupies stream bits [(t-1)k, tk), most significant bit first.  Every word
+// from W-1 down to 0 is written exactly once, unused low bits of the last word
+// stay zero.
+struct BackwardBitWriter {
+    uint32_t* words;
+    int idx;      // word being filled
+    uint32_t cur; // its bits so far
+
+    __device__ __forceinline__ BackwardBitWriter(uint32_t* w, int W) : words(w), idx(W - 1), cur(0) {}
+
+    __device__ __forceinline__ void put(int t, int k, uint32_t sym)
+    {
+        const int p1 = t * k - 1;  // stream position of the symbol's last bit
+        const int w1 = p1 >> 5;
+        if (w1 != idx) {           // the previous symbol closed word idx
+            words[idx] = cur;
+            idx = w1;
+            cur = 0;
+        }
+        const int nlow = (p1 & 31) + 1;  // symbol bits that land in word w1
+        if (nlow >= k) {
+            cur |= sym << (32 - nlow);
+        } else {                          // straddles words w1 - 1 and w1
+            cur |= (sym & ((1u << nlow) - 1u)) << (32 - nlow);
+            words[idx] = cur;
+            idx = w1 - 1;
+            cur = sym >> nlow;
+        }
+    }
+
+    __device__ __forceinline__ void finish() { words[idx] = cur; }
+};
+
+// Lexicographic (value, state) minimum: the smallest state wins a tie.
+__device__ __forceinline__ void keep_best(float v, uint32_t s, float& bv, uint32_t& bs)
+{
+    if (v < bv || (v == bv && s < bs)) {
+        bv = v;
+        bs = s;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host-side launch interface
+// ---------------------------------------------------------------------------
+struct EncodeKernelInfo {
+    const char* name;
+    int nteam;                              // blocks one CTA advances together
+    int threads;                            // CTA size
+    int max_ctas_per_sm;                    // cap on resident CTAs (0: occupancy decides)
+    size_t (*slot_bytes)(int L, int K, int T);  // workspace per CTA
+    size_t (*smem_bytes)(int L, int K, int T);  // dynamic shared memory per CTA
+    const void* kernel;                     // for occupancy queries
+    cudaError_t (*launch)(const EncodeArgs&, int grid, cudaStream_t);
+};
+
+// nullptr if no specialised grouped kernel exists for (L, k, codebook dtype).
+const EncodeKernelInfo* find_grouped_kernel(int L, int K, int cb_f16);
+const EncodeKernelInfo* generic_kernel_info(int L, int K);
+
+cudaError_t launch_decode(const DecodeArgs& a, int num_sms, cudaStream_t stream);
+
+}  // namespace tcq

@@ -1,0 +1,189 @@
+// tcq_abi.cu -- the C ABI declared in include/tcq.h: host-side argument checks,
+// kernel selection, grid sizing from the workspace, and launches.  No entry
+// point allocates, frees, synchronises or keeps state between calls.
+#include <stdint.h>
+
+#include "common.cuh"
+
+using namespace tcq;
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+tcq_status check_shape(int L, int k, int T)
+{
+    if (k < 1 || k > TCQ_MAX_K || L < k || L > TCQ_MAX_L) return TCQ_ERR_UNSUPPORTED;
+    if (T < 1 || T > TCQ_MAX_T) return TCQ_ERR_UNSUPPORTED;
+    return TCQ_OK;
+}
+
+bool valid_dtype(tcq_dtype dt) { return dt == TCQ_F32 || dt == TCQ_F16; }
+
+const EncodeKernelInfo* select_kernel(int L, int k, tcq_dtype dt)
+{
+    const EncodeKernelInfo* g = find_grouped_kernel(L, k, dt == TCQ_F16 ? 1 : 0);
+    return g ? g : generic_kernel_info(L, k);
+}
+
+// Streaming multiprocessors of the current device, or 0 without a device.
+int current_sms()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return sms;
+}
+
+// Resident CTAs per SM for this kernel (at least 1).
+int ctas_per_sm(const EncodeKernelInfo* info, int L, int k, int T)
+{
+    int n = 0;
+    const size_t smem = info->smem_bytes(L, k, T);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, info->kernel, info->threads, smem) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        n = 1;
+    }
+    if (info->max_ctas_per_sm > 0 && n > info->max_ctas_per_sm) n = info->max_ctas_per_sm;
+    return n > 0 ? n : 1;
+}
+
+// CTAs the encoder wants: enough for every block, at most what stays resident.
+long long wanted_ctas(const EncodeKernelInfo* info, int L, int k, int T, long long n_blocks,
+                      int sms)
+{
+    const long long by_blocks = (n_blocks + info->nteam - 1) / info->nteam;
+    const long long resident = (long long)(sms > 0 ? sms : 148) * ctas_per_sm(info, L, k, T);
+    return by_blocks < resident ? by_blocks : resident;
+}
+
+}  // namespace
+
+extern "C" {
+
+int tcq_words_per_block(int k, int T)
+{
+    if (k < 1 || k > TCQ_MAX_K || T < 1 || T > TCQ_MAX_T) return -1;
+    return (int)(((long long)T * k + 31) / 32);
+}
+
+size_t tcq_encode_workspace_bytes(int L, int k, int T, int64_t n_blocks, tcq_dtype cb_dtype)
+{
+    if (check_shape(L, k, T) != TCQ_OK || n_blocks <= 0 || !valid_dtype(cb_dtype)) return 0;
+    const EncodeKernelInfo* info = select_kernel(L, k, cb_dtype);
+    const long long ctas = wanted_ctas(info, L, k, T, n_blocks, current_sms());
+    return (size_t)ctas * info->slot_bytes(L, k, T);
+}
+
+const char* tcq_encode_path(int L, int k, tcq_dtype cb_dtype)
+{
+    if (check_shape(L, k, 1) != TCQ_OK || !valid_dtype(cb_dtype)) return "unsupported";
+    return select_kernel(L, k, cb_dtype)->name;
+}
+
+tcq_status tcq_encode(const float* x, const float* d, const void* codebook, tcq_dtype cb_dtype,
+                      int L, int k, int T, int64_t n_blocks, uint32_t* start_state,
+                      uint32_t* bits, float* path_cost, void* workspace, size_t workspace_bytes,
+                      tcq_stream_t stream)
+{
+    if (n_blocks < 0) return TCQ_ERR_INVALID_ARG;
+    if (!valid_dtype(cb_dtype)) return TCQ_ERR_INVALID_ARG;
+    const tcq_status shape = check_shape(L, k, T);
+    if (shape != TCQ_OK) return shape;
+    if (n_blocks == 0) return TCQ_OK;
+    if (!x || !codebook || !start_state || !bits || !path_cost || !workspace)
+        return TCQ_ERR_INVALID_ARG;
+    const size_t entry = cb_dtype == TCQ_F16 ? 2 : 4;
+    if (!aligned(x, 4) || (d && !aligned(d, 4)) || !aligned(codebook, entry) ||
+        !aligned(start_state, 4) || !aligned(bits, 4) || !aligned(path_cost, 4) ||
+        !aligned(workspace, 256))
+        return TCQ_ERR_INVALID_ARG;
+    if ((unsigned long long)n_blocks > (1ull << 40)) return TCQ_ERR_INVALID_ARG;
+
+    const EncodeKernelInfo* info = select_kernel(L, k, cb_dtype);
+    if (!info) return TCQ_ERR_INTERNAL;
+    const size_t slot = info->slot_bytes(L, k, T);
+    const int sms = current_sms();
+    if (sms <= 0) return TCQ_ERR_CUDA;
+    long long grid = wanted_ctas(info, L, k, T, n_blocks, sms);
+    if (slot > 0) {
+        const long long fit = (long long)(workspace_bytes / slot);
+        if (fit < 1) return TCQ_ERR_WORKSPACE;
+        if (grid > fit) grid = fit;
+    }
+    if (grid < 1) grid = 1;
+
+    EncodeArgs a;
+    a.x = x;
+    a.d = d;
+    a.cb = codebook;
+    a.cb_f16 = cb_dtype == TCQ_F16 ? 1 : 0;
+    a.L = L;
+    a.K = k;
+    a.T = T;
+    a.W = tcq_words_per_block(k, T);
+    a.n_blocks = n_blocks;
+    a.start_state = start_state;
+    a.bits = bits;
+    a.path_cost = path_cost;
+    a.ws = static_cast<unsigned char*>(workspace);
+    a.slot_bytes = slot;
+    const cudaError_t e = info->launch(a, (int)grid, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TCQ_OK : TCQ_ERR_CUDA;
+}
+
+tcq_status tcq_decode(const uint32_t* bits, const uint32_t* start_state, const void* codebook,
+                      tcq_dtype cb_dtype, int L, int k, int T, int64_t n_blocks, float* y,
+                      tcq_stream_t stream)
+{
+    if (n_blocks < 0) return TCQ_ERR_INVALID_ARG;
+    if (!valid_dtype(cb_dtype)) return TCQ_ERR_INVALID_ARG;
+    const tcq_status shape = check_shape(L, k, T);
+    if (shape != TCQ_OK) return shape;
+    if (n_blocks == 0) return TCQ_OK;
+    if (!bits || !start_state || !codebook || !y) return TCQ_ERR_INVALID_ARG;
+    const size_t entry = cb_dtype == TCQ_F16 ? 2 : 4;
+    if (!aligned(bits, 4) || !aligned(start_state, 4) || !aligned(codebook, entry) ||
+        !aligned(y, 4))
+        return TCQ_ERR_INVALID_ARG;
+    if ((unsigned long long)n_blocks > (1ull << 40)) return TCQ_ERR_INVALID_ARG;
+    const int sms = current_sms();
+    if (sms <= 0) return TCQ_ERR_CUDA;
+
+    DecodeArgs a;
+    a.bits = bits;
+    a.start_state = start_state;
+    a.cb = codebook;
+    a.cb_f16 = cb_dtype == TCQ_F16 ? 1 : 0;
+    a.L = L;
+    a.K = k;
+    a.T = T;
+    a.W = tcq_words_per_block(k, T);
+    a.n_blocks = n_blocks;
+    a.y = y;
+    const cudaError_t e = launch_decode(a, sms, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TCQ_OK : TCQ_ERR_CUDA;
+}
+
+const char* tcq_status_string(tcq_status status)
+{
+    switch (status) {
+    case TCQ_OK: return "TCQ_OK";
+    case TCQ_ERR_INVALID_ARG: return "TCQ_ERR_INVALID_ARG: null or misaligned pointer, or bad size";
+    case TCQ_ERR_UNSUPPORTED: return "TCQ_ERR_UNSUPPORTED: L, k or T outside the supported ranges";
+    case TCQ_ERR_WORKSPACE: return "TCQ_ERR_WORKSPACE: workspace smaller than one CTA's share";
+    case TCQ_ERR_CUDA: return "TCQ_ERR_CUDA: a CUDA runtime call or kernel launch failed";
+    case TCQ_ERR_INTERNAL: return "TCQ_ERR_INTERNAL: library invariant violated";
+    }
+    return "unknown tcq_status";
+}
+
+}  // extern "C"

@@ -1,0 +1,237 @@
+"""Python binding of the C ABI in ``include/tcq.h`` (argument marshalling only).
+
+The functions named like the C entry points (``tcq_encode`` ...) take raw device
+pointers and sizes exactly as the C ABI does.  ``encode``/``decode`` accept
+torch CUDA tensors, allocate outputs and workspace with torch, and launch on the
+current torch stream; ``encode_host`` additionally stages host arrays through
+pinned memory (the end-to-end path).  Every step of the search and the decode
+runs in the CUDA library: when it is missing this module raises instead of
+computing anything itself.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from dataclasses import dataclass
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libtcq.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "tcq.h")
+
+TCQ_OK = 0
+TCQ_ERR_INVALID_ARG = 1
+TCQ_ERR_UNSUPPORTED = 2
+TCQ_ERR_WORKSPACE = 3
+TCQ_ERR_CUDA = 4
+TCQ_ERR_INTERNAL = 5
+TCQ_F32 = 0
+TCQ_F16 = 1
+TCQ_MAX_L = 16
+TCQ_MAX_K = 4
+TCQ_MAX_T = 1 << 20
+
+_lib = None
+
+
+class TCQError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {tcq_status_string(status)}")
+
+
+def load_library() -> ctypes.CDLL:
+    """Load ``libtcq.so``; raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m trellis_coded_weight_tcq_b200.build` "
+            "(there is no CPU fallback)"
+        )
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, sz, i64, ci = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int64, ctypes.c_int
+    lib.tcq_words_per_block.argtypes = [ci, ci]
+    lib.tcq_words_per_block.restype = ci
+    lib.tcq_encode_workspace_bytes.argtypes = [ci, ci, ci, i64, ci]
+    lib.tcq_encode_workspace_bytes.restype = sz
+    lib.tcq_encode.argtypes = [vp, vp, vp, ci, ci, ci, ci, i64, vp, vp, vp, vp, sz, vp]
+    lib.tcq_encode.restype = ci
+    lib.tcq_decode.argtypes = [vp, vp, vp, ci, ci, ci, ci, i64, vp, vp]
+    lib.tcq_decode.restype = ci
+    lib.tcq_status_string.argtypes = [ci]
+    lib.tcq_status_string.restype = ctypes.c_char_p
+    lib.tcq_encode_path.argtypes = [ci, ci, ci]
+    lib.tcq_encode_path.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions ``include/tcq.h`` declares."""
+    with open(HEADER_PATH) as f:
+        text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+    return sorted(set(re.findall(r"\b(tcq_[a-z0-9_]+)\s*\(", text)))
+
+
+# ---------------------------------------------------------------------------
+# the C entry points, one to one
+# ---------------------------------------------------------------------------
+def tcq_words_per_block(k: int, T: int) -> int:
+    return int(load_library().tcq_words_per_block(k, T))
+
+
+def tcq_encode_workspace_bytes(L: int, k: int, T: int, n_blocks: int, cb_dtype: int) -> int:
+    return int(load_library().tcq_encode_workspace_bytes(L, k, T, n_blocks, cb_dtype))
+
+
+def tcq_encode(x, d, codebook, cb_dtype, L, k, T, n_blocks, start_state, bits, path_cost,
+               workspace, workspace_bytes, stream) -> int:
+    return int(load_library().tcq_encode(x, d, codebook, cb_dtype, L, k, T, n_blocks, start_state,
+                                          bits, path_cost, workspace, workspace_bytes, stream))
+
+
+def tcq_decode(bits, start_state, codebook, cb_dtype, L, k, T, n_blocks, y, stream) -> int:
+    return int(load_library().tcq_decode(bits, start_state, codebook, cb_dtype, L, k, T, n_blocks,
+                                          y, stream))
+
+
+def tcq_status_string(status: int) -> str:
+    return load_library().tcq_status_string(status).decode()
+
+
+def tcq_encode_path(L: int, k: int, cb_dtype: int) -> str:
+    return load_library().tcq_encode_path(L, k, cb_dtype).decode()
+
+
+# ---------------------------------------------------------------------------
+# torch conveniences (device memory and streams only)
+# ---------------------------------------------------------------------------
+def _torch():
+    import torch
+
+    return torch
+
+
+def cb_dtype_of(codebook) -> int:
+    torch = _torch()
+    if codebook.dtype == torch.float16:
+        return TCQ_F16
+    if codebook.dtype == torch.float32:
+        return TCQ_F32
+    raise TypeError(f"codebook must be float16 or float32, got {codebook.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream=None):
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status: int, what: str) -> None:
+    if status != TCQ_OK:
+        raise TCQError(status, what)
+
+
+@dataclass
+class Encoded:
+    start_state: "object"  # uint32 [n] as torch.int32 storage
+    bits: "object"         # uint32 [n, W] as torch.int32 storage
+    path_cost: "object"    # float32 [n]
+
+
+class Workspace:
+    """A reusable device workspace for ``encode`` (torch-allocated)."""
+
+    def __init__(self, L: int, k: int, T: int, n_blocks: int, cb_dtype: int, device=None):
+        torch = _torch()
+        self.nbytes = max(tcq_encode_workspace_bytes(L, k, T, n_blocks, cb_dtype), 256)
+        self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=device or "cuda")
+
+
+def encode(x, d, codebook, L: int, k: int, workspace: Workspace | None = None, out=None,
+           stream=None) -> Encoded:
+    """Viterbi TCQ of every row of ``x`` (fp32 CUDA tensor [n_blocks, T])."""
+    torch = _torch()
+    if x.dim() != 2 or x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous float32 CUDA tensor [n_blocks, T]")
+    n, T = x.shape
+    if d is not None and (d.shape != x.shape or d.dtype != torch.float32 or not d.is_contiguous()):
+        raise ValueError("d must be None or a contiguous float32 tensor shaped like x")
+    W = tcq_words_per_block(k, T)
+    if W < 0:
+        raise TCQError(TCQ_ERR_UNSUPPORTED, "tcq_words_per_block")
+    if out is None:
+        out = Encoded(
+            torch.empty(n, dtype=torch.int32, device=x.device),
+            torch.empty((n, W), dtype=torch.int32, device=x.device),
+            torch.empty(n, dtype=torch.float32, device=x.device),
+        )
+    ws = workspace or Workspace(L, k, T, n, cb_dtype_of(codebook), x.device)
+    _check(tcq_encode(_ptr(x), _ptr(d), _ptr(codebook), cb_dtype_of(codebook), L, k, T, n,
+                      _ptr(out.start_state), _ptr(out.bits), _ptr(out.path_cost),
+                      ctypes.c_void_p(ws.buf.data_ptr()), ws.nbytes, _stream_handle(stream)),
+           "tcq_encode")
+    return out
+
+
+def decode(bits, start_state, codebook, L: int, k: int, T: int, out=None, stream=None):
+    """Values [n_blocks, T] (fp32) of packed ``bits`` from ``start_state``."""
+    torch = _torch()
+    n = start_state.shape[0]
+    if out is None:
+        out = torch.empty((n, T), dtype=torch.float32, device=bits.device)
+    _check(tcq_decode(_ptr(bits), _ptr(start_state), _ptr(codebook), cb_dtype_of(codebook), L, k,
+                      T, n, _ptr(out), _stream_handle(stream)), "tcq_decode")
+    return out
+
+
+class HostPipeline:
+    """End-to-end encode of host arrays: pinned host -> device -> encode -> host.
+
+    Buffers are allocated once; ``run`` copies one step's inputs in, encodes and
+    decodes on the device, and copies start states, bits, costs (and optionally
+    the decoded values) back, all on one stream.
+    """
+
+    def __init__(self, n_blocks: int, T: int, L: int, k: int, weighted: bool, codebook_host,
+                 device=None, with_decode: bool = True):
+        torch = _torch()
+        dev = torch.device(device or "cuda")
+        self.L, self.k, self.T, self.n = L, k, T, n_blocks
+        W = tcq_words_per_block(k, T)
+        self.x_dev = torch.empty((n_blocks, T), dtype=torch.float32, device=dev)
+        self.d_dev = torch.empty((n_blocks, T), dtype=torch.float32, device=dev) if weighted else None
+        self.cb_dev = codebook_host.to(dev)
+        self.ws = Workspace(L, k, T, n_blocks, cb_dtype_of(self.cb_dev), dev)
+        self.enc = Encoded(torch.empty(n_blocks, dtype=torch.int32, device=dev),
+                           torch.empty((n_blocks, W), dtype=torch.int32, device=dev),
+                           torch.empty(n_blocks, dtype=torch.float32, device=dev))
+        self.y_dev = torch.empty((n_blocks, T), dtype=torch.float32, device=dev) if with_decode else None
+        self.start_h = torch.empty(n_blocks, dtype=torch.int32, pin_memory=True)
+        self.bits_h = torch.empty((n_blocks, W), dtype=torch.int32, pin_memory=True)
+        self.cost_h = torch.empty(n_blocks, dtype=torch.float32, pin_memory=True)
+
+    def h2d_bytes(self) -> int:
+        return self.x_dev.numel() * 4 + (self.d_dev.numel() * 4 if self.d_dev is not None else 0)
+
+    def d2h_bytes(self) -> int:
+        return (self.start_h.numel() + self.bits_h.numel() + self.cost_h.numel()) * 4
+
+    def run(self, x_pinned, d_pinned=None, stream=None):
+        self.x_dev.copy_(x_pinned, non_blocking=True)
+        if self.d_dev is not None:
+            self.d_dev.copy_(d_pinned, non_blocking=True)
+        encode(self.x_dev, self.d_dev, self.cb_dev, self.L, self.k, self.ws, self.enc, stream)
+        if self.y_dev is not None:
+            decode(self.enc.bits, self.enc.start_state, self.cb_dev, self.L, self.k, self.T,
+                   self.y_dev, stream)
+        self.start_h.copy_(self.enc.start_state, non_blocking=True)
+        self.bits_h.copy_(self.enc.bits, non_blocking=True)
+        self.cost_h.copy_(self.enc.path_cost, non_blocking=True)
+        return self.start_h, self.bits_h, self.cost_h
