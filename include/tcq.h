@@ -142,6 +142,42 @@ const char* tcq_status_string(tcq_status status);
  */
 const char* tcq_encode_path(int L, int k, tcq_dtype cb_dtype);
 
+/*
+ * Encoder for callers that cannot allocate device memory.  (The sources have no
+ * counterpart: this is an engineering addition of this library.)
+ *
+ * Some callers cannot provide tcq_encode's workspace: a host program whose own
+ * pool allocator owns the GPU's memory (a raw cudaMalloc would fail or fragment
+ * that pool), code held to a fixed device-memory budget, or a latency-critical
+ * path that must not call cudaMalloc because it may synchronise the device.
+ * This entry point takes the same arguments as tcq_encode without the
+ * workspace, and allocates nothing: it calls no cudaMalloc, cudaFree or other
+ * allocating routine.  Its scratch is a single file-scope device array of
+ * TCQ_STATIC_SCRATCH_BYTES that every GPU loading this library holds until the
+ * process exits.
+ *
+ *   - The first call on a device looks up that array's device address (with the
+ *     device current) and caches it; make that first call before any stream
+ *     capture.  Calls are thread-safe on the host.
+ *   - The scratch limits concurrency, not problem size: blocks are processed by
+ *     as many persistent CTAs as the scratch holds (at L=16, k=2, T=256 each CTA
+ *     needs about 2 MiB, so about 15 CTAs run and the call is roughly 10x slower
+ *     than tcq_encode with a full workspace).  A shape whose single-CTA share
+ *     exceeds TCQ_STATIC_SCRATCH_BYTES (very long blocks) returns
+ *     TCQ_ERR_WORKSPACE.
+ *   - Every call uses the same array.  Nothing in it needs to start at zero, and
+ *     a call never depends on what an earlier call left there; but calls that
+ *     overlap on the GPU (two streams, or two host threads on different
+ *     streams) race on it and produce garbage.  Serialise them.
+ * Other arguments, outputs and errors: as tcq_encode.
+ */
+#define TCQ_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+tcq_status tcq_encode_static_scratch(const float* x, const float* d, const void* codebook,
+                                     tcq_dtype cb_dtype, int L, int k, int T, int64_t n_blocks,
+                                     uint32_t* start_state, uint32_t* bits, float* path_cost,
+                                     tcq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -24,6 +24,25 @@ def test_every_declared_function_is_exported(lib):
         assert hasattr(lib, name), f"{name} declared in include/tcq.h but not exported"
 
 
+def test_binding_signatures_match_header(lib):
+    """Every declared function has ctypes argtypes with one entry per C parameter
+    (a missing declaration would pass 64-bit arguments as 32-bit ints)."""
+    import re
+
+    with open(tcq.HEADER_PATH) as f:
+        text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+    tcq._static_scratch_fn()
+    for name in tcq.header_functions():
+        m = re.search(r"\b" + name + r"\s*\(([^)]*)\)", text)
+        params = [p for p in m.group(1).split(",") if p.strip() and p.strip() != "void"]
+        fn = getattr(lib, name)
+        assert fn.argtypes is not None, f"{name}: binding sets no argtypes"
+        assert len(fn.argtypes) == len(params), f"{name}: {len(fn.argtypes)} != {len(params)}"
+        for c_param, py_type in zip(params, fn.argtypes):
+            if "int64_t" in c_param or "size_t" in c_param:
+                assert ctypes.sizeof(py_type) == 8, f"{name}: {c_param.strip()} must be 64-bit"
+
+
 def test_words_per_block(lib):
     assert tcq.tcq_words_per_block(2, 256) == 16
     assert tcq.tcq_words_per_block(3, 256) == 24

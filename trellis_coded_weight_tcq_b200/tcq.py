@@ -235,3 +235,21 @@ class HostPipeline:
         self.bits_h.copy_(self.enc.bits, non_blocking=True)
         self.cost_h.copy_(self.enc.path_cost, non_blocking=True)
         return self.start_h, self.bits_h, self.cost_h
+
+
+def tcq_encode_static_scratch(x, d, codebook, cb_dtype, L, k, T, n_blocks, start_state, bits,
+                              path_cost, stream) -> int:
+    """The allocation-free encoder (scratch in a static device array of the library)."""
+    fn = _static_scratch_fn()
+    return int(fn(x, d, codebook, cb_dtype, L, k, T, n_blocks, start_state, bits, path_cost,
+                  stream))
+
+
+def _static_scratch_fn():
+    lib = load_library()
+    fn = lib.tcq_encode_static_scratch
+    if fn.argtypes is None:
+        vp, i64, ci = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        fn.argtypes = [vp, vp, vp, ci, ci, ci, ci, i64, vp, vp, vp, vp]
+        fn.restype = ci
+    return fn
