@@ -201,6 +201,10 @@ def run_ours(args, rank, world, local_rank):
                                 timeout=__import__("datetime").timedelta(seconds=300))
 
     wl = workloads.NAMED[args.workload](rank)
+    if args.blocks and args.blocks < wl.n_blocks:
+        wl.x = np.ascontiguousarray(wl.x[:args.blocks])
+        wl.d = None if wl.d is None else np.ascontiguousarray(wl.d[:args.blocks])
+        wl.name += f"_first{args.blocks}blocks"
     L, k, T, n = wl.L, wl.k, wl.T, wl.n_blocks
     x = torch.from_numpy(wl.x).to(dev)
     d = None if wl.d is None else torch.from_numpy(wl.d).to(dev)
@@ -332,7 +336,10 @@ def main():
     ap.add_argument("--workload", choices=["mlp", "qtip", "heavy", "l12", "tiny"], default="mlp")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-blocks-per-core", type=int, default=2)
+    ap.add_argument("--cpu-blocks-per-core", type=int, default=4)
+    ap.add_argument("--blocks", type=int, default=0,
+                    help="encode only the first N blocks of the workload (a smaller profiling "
+                         "case; reported in config.n_blocks)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -79,8 +79,9 @@ def test_workspace_query(lib):
     assert tcq.tcq_encode_workspace_bytes(8, 9, 256, 10, F32) == 0
     assert tcq.tcq_encode_workspace_bytes(8, 2, 256, 10, 5) == 0
     one = tcq.tcq_encode_workspace_bytes(16, 2, 256, 1, F16)
-    # one CTA, two round buffers of (T-1) steps x 512 threads x 8 bytes of backpointers
-    assert one == 2 * ((255 * 512 * 8 + 255) // 256 * 256)
+    # one CTA: two round buffers of (T-1) steps x 512 threads x 8 bytes of
+    # backpointers, plus the traced path (T states of 2 bytes)
+    assert one == 2 * ((255 * 512 * 8 + 255) // 256 * 256) + 512
     many = tcq.tcq_encode_workspace_bytes(16, 2, 256, 10**6, F16)
     assert many >= one and many % one == 0
     # the generic kernel (fp32 codebook at L=16): one byte per (step, u) plus

@@ -107,6 +107,29 @@ def test_random_shapes(L, k, T, n, weighted, cb):
     check_encode(wl, start, bits, cost)
 
 
+@pytest.mark.parametrize("L,k,cb", [(16, 2, "f16"), (16, 3, "f16"), (12, 2, "f32"), (8, 2, "f32"),
+                                    (10, 2, "f16"), (16, 2, "f32")])
+@pytest.mark.parametrize("pattern", ["some_zero", "all_zero", "subnormal", "wide_range"])
+def test_weight_edge_cases(L, k, cb, pattern):
+    """d with zeros, all zero, subnormal entries, or spread over 32 decades:
+    the weighted search still returns an optimal path (the fp16 kernels carry
+    metrics divided by d and floor d relative to the block's largest weight)."""
+    wl = workloads.small_random(L, k, 48, 12, True, cb, seed=["some_zero", "all_zero", "subnormal", "wide_range"].index(pattern) * 100 + L + k)
+    rng = np.random.default_rng(L * 10 + k)
+    d = wl.d.astype(np.float64)
+    if pattern == "some_zero":
+        d[:, ::3] = 0.0
+    elif pattern == "all_zero":
+        d[:] = 0.0
+    elif pattern == "subnormal":
+        d[:, ::2] = 1e-41
+    else:
+        d = 10.0 ** rng.uniform(-20, 12, d.shape)
+    wl.d = d.astype(np.float32)
+    start, bits, cost = gpu_encode(wl)
+    check_encode(wl, start, bits, cost)
+
+
 @pytest.mark.parametrize("L,k,cb", [(8, 2, "f32"), (12, 2, "f32"), (16, 2, "f16"), (16, 3, "f16"),
                                     (10, 2, "f32"), (6, 3, "f16"), (16, 2, "f32")])
 @pytest.mark.parametrize("weighted", [False, True])

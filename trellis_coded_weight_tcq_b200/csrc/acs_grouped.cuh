@@ -17,12 +17,19 @@
 // M_{t-1}[(h << (L-2k)) | g].  The codewords of a thread's states are fixed for
 // every step and every block, so they live in registers for the whole kernel.
 //
-// Branch metric, two forms, both without cancellation so the path metrics stay
-// the true partial costs:
+// Branch metric, two forms, both without cancellation:
 //   fp32 codewords: a = -sqrt(d_t), xs = sqrt(d_t) x_t per step,
 //                   e = fma(a, c, xs) = sqrt(d_t)(x_t - c), cand = fma(e, e, M);
-//   fp16 codewords: e = c - x_t in one mixed-precision add,
-//                   cand = fma(d_t e, e, M) (the product is skipped when d = 1).
+//   fp16 codewords: e = c - x_t in one mixed-precision add and cand = fma(e, e, M'),
+//                   where the path metrics are carried divided by the current
+//                   weight, M'_t = M_t / d_t.  Dividing every candidate of a step
+//                   by the same d_t > 0 leaves the step's argmins unchanged, and
+//                   the per-node product by d_t becomes one product per metric
+//                   read, M'_{t-1} * (d_{t-1} / d_t).  To keep the ratio finite,
+//                   d_t is floored at max(2^-60 max_t d_t, FLT_MIN) per block: the
+//                   change to the cost is below 2^-60 T max d (x - c)^2, far under
+//                   any fp32 tolerance, and an all-zero d becomes a plain
+//                   Euclidean search, where every path costs 0 anyway.
 //
 // CTA layout: NTEAM teams of NT threads; each team advances one block per
 // round and the CTA loops over rounds (persistent).  Backpointers go to the
@@ -49,7 +56,8 @@ struct GCfg {
     static constexpr int LK = L - K;           // bits of u
     static constexpr int NU = 1 << LK;         // path metrics per block
     static constexpr int G = 1 << (L - 2 * K); // groups per block
-    static constexpr int REC_BITS = GPT * H * K;  // backpointer bits per thread per step
+    static constexpr int P = GPT * H;             // u values per thread (bits per plane)
+    static constexpr int REC_BITS = K * P;        // backpointer bits per thread per step
     static constexpr int UNIT_BITS = REC_BITS <= 32 ? 32 : 64;
     static constexpr int SPU = UNIT_BITS / REC_BITS;  // steps per stored unit
     static constexpr int NCOMP = NT * NTEAM;
@@ -60,6 +68,7 @@ struct GCfg {
     static_assert(L >= 2 * K, "grouped kernel needs L >= 2k");
     static_assert(NT * GPT == G, "threads x groups per thread must cover every group");
     static_assert(REC_BITS <= 64, "backpointer record must fit 64 bits");
+    static_assert(P <= 32, "a bit plane is one 32-bit register");
     static_assert(NCOMP % 32 == 0, "compute threads must be whole warps");
     static_assert(NT >= 32 ? (NT % 32 == 0) : (32 % NT == 0), "teams tile warps");
     static_assert(NTEAM == 1 || NT <= 32, "multi-team CTAs use sub-warp teams");
@@ -70,13 +79,18 @@ struct GCfg {
         size_t units = (size_t)((T - 1 + SPU - 1) / SPU) * NT;
         return (units * (UNIT_BITS / 8) + 255) & ~(size_t)255;
     }
-    static __host__ __device__ size_t slot_bytes(int, int, int T) { return 2 * NTEAM * team_bytes(T); }
+    // states s_1..s_T of the block being traced, one buffer per team
+    static __host__ __device__ size_t path_bytes(int T) { return ((size_t)T * 2 + 255) & ~(size_t)255; }
+    static __host__ __device__ size_t slot_bytes(int, int, int T)
+    {
+        return 2 * NTEAM * team_bytes(T) + NTEAM * path_bytes(T);
+    }
     static __host__ __device__ size_t smem_bytes(int, int, int)
     {
         return sizeof(float) * NTEAM * 2 * NU       // path metrics, ping-pong
                + sizeof(float2) * NTEAM * TCHUNK    // staged (a, xs)
-               + 8 * (NCOMP / 32)                   // per-warp reduction
-               + 8 * NTEAM;                         // final states
+               + 8 * (NCOMP / 32)                   // per-warp reduction (value, state)
+               + 8 * (NCOMP / 32);                  // per-warp reduction (fp64 cost)
     }
 };
 
@@ -140,27 +154,43 @@ struct Codewords<C, true> {  // binary16 pairs; the input codebook is binary16
 };
 
 // ---------------------------------------------------------------------------
-// argmin over N consecutive candidates by a tournament; the smallest index wins
-// a tie (strict compare), like the textbook recurrence.
+// Minimum of N consecutive candidates by a tournament, with the argmin given
+// as sign bits: sb[0] is a register whose sign bit is the argmin's most
+// significant bit (1: the right half won), sb[1] the next bit, and so on.  Each
+// match is decided by the sign of the fp32 difference right - left, which is
+// exact (a difference of distinct finite floats never rounds to zero with
+// gradual underflow), and a tie leaves the bit at 0, so the smallest index
+// wins like the textbook recurrence's strict compare.  The differences run on
+// the FMA pipe; only the minima and one LOP3 mux per lower bit use the ALU.
 // ---------------------------------------------------------------------------
-template <int N, int OFF, int H>
-struct ArgminTree {
-    static __device__ __forceinline__ float run(const float (&c)[H], int& idx)
+__device__ __forceinline__ uint32_t mux_sign(uint32_t s, uint32_t r, uint32_t l)
+{
+    return (s & r) | (~s & l);  // bitwise: where s has its sign bit set take r, else l
+}
+
+template <int N, int OFF>
+struct SignTree {
+    template <int H, int K>
+    static __device__ __forceinline__ float run(const float (&c)[H], uint32_t (&sb)[K])
     {
-        int il, ir;
-        const float vl = ArgminTree<N / 2, OFF, H>::run(c, il);
-        const float vr = ArgminTree<N / 2, OFF + N / 2, H>::run(c, ir);
-        const bool p = vr < vl;
-        idx = p ? ir : il;
-        return p ? vr : vl;
+        constexpr int D = (N >= 2) + (N >= 4) + (N >= 8) + (N >= 16);  // log2 N
+        uint32_t l[K], r[K];
+        const float vl = SignTree<N / 2, OFF>::template run<H, K>(c, l);
+        const float vr = SignTree<N / 2, OFF + N / 2>::template run<H, K>(c, r);
+        const uint32_t s = __float_as_uint(vr - vl);
+        sb[0] = s;
+#pragma unroll
+        for (int q = 1; q < D; ++q) sb[q] = mux_sign(s, r[q - 1], l[q - 1]);
+        return fminf(vl, vr);
     }
 };
-template <int OFF, int H>
-struct ArgminTree<1, OFF, H> {
-    static __device__ __forceinline__ float run(const float (&c)[H], int& idx)
+template <int OFF>
+struct SignTree<2, OFF> {
+    template <int H, int K>
+    static __device__ __forceinline__ float run(const float (&c)[H], uint32_t (&sb)[K])
     {
-        idx = OFF;
-        return c[OFF];
+        sb[0] = __float_as_uint(c[OFF + 1] - c[OFF]);
+        return fminf(c[OFF], c[OFF + 1]);
     }
 };
 
@@ -181,22 +211,27 @@ __device__ __forceinline__ void store_metrics(float* dst, const float (&v)[H])
 
 // One trellis step for one thread.  FIRST: M_0 = 0 (free start).  LAST: no
 // metrics or backpointers are stored; the thread keeps its best final state.
-// (p0, p1) is the step's staged pair: (a, xs) for fp32 codewords, (-x_t, d_t)
-// for fp16 codewords.
+// (p0, p1) is the step's staged pair: (a, xs) for fp32 codewords,
+// (-x_t, d_{t-1} / d_t) for fp16 codewords.  Backpointers come back as K bit planes: bit P-1-q of
+// plane l is bit K-1-l of the argmin h of the thread's q-th u value
+// (q = i * 2^k + j).
 template <class C, bool WEIGHTED, bool FIRST, bool LAST>
 __device__ __forceinline__ void acs_step(const Codewords<C, C::CB16>& cw, float p0, float p1,
                                          const float* __restrict__ Mp, float* __restrict__ Mn,
-                                         int tid, uint32_t& rec_lo, uint32_t& rec_hi,
-                                         float& bestv, uint32_t& bests)
+                                         int tid, uint32_t (&planes)[C::K], float& bestv,
+                                         uint32_t& bests)
 {
-    rec_lo = 0;
-    rec_hi = 0;
+#pragma unroll
+    for (int l = 0; l < C::K; ++l) planes[l] = 0;
 #pragma unroll
     for (int i = 0; i < C::GPT; ++i) {
         const int g = tid + i * C::NT;
         float Mh[C::H];
 #pragma unroll
-        for (int h = 0; h < C::H; ++h) Mh[h] = FIRST ? 0.f : Mp[(h << (C::L - 2 * C::K)) | g];
+        for (int h = 0; h < C::H; ++h) {
+            Mh[h] = FIRST ? 0.f : Mp[(h << (C::L - 2 * C::K)) | g];
+            if constexpr (C::CB16 && WEIGHTED) Mh[h] *= p1;  // M_{t-1}/d_{t-1} -> M_{t-1}/d_t
+        }
         float mn[C::H];
 #pragma unroll
         for (int j = 0; j < C::H; ++j) {
@@ -205,99 +240,163 @@ __device__ __forceinline__ void acs_step(const Codewords<C, C::CB16>& cw, float 
             for (int h = 0; h < C::H; ++h) {
                 if constexpr (C::CB16) {
                     const float e = cw.diff(i, h, j, p0);
-                    cand[h] = fmaf(WEIGHTED ? e * p1 : e, e, Mh[h]);
+                    cand[h] = fmaf(e, e, Mh[h]);
                 } else {
                     const float e = fmaf(p0, cw.get(i, h, j), p1);
                     cand[h] = fmaf(e, e, Mh[h]);
                 }
             }
-            int idx;
-            const float v = ArgminTree<C::H, 0, C::H>::run(cand, idx);
+            uint32_t sb[C::K];
+            const float v = SignTree<C::H, 0>::template run<C::H, C::K>(cand, sb);
             mn[j] = v;
             if constexpr (LAST) {
-                const uint32_t s = ((uint32_t)idx << C::LK) | ((uint32_t)g << C::K) | (uint32_t)j;
+                uint32_t idx = 0;
+#pragma unroll
+                for (int l = 0; l < C::K; ++l) idx = (idx << 1) | (sb[l] >> 31);
+                const uint32_t s = (idx << C::LK) | ((uint32_t)g << C::K) | (uint32_t)j;
                 keep_best(v, s, bestv, bests);
             } else {
-                const int pos = (i * C::H + j) * C::K;  // compile-time after unrolling
-                if (pos < 32) {
-                    rec_lo |= (uint32_t)idx << pos;
-                    if (pos + C::K > 32) rec_hi |= (uint32_t)idx >> (32 - pos);
-                } else {
-                    rec_hi |= (uint32_t)idx << (pos - 32);
-                }
+#pragma unroll
+                for (int l = 0; l < C::K; ++l) planes[l] = __funnelshift_l(sb[l], planes[l], 1);
             }
         }
         if constexpr (!LAST) store_metrics<C::H>(Mn + ((size_t)g << C::K), mn);
     }
 }
 
-// Traceback of one block, advanced one trellis step at a time by one thread.
-// issue() starts the loads of the current step; retire() consumes them, emits
-// the symbol, adds d_t (x_t - c[s_t])^2 to the fp64 cost and moves to s_{t-1}.
+// Traceback of one block, advanced one trellis step at a time by one thread:
+// only the dependent walk through the backpointers, storing s_tau per step.
+// issue() starts the load that decides s_{tau-1}; retire() stores s_tau and
+// moves on.  Bits, start state and cost are formed afterwards by the whole team
+// (finish_block), so the per-step work on the tracing thread stays small.
 template <class C>
 struct Tracer {
     using unit_t = typename C::unit_t;
     long long b;        // block being traced, -1 when idle
     const unit_t* bp;   // its backpointers
+    uint16_t* path;     // its states s_1..s_T
     uint32_t s;         // s_tau
-    int tau;            // step about to be emitted (T .. 1)
-    double cost;
-    int widx;           // backward bit writer state
-    uint32_t wcur;
-    // loads in flight
-    unit_t unit;
-    float cval, xval, dval;
+    int tau;            // step about to be stored (T .. 1)
+    unit_t unit;        // load in flight
 
-    __device__ __forceinline__ void start(long long blk, uint32_t sT, const unit_t* p, int T, int W)
+    __device__ __forceinline__ void start(long long blk, uint32_t sT, const unit_t* p,
+                                          uint16_t* pth, int T)
     {
         b = blk;
         bp = p;
+        path = pth;
         s = sT;
         tau = T;
-        cost = 0.0;
-        widx = W - 1;
-        wcur = 0;
     }
 
-    __device__ __forceinline__ void issue(const EncodeArgs& a)
+    __device__ __forceinline__ void issue()
     {
-        const int T = a.T;
         if (tau > 1) {  // bp_{tau-1}[s_tau >> k] decides s_{tau-1}
-            const uint32_t u = s >> C::K;
-            const uint32_t g = u >> C::K;
+            const uint32_t g = s >> (2 * C::K);
             unit = bp[(size_t)((tau - 2) / C::SPU) * C::NT + (g % C::NT)];
         }
-        cval = load_codeword(a.cb, a.cb_f16, s);
-        xval = a.x[b * T + tau - 1];
-        dval = a.d ? a.d[b * T + tau - 1] : 1.f;
     }
 
-    // returns true when the block is finished
-    __device__ __forceinline__ bool retire(const EncodeArgs& a)
+    // returns true when the block's path is complete
+    __device__ __forceinline__ bool retire()
     {
-        const double e = (double)xval - (double)cval;
-        cost += (double)dval * e * e;
-        BackwardBitWriter bw(a.bits + b * a.W, 0);
-        bw.idx = widx;
-        bw.cur = wcur;
-        bw.put(tau, C::K, s & (C::H - 1));
-        if (tau > 1) {
-            const uint32_t u = s >> C::K;
-            const uint32_t g = u >> C::K, j = u & (C::H - 1);
-            const int off = ((tau - 2) % C::SPU) * C::REC_BITS + (int)((g / C::NT) * C::H + j) * C::K;
-            const uint32_t h = (uint32_t)(unit >> off) & (C::H - 1);
-            s = (h << C::LK) | u;
-            widx = bw.idx;
-            wcur = bw.cur;
-            --tau;
-            return false;
-        }
-        bw.finish();
-        a.start_state[b] = s >> C::K;
-        a.path_cost[b] = (float)cost;
-        return true;
+        path[tau - 1] = (uint16_t)s;
+        if (tau == 1) return true;
+        const uint32_t u = s >> C::K;
+        const uint32_t g = u >> C::K, j = u & (C::H - 1);
+        const int q = (int)((g / C::NT) * C::H + j);  // position of u among its thread's
+        const int off = ((tau - 2) % C::SPU) * C::REC_BITS + (C::P - 1 - q);
+        uint32_t h = 0;
+#pragma unroll
+        for (int l = 0; l < C::K; ++l) h = (h << 1) | ((uint32_t)(unit >> (off + l * C::P)) & 1u);
+        s = (h << C::LK) | u;
+        --tau;
+        return false;
     }
 };
+
+// Sum of v over a team; the team's thread 0 gets the total.  Called by all
+// threads of the CTA (it contains __syncthreads for multi-warp teams).
+template <class C>
+__device__ __forceinline__ double team_sum(double v, double* redd, int m, int tid)
+{
+    if constexpr (C::NT >= 32) {
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if ((threadIdx.x & 31) == 0) redd[threadIdx.x >> 5] = v;
+        __syncthreads();
+        double r = 0.0;
+        if (tid == 0) {
+            const int w0 = (m * C::NT) >> 5;
+            for (int w = 0; w < C::NT / 32; ++w) r += redd[w0 + w];
+        }
+        __syncthreads();
+        return r;
+    } else {
+#pragma unroll
+        for (int o = C::NT / 2; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        return v;
+    }
+}
+
+// Outputs of one traced block, formed by its whole team from the stored path:
+// packed symbols (stream bit p is bit 31 - p mod 32 of word p / 32, symbol t at
+// bits [(t-1)k, tk), most significant first, zero padding), the canonical start
+// state s_1 >> k, and the cost sum_t d_t (x_t - c[s_t])^2 accumulated in fp64.
+// All threads of the CTA call it; b < 0 marks a team with nothing to finish.
+template <class C>
+__device__ __forceinline__ void finish_block(const EncodeArgs& a, long long b,
+                                             const uint16_t* __restrict__ path, double* redd,
+                                             int m, int tid)
+{
+    const int T = a.T;
+    double acc = 0.0;
+    if (b >= 0) {
+        const float* xb = a.x + b * T;
+        const float* db = a.d ? a.d + b * T : nullptr;
+        for (int t = tid; t < T; t += C::NT) {
+            const double e = (double)xb[t] - (double)load_codeword(a.cb, a.cb_f16, path[t]);
+            acc += (double)(db ? db[t] : 1.f) * e * e;
+        }
+        const int nbits = T * C::K;
+        for (int w = tid; w < a.W; w += C::NT) {
+            uint32_t word = 0;
+            for (int i = 0; i < 32; ++i) {
+                const int p = 32 * w + i;
+                if (p >= nbits) break;
+                const uint32_t sym = path[p / C::K] & (C::H - 1);
+                word |= ((sym >> (C::K - 1 - p % C::K)) & 1u) << (31 - i);
+            }
+            a.bits[b * a.W + w] = word;
+        }
+    }
+    const double total = team_sum<C>(acc, redd, m, tid);
+    if (b >= 0 && tid == 0) {
+        a.start_state[b] = (uint32_t)path[0] >> C::K;
+        a.path_cost[b] = (float)total;
+    }
+}
+
+// Maximum of v over a team (every team thread gets it).  Called by all threads.
+template <class C>
+__device__ __forceinline__ float team_max(float v, float* redv, int m)
+{
+    if constexpr (C::NT >= 32) {
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+        if ((threadIdx.x & 31) == 0) redv[threadIdx.x >> 5] = v;
+        __syncthreads();
+        const int w0 = (m * C::NT) >> 5;
+        float r = redv[w0];
+        for (int w = 1; w < C::NT / 32; ++w) r = fmaxf(r, redv[w0 + w]);
+        __syncthreads();
+        return r;
+    } else {
+#pragma unroll
+        for (int o = C::NT / 2; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+        return v;
+    }
+}
 
 template <class C, bool WEIGHTED>
 __global__ void __launch_bounds__(C::NTHREADS, 1) acs_grouped_kernel(EncodeArgs a)
@@ -308,7 +407,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1) acs_grouped_kernel(EncodeArgs 
     float2* stage_all = reinterpret_cast<float2*>(Mall + C::NTEAM * 2 * C::NU);
     float* redv = reinterpret_cast<float*>(stage_all + C::NTEAM * C::TCHUNK);
     uint32_t* reds = reinterpret_cast<uint32_t*>(redv + C::NCOMP / 32);
-    uint32_t* fin_state = reds + C::NCOMP / 32;  // [NTEAM]
+    double* redd = reinterpret_cast<double*>(reds + C::NCOMP / 32);  // 8-byte aligned
 
     const int T = a.T;
     const long long nb = a.n_blocks;
@@ -323,6 +422,8 @@ __global__ void __launch_bounds__(C::NTHREADS, 1) acs_grouped_kernel(EncodeArgs 
     const bool tracer = tid == 0;
     float* Mteam = Mall + m * 2 * C::NU;
     float2* stage = stage_all + m * C::TCHUNK;
+    uint16_t* path = reinterpret_cast<uint16_t*>(slot + 2 * C::NTEAM * team_bytes +
+                                                 (size_t)m * C::path_bytes(T));
     Codewords<C, C::CB16> cw;
     cw.load(a.cb, a.cb_f16, tid);
     Tracer<C> tr;
@@ -335,6 +436,13 @@ __global__ void __launch_bounds__(C::NTHREADS, 1) acs_grouped_kernel(EncodeArgs 
         unit_t* bp = reinterpret_cast<unit_t*>(slot + (size_t)(par * C::NTEAM + m) * team_bytes);
         const float* xb = a.x + (valid ? b : 0) * T;
         const float* db = a.d ? a.d + (valid ? b : 0) * T : nullptr;
+        float dfloor = 0.f;
+        if constexpr (C::CB16 && WEIGHTED) {
+            float dm = 0.f;
+            if (valid)
+                for (int q = tid; q < T; q += C::NT) dm = fmaxf(dm, db ? db[q] : 1.f);
+            dfloor = fmaxf(team_max<C>(dm, redv, m) * 0x1p-60f, 1.17549435e-38f);
+        }
         unit_t acc = 0;
         float bestv = __int_as_float(0x7f800000);  // +inf
         uint32_t bests = 0xffffffffu;
@@ -345,9 +453,15 @@ __global__ void __launch_bounds__(C::NTHREADS, 1) acs_grouped_kernel(EncodeArgs 
                 if (valid) {
                     for (int q = tid; q < C::TCHUNK && t + q <= T; q += C::NT) {
                         const float xv = xb[t - 1 + q];
-                        const float dv = WEIGHTED ? db[t - 1 + q] : 1.f;
+                        const float dv = (WEIGHTED && db) ? db[t - 1 + q] : 1.f;
                         if constexpr (C::CB16) {
-                            stage[q] = make_float2(-xv, dv);
+                            float r = 1.f;  // d_{t-1} / d_t, applied to the metrics read at step t
+                            if (WEIGHTED) {
+                                const float dc = fmaxf(dv, dfloor);
+                                const float dp = (t - 1 + q) > 0 ? fmaxf(db ? db[t - 2 + q] : 1.f, dfloor) : dc;
+                                r = dp / dc;
+                            }
+                            stage[q] = make_float2(-xv, r);
                         } else {
                             const float sd = WEIGHTED ? sqrtf(dv) : 1.f;
                             stage[q] = make_float2(-sd, sd * xv);
@@ -357,27 +471,25 @@ __global__ void __launch_bounds__(C::NTHREADS, 1) acs_grouped_kernel(EncodeArgs 
                 __syncthreads();
             }
             const bool tracing = tracer && tr.b >= 0;
-            if (tracing) tr.issue(a);
+            if (tracing) tr.issue();
             if (valid) {
                 const float2 ax = stage[tc];
                 const float* Mp = Mteam + ((t - 1) & 1) * C::NU;
                 float* Mn = Mteam + (t & 1) * C::NU;
-                uint32_t lo, hi;
+                uint32_t planes[C::K];
                 if (t == T) {
                     if (t == 1)
-                        acs_step<C, WEIGHTED, true, true>(cw, ax.x, ax.y, Mp, Mn, tid, lo, hi, bestv, bests);
+                        acs_step<C, WEIGHTED, true, true>(cw, ax.x, ax.y, Mp, Mn, tid, planes, bestv, bests);
                     else
-                        acs_step<C, WEIGHTED, false, true>(cw, ax.x, ax.y, Mp, Mn, tid, lo, hi, bestv, bests);
+                        acs_step<C, WEIGHTED, false, true>(cw, ax.x, ax.y, Mp, Mn, tid, planes, bestv, bests);
                 } else {
                     if (t == 1)
-                        acs_step<C, WEIGHTED, true, false>(cw, ax.x, ax.y, Mp, Mn, tid, lo, hi, bestv, bests);
+                        acs_step<C, WEIGHTED, true, false>(cw, ax.x, ax.y, Mp, Mn, tid, planes, bestv, bests);
                     else
-                        acs_step<C, WEIGHTED, false, false>(cw, ax.x, ax.y, Mp, Mn, tid, lo, hi, bestv, bests);
-                    unit_t rec;
-                    if constexpr (C::UNIT_BITS == 64)
-                        rec = ((unit_t)hi << 32) | (unit_t)lo;
-                    else
-                        rec = (unit_t)lo;
+                        acs_step<C, WEIGHTED, false, false>(cw, ax.x, ax.y, Mp, Mn, tid, planes, bestv, bests);
+                    unit_t rec = 0;
+#pragma unroll
+                    for (int l = 0; l < C::K; ++l) rec |= (unit_t)planes[l] << (l * C::P);
                     const int q = (t - 1) % C::SPU;
                     acc |= rec << (q * C::REC_BITS);
                     if (q == C::SPU - 1 || t == T - 1) {
@@ -386,7 +498,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1) acs_grouped_kernel(EncodeArgs 
                     }
                 }
             }
-            if (tracing && tr.retire(a)) tr.b = -1;
+            if (tracing && tr.retire()) tr.b = -1;
             if (t < T) __syncthreads();
         }
 
@@ -419,18 +531,29 @@ __global__ void __launch_bounds__(C::NTHREADS, 1) acs_grouped_kernel(EncodeArgs 
                 keep_best(ov, os, bestv, bests);
             }
         }
+        // the previous round's block was traced during this round's T steps:
+        // its path is complete, the team forms its outputs
+        __syncthreads();
+        if (r > 0) {
+            const long long pb = b - stride;  // this team's block of round r-1 (always valid)
+            finish_block<C>(a, pb, path, redd, m, tid);
+        }
+        __syncthreads();  // path consumed; this round's backpointers visible to the tracer
         // the team's thread 0 holds the final state; its trace runs during the next round
-        if (tracer && valid) tr.start(b, bests, bp, T, a.W);
-        __syncthreads();  // backpointers of this round visible to the tracer; redv reusable
+        if (tracer && valid) tr.start(b, bests, bp, path, T);
     }
     // the last block of each team has no next round to hide behind
     if (tracer && tr.b >= 0) {
         while (true) {
-            tr.issue(a);
-            if (tr.retire(a)) break;
+            tr.issue();
+            if (tr.retire()) break;
         }
     }
-    (void)fin_state;
+    __syncthreads();
+    if (R > 0) {
+        const long long lb = first + (long long)(R - 1) * stride + m;
+        finish_block<C>(a, lb < nb ? lb : -1, path, redd, m, tid);
+    }
 }
 
 template <class C, bool WEIGHTED>
@@ -447,6 +570,10 @@ cudaError_t launch_grouped_w(const EncodeArgs& a, int grid, cudaStream_t stream)
 template <class C>
 cudaError_t launch_grouped(const EncodeArgs& a, int grid, cudaStream_t stream)
 {
+    // The fp16-pair kernels always run the weighted form (an absent d reads as 1,
+    // every ratio d_{t-1}/d_t is then 1): measured faster than a separate
+    // unweighted instantiation, whose schedule came out worse.
+    if constexpr (C::CB16) return launch_grouped_w<C, true>(a, grid, stream);
     return a.d ? launch_grouped_w<C, true>(a, grid, stream) : launch_grouped_w<C, false>(a, grid, stream);
 }
 
