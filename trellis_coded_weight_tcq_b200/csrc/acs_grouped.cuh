@@ -297,10 +297,11 @@ struct Tracer {
         }
     }
 
-    // returns true when the block's path is complete
-    __device__ __forceinline__ bool retire()
+    // returns true when the block's path is complete; every lane running the
+    // tracer holds the same state, thread 0 of the team stores it
+    __device__ __forceinline__ bool retire(bool store)
     {
-        path[tau - 1] = (uint16_t)s;
+        if (store) path[tau - 1] = (uint16_t)s;
         if (tau == 1) return true;
         const uint32_t u = s >> C::K;
         const uint32_t g = u >> C::K, j = u & (C::H - 1);
@@ -419,7 +420,9 @@ __global__ void __launch_bounds__(C::NTHREADS, 1) acs_grouped_kernel(EncodeArgs 
 
     const int m = threadIdx.x / C::NT;    // team
     const int tid = threadIdx.x % C::NT;  // thread within the team
-    const bool tracer = tid == 0;
+    // the team's first warp (or whole sub-warp team) runs the traceback in
+    // lockstep: no divergent branch, the loads of all lanes hit one address
+    const bool tracer = tid < 32;
     float* Mteam = Mall + m * 2 * C::NU;
     float2* stage = stage_all + m * C::TCHUNK;
     uint16_t* path = reinterpret_cast<uint16_t*>(slot + 2 * C::NTEAM * team_bytes +
@@ -447,7 +450,11 @@ __global__ void __launch_bounds__(C::NTHREADS, 1) acs_grouped_kernel(EncodeArgs 
         float bestv = __int_as_float(0x7f800000);  // +inf
         uint32_t bests = 0xffffffffu;
 
-        for (int t = 1; t <= T; ++t) {
+        unit_t* bpw = bp + tid;  // next backpointer record of this thread
+        // one trellis step; FIRST and LAST select the variant
+        auto step = [&](auto first_tag, auto last_tag, int t) {
+            constexpr bool FIRST = decltype(first_tag)::value;
+            constexpr bool LAST = decltype(last_tag)::value;
             const int tc = (t - 1) % C::TCHUNK;
             if (tc == 0) {
                 if (valid) {
@@ -455,13 +462,13 @@ __global__ void __launch_bounds__(C::NTHREADS, 1) acs_grouped_kernel(EncodeArgs 
                         const float xv = xb[t - 1 + q];
                         const float dv = (WEIGHTED && db) ? db[t - 1 + q] : 1.f;
                         if constexpr (C::CB16) {
-                            float r = 1.f;  // d_{t-1} / d_t, applied to the metrics read at step t
+                            float rr = 1.f;  // d_{t-1} / d_t, applied to the metrics read at step t
                             if (WEIGHTED) {
                                 const float dc = fmaxf(dv, dfloor);
                                 const float dp = (t - 1 + q) > 0 ? fmaxf(db ? db[t - 2 + q] : 1.f, dfloor) : dc;
-                                r = dp / dc;
+                                rr = dp / dc;
                             }
-                            stage[q] = make_float2(-xv, r);
+                            stage[q] = make_float2(-xv, rr);
                         } else {
                             const float sd = WEIGHTED ? sqrtf(dv) : 1.f;
                             stage[q] = make_float2(-sd, sd * xv);
@@ -477,29 +484,36 @@ __global__ void __launch_bounds__(C::NTHREADS, 1) acs_grouped_kernel(EncodeArgs 
                 const float* Mp = Mteam + ((t - 1) & 1) * C::NU;
                 float* Mn = Mteam + (t & 1) * C::NU;
                 uint32_t planes[C::K];
-                if (t == T) {
-                    if (t == 1)
-                        acs_step<C, WEIGHTED, true, true>(cw, ax.x, ax.y, Mp, Mn, tid, planes, bestv, bests);
-                    else
-                        acs_step<C, WEIGHTED, false, true>(cw, ax.x, ax.y, Mp, Mn, tid, planes, bestv, bests);
-                } else {
-                    if (t == 1)
-                        acs_step<C, WEIGHTED, true, false>(cw, ax.x, ax.y, Mp, Mn, tid, planes, bestv, bests);
-                    else
-                        acs_step<C, WEIGHTED, false, false>(cw, ax.x, ax.y, Mp, Mn, tid, planes, bestv, bests);
+                acs_step<C, WEIGHTED, FIRST, LAST>(cw, ax.x, ax.y, Mp, Mn, tid, planes, bestv, bests);
+                if constexpr (!LAST) {
                     unit_t rec = 0;
 #pragma unroll
                     for (int l = 0; l < C::K; ++l) rec |= (unit_t)planes[l] << (l * C::P);
-                    const int q = (t - 1) % C::SPU;
-                    acc |= rec << (q * C::REC_BITS);
-                    if (q == C::SPU - 1 || t == T - 1) {
-                        bp[(size_t)((t - 1) / C::SPU) * C::NT + tid] = acc;
-                        acc = 0;
+                    if constexpr (C::SPU == 1) {
+                        *bpw = rec;
+                        bpw += C::NT;
+                    } else {
+                        const int q = (t - 1) % C::SPU;
+                        acc |= rec << (q * C::REC_BITS);
+                        if (q == C::SPU - 1 || t == T - 1) {
+                            *bpw = acc;
+                            bpw += C::NT;
+                            acc = 0;
+                        }
                     }
                 }
             }
-            if (tracing && tr.retire()) tr.b = -1;
-            if (t < T) __syncthreads();
+            if (tracing && tr.retire(tid == 0)) tr.b = -1;
+            if (!LAST) __syncthreads();
+        };
+        using T0 = std::false_type;
+        using T1 = std::true_type;
+        if (T == 1) {
+            step(T1{}, T1{}, 1);
+        } else {
+            step(T1{}, T0{}, 1);
+            for (int t = 2; t < T; ++t) step(T0{}, T0{}, t);
+            step(T0{}, T1{}, T);
         }
 
         // ---- final state of the block: lexicographic (cost, state) minimum over the team
@@ -546,7 +560,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1) acs_grouped_kernel(EncodeArgs 
     if (tracer && tr.b >= 0) {
         while (true) {
             tr.issue();
-            if (tr.retire()) break;
+            if (tr.retire(tid == 0)) break;
         }
     }
     __syncthreads();
@@ -573,8 +587,11 @@ cudaError_t launch_grouped(const EncodeArgs& a, int grid, cudaStream_t stream)
     // The fp16-pair kernels always run the weighted form (an absent d reads as 1,
     // every ratio d_{t-1}/d_t is then 1): measured faster than a separate
     // unweighted instantiation, whose schedule came out worse.
-    if constexpr (C::CB16) return launch_grouped_w<C, true>(a, grid, stream);
-    return a.d ? launch_grouped_w<C, true>(a, grid, stream) : launch_grouped_w<C, false>(a, grid, stream);
+    if constexpr (C::CB16)
+        return launch_grouped_w<C, true>(a, grid, stream);
+    else
+        return a.d ? launch_grouped_w<C, true>(a, grid, stream)
+                   : launch_grouped_w<C, false>(a, grid, stream);
 }
 
 template <class C>
