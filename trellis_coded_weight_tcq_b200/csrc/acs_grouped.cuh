@@ -184,6 +184,25 @@ struct SignTree {
         return fminf(vl, vr);
     }
 };
+// Four candidates: m01 = min(c0, c1) and the three-input m = min(m01, c2, c3)
+// give the minimum without forming min(c2, c3); the top bit is the sign of
+// m - m01 (negative exactly when the right pair holds a strictly smaller
+// value, +0 on a tie, so the left pair wins ties as required).
+template <int OFF>
+struct SignTree<4, OFF> {
+    template <int H, int K>
+    static __device__ __forceinline__ float run(const float (&c)[H], uint32_t (&sb)[K])
+    {
+        const float m01 = fminf(c[OFF], c[OFF + 1]);
+        float m;
+        asm("min.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(m01), "f"(c[OFF + 2]), "f"(c[OFF + 3]));
+        const uint32_t s = __float_as_uint(m - m01);
+        sb[0] = s;
+        sb[1] = mux_sign(s, __float_as_uint(c[OFF + 3] - c[OFF + 2]),
+                         __float_as_uint(c[OFF + 1] - c[OFF]));
+        return m;
+    }
+};
 template <int OFF>
 struct SignTree<2, OFF> {
     template <int H, int K>
