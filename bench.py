@@ -218,15 +218,20 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.current_stream()
     enc_ev = []
 
+    dec_ev = []
+
     def step(record=False):
         if record:
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
             a.record(stream)
         tcq.encode(x, d, cb, L, k, ws, out)
         if record:
             b.record(stream)
             enc_ev.append((a, b))
         tcq.decode(out.bits, out.start_state, cb, L, k, T, y)
+        if record:
+            c.record(stream)
+            dec_ev.append((b, c))
 
     def barrier():
         if world > 1:
@@ -247,10 +252,11 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     ms = t_start.elapsed_time(t_end) / args.steps
     acs_ms = sum(a.elapsed_time(b) for a, b in enc_ev) / len(enc_ev)
+    dec_ms = sum(a.elapsed_time(b) for a, b in dec_ev) / len(dec_ev)
     if world > 1:
-        t = torch.tensor([ms, acs_ms], dtype=torch.float64, device=dev)
+        t = torch.tensor([ms, acs_ms, dec_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, acs_ms = t.tolist()
+        ms, acs_ms, dec_ms = t.tolist()
     gpu_launches = 2 * args.steps  # one encoder kernel + one decoder kernel per step
 
     # ---- end to end through the C ABI from pinned host buffers
@@ -302,6 +308,14 @@ def run_ours(args, rank, world, local_rank):
                       f"({peak_kind} max SM clock); {ALGO_OPS_PER_NODE} ops per trellis node",
         "acs_ms_per_launch": acs_ms,
     }
+    # the decoder, HBM bound: y written (4 B per weight), bits and start states read
+    dec_bytes = wl.weights * 4 + n * W * 4 + n * 4
+    decode_roofline = {
+        "bound": "hbm", "kernel": "decode_kernel", "ms_per_launch": dec_ms,
+        "achieved": dec_bytes / (dec_ms / 1e3) / 1e9, "peak": float(peaks.get("hbm_gbs", 6650.0)),
+        "unit": "GB/s", "frac": dec_bytes / (dec_ms / 1e3) / 1e9 / float(peaks.get("hbm_gbs", 6650.0)),
+        "bytes_per_launch": dec_bytes,
+    }
     cpu_baseline = None
     if pool is not None:
         nb, wall = time_oracle(pool, cores, wl, args.cpu_blocks_per_core)
@@ -320,8 +334,8 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "inputs larger than L2 (x and d are 470 MB per GPU), no flush",
                    "parallelism": f"blocks sharded per GPU (dp{world})"},
         "weights_per_s": world * wl.weights / (ms / 1e3),
-        "encode_ms_per_step": acs_ms, "decode_ms_per_step": ms - acs_ms,
-        "roofline": roofline, "cpu_baseline": cpu_baseline, "e2e": e2e,
+        "encode_ms_per_step": acs_ms, "decode_ms_per_step": dec_ms,
+        "roofline": roofline, "decode_roofline": decode_roofline, "cpu_baseline": cpu_baseline, "e2e": e2e,
         "clocks": clocks.summary(), "gpu_launches": gpu_launches,
     }
     print(json.dumps(line), flush=True)

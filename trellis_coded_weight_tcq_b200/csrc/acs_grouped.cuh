@@ -62,6 +62,9 @@ struct GCfg {
     static constexpr int SPU = UNIT_BITS / REC_BITS;  // steps per stored unit
     static constexpr int NCOMP = NT * NTEAM;
     static constexpr int NTHREADS = NCOMP;
+    // resident CTAs per SM the register allocation must allow: 128 registers
+    // per thread for every configuration (the fp16-pair codewords alone take 64)
+    static constexpr int MINB = NTHREADS >= 512 ? 1 : 512 / NTHREADS;
     static constexpr int TCHUNK = 256;         // steps of (a, xs) staged at a time
     using unit_t = typename std::conditional<UNIT_BITS == 32, uint32_t, unsigned long long>::type;
 
@@ -71,7 +74,6 @@ struct GCfg {
     static_assert(P <= 32, "a bit plane is one 32-bit register");
     static_assert(NCOMP % 32 == 0, "compute threads must be whole warps");
     static_assert(NT >= 32 ? (NT % 32 == 0) : (32 % NT == 0), "teams tile warps");
-    static_assert(NTEAM == 1 || NT <= 32, "multi-team CTAs use sub-warp teams");
 
     // bytes of one team's backpointers for one block, rounded to 256
     static __host__ __device__ size_t team_bytes(int T)
@@ -419,7 +421,7 @@ __device__ __forceinline__ float team_max(float v, float* redv, int m)
 }
 
 template <class C, bool WEIGHTED>
-__global__ void __launch_bounds__(C::NTHREADS, 1) acs_grouped_kernel(EncodeArgs a)
+__global__ void __launch_bounds__(C::NTHREADS, C::MINB) acs_grouped_kernel(EncodeArgs a)
 {
     using unit_t = typename C::unit_t;
     extern __shared__ __align__(16) unsigned char smem[];

@@ -5,11 +5,13 @@
 // the last L bits of (start || stream[0, tk)), so every output is independent:
 // one window extract and one codebook gather, no serial state.
 //
-// One warp per block in flight, each lane four consecutive weights (one
-// 16-byte store when the row allows it).  The codebook is staged once per CTA
-// in shared memory (fp32 if it fits in 64 KiB, else as binary16 when the input
-// is binary16); a binary32 codebook too large for that is gathered through L1.
-// The kernel reads k/8 bytes and writes 4 bytes per weight: HBM bound.
+// Each thread produces four consecutive weights of one block (one 16-byte store
+// when the row allows it); a CTA covers as many whole blocks as its threads
+// span and strides over the rest, so every thread has independent loads in
+// flight.  The codebook is staged once per CTA in shared memory (fp32 if it
+// fits in 64 KiB, else as binary16 when the input is binary16); a binary32
+// codebook too large for that is gathered through L1.  The kernel reads k/8
+// bytes and writes 4 bytes per weight: HBM bound.
 #include "common.cuh"
 
 namespace tcq {
@@ -18,24 +20,7 @@ namespace {
 
 enum TableMode { kTableF32 = 0, kTableF16 = 1, kTableGlobal = 2 };
 
-constexpr int kDecodeThreads = 512;
-
-__device__ __forceinline__ uint32_t state_at(const uint32_t* __restrict__ w, int W, uint32_t start,
-                                             int t, int K, int L)
-{
-    const uint32_t mask = (1u << L) - 1u;
-    const int pend = t * K;  // stream bits consumed through symbol t
-    if (pend >= L) {
-        const int p0 = pend - L;
-        const int wi = p0 >> 5, off = p0 & 31;
-        const unsigned long long hi = w[wi];
-        const unsigned long long lo = (off + L > 32 && wi + 1 < W) ? w[wi + 1] : 0ull;
-        const unsigned long long v = (hi << 32) | lo;
-        return (uint32_t)(v >> (64 - off - L)) & mask;
-    }
-    // fewer than L stream bits so far: the start state supplies the rest
-    return ((start << pend) | (w[0] >> (32 - pend))) & mask;
-}
+constexpr int kDecodeThreads = 1024;
 
 template <int MODE, bool VEC>
 __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a)
@@ -46,44 +31,107 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a)
         float* tab = reinterpret_cast<float*>(dsm);
         for (int i = threadIdx.x; i < n_entries; i += blockDim.x) tab[i] = load_codeword(a.cb, a.cb_f16, i);
     } else if constexpr (MODE == kTableF16) {
-        __half* tab = reinterpret_cast<__half*>(dsm);
+        // 16-byte copies when the source allows (the table size, 2^L entries of 2
+        // bytes, is a multiple of 16 for L >= 3)
         const __half* src = reinterpret_cast<const __half*>(a.cb);
-        for (int i = threadIdx.x; i < n_entries; i += blockDim.x) tab[i] = src[i];
+        if ((reinterpret_cast<uintptr_t>(src) & 15) == 0 && n_entries % 8 == 0) {
+            const uint4* s4 = reinterpret_cast<const uint4*>(src);
+            uint4* d4 = reinterpret_cast<uint4*>(dsm);
+            for (int i = threadIdx.x; i < n_entries / 8; i += blockDim.x) d4[i] = s4[i];
+        } else {
+            __half* tab = reinterpret_cast<__half*>(dsm);
+            for (int i = threadIdx.x; i < n_entries; i += blockDim.x) tab[i] = src[i];
+        }
     }
     __syncthreads();
 
     const int T = a.T, K = a.K, L = a.L, W = a.W;
+    const uint32_t mask = (1u << L) - 1u;
     const int Q = (T + 3) >> 2;  // quads per block
-    const int lane = threadIdx.x & 31;
-    const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
-    for (long long b = warp; b < a.n_blocks; b += nwarps) {
-        const uint32_t* wb = a.bits + b * W;
-        const uint32_t start = a.start_state[b];
-        float* yb = a.y + b * T;
-        for (int q = lane; q < Q; q += 32) {
+    const bool qpow2 = (Q & (Q - 1)) == 0;
+    const int qshift = __ffs(Q) - 1;
+    const int per_iter = blockDim.x >= Q ? (int)blockDim.x / Q : 1;  // whole blocks per CTA pass
+    const int span = per_iter * Q;  // quads of one pass (i in [0, span) covers per_iter blocks)
+    auto lookup = [&](uint32_t s) -> float {
+        if constexpr (MODE == kTableF32)
+            return reinterpret_cast<const float*>(dsm)[s];
+        else if constexpr (MODE == kTableF16)
+            return __half2float(reinterpret_cast<const __half*>(dsm)[s]);
+        else
+            return load_codeword(a.cb, a.cb_f16, s);
+    };
+    // Stream word -1 is the start state itself: stream bit p < 0 is bit -p-1 of
+    // start, so s_t is the L-bit window ending at stream bit t k for every t,
+    // and each thread's four windows [p0 + e k, p0 + e k + L), p0 = (4q+1)k - L
+    // >= k - L > -32, lie inside one 64-bit read of words (p0 >> 5, +1).
+    constexpr int UNROLL = 4;
+    struct Frag {
+        unsigned long long win[UNROLL];
+        int off[UNROLL];
+        int q[UNROLL];
+        long long b[UNROLL];
+    };
+    auto fetch = [&](Frag& f, long long b0, int i0) {
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+            const int i = i0 + u * span;
+            const int bl = qpow2 ? (i >> qshift) : i / Q;
+            const int q = i - bl * Q;
+            const long long b = b0 + bl;
+            f.q[u] = q;
+            f.b[u] = b;
+            f.win[u] = 0ull;
+            const int p0 = (4 * q + 1) * K - L;
+            f.off[u] = p0 & 31;
+            if (b < a.n_blocks) {
+                const uint32_t* wb = a.bits + b * W;
+                const int wi = p0 >> 5;  // -1 for the first windows
+                const unsigned long long hi = wi < 0 ? a.start_state[b] : wb[wi];
+                const unsigned long long lo = wi + 1 < W ? wb[wi + 1] : 0ull;
+                f.win[u] = (hi << 32) | lo;
+            }
+        }
+    };
+    auto emit = [&](const Frag& f) {
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+            const long long b = f.b[u];
+            if (b >= a.n_blocks) continue;
+            const int q = f.q[u];
             float v[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int t = 4 * q + e + 1;
-                float val = 0.f;
-                if (t <= T) {
-                    const uint32_t s = state_at(wb, W, start, t, K, L);
-                    if constexpr (MODE == kTableF32)
-                        val = reinterpret_cast<const float*>(dsm)[s];
-                    else if constexpr (MODE == kTableF16)
-                        val = __half2float(reinterpret_cast<const __half*>(dsm)[s]);
-                    else
-                        val = load_codeword(a.cb, a.cb_f16, s);
-                }
-                v[e] = val;
-            }
+            for (int e = 0; e < 4; ++e)
+                v[e] = lookup((uint32_t)(f.win[u] >> (64 - f.off[u] - e * K - L)) & mask);
+            float* yb = a.y + b * T;
             if constexpr (VEC) {
-                *reinterpret_cast<float4*>(yb + 4 * q) = make_float4(v[0], v[1], v[2], v[3]);
+                __stcs(reinterpret_cast<float4*>(yb + 4 * q), make_float4(v[0], v[1], v[2], v[3]));
             } else {
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
                     if (4 * q + e < T) yb[4 * q + e] = v[e];
+            }
+        }
+    };
+    const int blocks_per_pass = per_iter * UNROLL;
+    const long long stride = (long long)gridDim.x * blocks_per_pass;
+    const long long first = (long long)blockIdx.x * blocks_per_pass;
+    if (span <= (int)blockDim.x) {
+        // one fragment per thread per pass; the next pass's loads are issued
+        // before the current pass's lookups and stores
+        if ((int)threadIdx.x >= span) return;
+        Frag cur, nxt;
+        if (first < a.n_blocks) fetch(cur, first, threadIdx.x);
+        for (long long b0 = first; b0 < a.n_blocks; b0 += stride) {
+            if (b0 + stride < a.n_blocks) fetch(nxt, b0 + stride, threadIdx.x);
+            emit(cur);
+            cur = nxt;
+        }
+    } else {  // blocks longer than 4 * blockDim weights
+        for (long long b0 = first; b0 < a.n_blocks; b0 += stride) {
+            for (int i0 = threadIdx.x; i0 < span; i0 += blockDim.x) {
+                Frag f;
+                fetch(f, b0, i0);
+                emit(f);
             }
         }
     }
@@ -116,11 +164,11 @@ cudaError_t launch_decode(const DecodeArgs& a, int num_sms, cudaStream_t stream)
         mode = kTableGlobal;
         smem = 0;
     }
-    // warps in flight: one per block, capped at what the SMs hold
-    const long long warps_needed = a.n_blocks;
-    const int per_cta = kDecodeThreads / 32;
-    long long grid = (warps_needed + per_cta - 1) / per_cta;
-    const int ctas_per_sm = smem > 100 * 1024 ? 1 : (smem > 64 * 1024 ? 2 : 4);
+    // CTAs: enough to cover every block once, capped at what the SMs hold
+    const int Q = (a.T + 3) / 4;
+    const long long per_cta = 4 * (kDecodeThreads >= Q ? kDecodeThreads / Q : 1);
+    long long grid = (a.n_blocks + per_cta - 1) / per_cta;
+    const int ctas_per_sm = smem > 100 * 1024 ? 1 : 2;
     const long long cap = (long long)num_sms * ctas_per_sm;
     if (grid > cap) grid = cap;
     if (grid < 1) grid = 1;
