@@ -200,7 +200,9 @@ def run_ours(args, rank, world, local_rank):
         dist.init_process_group("nccl", device_id=dev,
                                 timeout=__import__("datetime").timedelta(seconds=300))
 
-    wl = workloads.NAMED[args.workload](rank)
+    from trellis_coded_weight_tcq_b200.dist import max_over_ranks, workload_for_rank
+
+    wl = workload_for_rank(args.workload, rank)
     if args.blocks and args.blocks < wl.n_blocks:
         wl.x = np.ascontiguousarray(wl.x[:args.blocks])
         wl.d = None if wl.d is None else np.ascontiguousarray(wl.d[:args.blocks])
@@ -253,10 +255,7 @@ def run_ours(args, rank, world, local_rank):
     ms = t_start.elapsed_time(t_end) / args.steps
     acs_ms = sum(a.elapsed_time(b) for a, b in enc_ev) / len(enc_ev)
     dec_ms = sum(a.elapsed_time(b) for a, b in dec_ev) / len(dec_ev)
-    if world > 1:
-        t = torch.tensor([ms, acs_ms, dec_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, acs_ms, dec_ms = t.tolist()
+    ms, acs_ms, dec_ms = max_over_ranks([ms, acs_ms, dec_ms], dev)
     gpu_launches = 2 * args.steps  # one encoder kernel + one decoder kernel per step
 
     # ---- end to end through the C ABI from pinned host buffers
@@ -276,11 +275,7 @@ def run_ours(args, rank, world, local_rank):
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        e2e_ms = e0.elapsed_time(e1) / args.steps
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = t.item()
+        e2e_ms = max_over_ranks([e0.elapsed_time(e1) / args.steps], dev)[0]
         e2e = {"value": world * wl.nodes / (e2e_ms / 1e3), "unit": "nodes/s",
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": pipe.h2d_bytes(),
                "d2h_bytes_per_step": pipe.d2h_bytes()}
