@@ -140,6 +140,41 @@ def time_oracle(pool, cores, wl, blocks_per_core: int):
     return n, wall
 
 
+def peaks_ops() -> float:
+    peaks, _ = _peaks()
+    return SMS * LANES_PER_SM * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
+
+
+def time_workload(name, dev, tcq, workloads, peak_ops, steps=3):
+    """Encode and decode timing of one named workload (1 warm-up, best of `steps`)."""
+    import torch
+
+    wl = workloads.NAMED[name](0)
+    x = torch.from_numpy(wl.x).to(dev)
+    d = None if wl.d is None else torch.from_numpy(wl.d).to(dev)
+    cb = torch.from_numpy(wl.codebook).to(dev)
+    ws = tcq.Workspace(wl.L, wl.k, wl.T, wl.n_blocks, tcq.cb_dtype_of(cb), dev)
+    out = tcq.encode(x, d, cb, wl.L, wl.k, ws)
+    y = tcq.decode(out.bits, out.start_state, cb, wl.L, wl.k, wl.T)
+    enc, dec = [], []
+    for _ in range(steps):
+        a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        a.record()
+        tcq.encode(x, d, cb, wl.L, wl.k, ws, out)
+        b.record()
+        tcq.decode(out.bits, out.start_state, cb, wl.L, wl.k, wl.T, y)
+        c.record()
+        enc.append((a, b))
+        dec.append((b, c))
+    torch.cuda.synchronize()
+    e_ms = min(a.elapsed_time(b) for a, b in enc)
+    d_ms = min(a.elapsed_time(b) for a, b in dec)
+    return {"workload": wl.name, "nodes_per_s": wl.nodes / (e_ms / 1e3),
+            "weights_per_s": wl.weights / (e_ms / 1e3), "encode_ms": e_ms, "decode_ms": d_ms,
+            "alu_frac": wl.nodes * ALGO_OPS_PER_NODE / (e_ms / 1e3) / peak_ops,
+            "kernel": tcq.tcq_encode_path(wl.L, wl.k, tcq.cb_dtype_of(cb))}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -208,6 +243,7 @@ def run_ours(args, rank, world, local_rank):
         wl.d = None if wl.d is None else np.ascontiguousarray(wl.d[:args.blocks])
         wl.name += f"_first{args.blocks}blocks"
     L, k, T, n = wl.L, wl.k, wl.T, wl.n_blocks
+    weighted = wl.d is not None
     x = torch.from_numpy(wl.x).to(dev)
     d = None if wl.d is None else torch.from_numpy(wl.d).to(dev)
     cb = torch.from_numpy(wl.codebook).to(dev)
@@ -256,7 +292,36 @@ def run_ours(args, rank, world, local_rank):
     acs_ms = sum(a.elapsed_time(b) for a, b in enc_ev) / len(enc_ev)
     dec_ms = sum(a.elapsed_time(b) for a, b in dec_ev) / len(dec_ev)
     ms, acs_ms, dec_ms = max_over_ranks([ms, acs_ms, dec_ms], dev)
+    cost_last = out.path_cost.cpu().numpy()
     gpu_launches = 2 * args.steps  # one encoder kernel + one decoder kernel per step
+
+    # ---- decode-in-matvec on the encoded matrix (one row of the matrix per
+    # block row: rows = blocks * T / cols)
+    gemv = None
+    mat = wl.meta.get("matrix")
+    if mat and rank == 0:
+        rows_m, cols_m = int(mat[0]), int(mat[1])
+        xv = torch.randn(cols_m, device=dev)
+        scale = torch.ones(n, device=dev)
+        ym = torch.empty(rows_m, device=dev)
+        for _ in range(3):
+            tcq.gemv(out.bits, out.start_state, scale, cb, L, k, T, rows_m, cols_m, xv, ym)
+        g_ev = []
+        for _ in range(10):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            tcq.gemv(out.bits, out.start_state, scale, cb, L, k, T, rows_m, cols_m, xv, ym)
+            b.record(stream)
+            g_ev.append((a, b))
+        torch.cuda.synchronize()
+        g_ms = min(a.elapsed_time(b) for a, b in g_ev)
+        g_bytes = n * W * 4 + n * 4 + n * 4 + cols_m * 4 + rows_m * 4
+        peaks_g, _ = _peaks()
+        gemv = {"rows": rows_m, "cols": cols_m, "ms": g_ms,
+                "weights_per_s": rows_m * cols_m / (g_ms / 1e3),
+                "hbm_gbs": g_bytes / (g_ms / 1e3) / 1e9,
+                "hbm_frac": g_bytes / (g_ms / 1e3) / 1e9 / float(peaks_g.get("hbm_gbs", 6650.0)),
+                "bytes": g_bytes}
 
     # ---- end to end through the C ABI from pinned host buffers
     e2e = None
@@ -281,8 +346,21 @@ def run_ours(args, rank, world, local_rank):
                "d2h_bytes_per_step": pipe.d2h_bytes()}
         del pipe
 
+    # ---- the other named workloads: encode + decode throughput, short runs
+    per_workload = []
+    if rank == 0 and world == 1 and not args.no_per_workload:
+        del x, d, y, ws, out
+        torch.cuda.empty_cache()
+        for name in [n for n in ("tiny", "l12", "qtip", "heavy", "mlp") if n != args.workload]:
+            per_workload.append(time_workload(name, dev, tcq, workloads, peaks_ops()))
+        per_workload.append({"workload": wl.name, "nodes_per_s": wl.nodes / (acs_ms / 1e3),
+                             "weights_per_s": wl.weights / (acs_ms / 1e3), "encode_ms": acs_ms,
+                             "decode_ms": dec_ms,
+                             "alu_frac": wl.nodes * ALGO_OPS_PER_NODE / (acs_ms / 1e3) / peaks_ops(),
+                             "kernel": tcq.tcq_encode_path(L, k, tcq.cb_dtype_of(cb))})
+
     # sanity: the last step's result is a valid encode of the workload (cheap host check)
-    cost_h = out.path_cost.cpu().numpy()
+    cost_h = cost_last
     assert np.all(np.isfinite(cost_h)) and np.all(cost_h >= 0)
 
     if world > 1:
@@ -325,12 +403,13 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
         "config": {"workload": wl.name, "L": L, "k": k, "T": T, "n_blocks": n,
-                   "codebook": str(wl.codebook.dtype), "weighted": d is not None,
+                   "codebook": str(wl.codebook.dtype), "weighted": weighted,
                    "l2": "inputs larger than L2 (x and d are 470 MB per GPU), no flush",
                    "parallelism": f"blocks sharded per GPU (dp{world})"},
         "weights_per_s": world * wl.weights / (ms / 1e3),
         "encode_ms_per_step": acs_ms, "decode_ms_per_step": dec_ms,
         "roofline": roofline, "decode_roofline": decode_roofline, "cpu_baseline": cpu_baseline, "e2e": e2e,
+        "per_workload": per_workload, "gemv": gemv,
         "clocks": clocks.summary(), "gpu_launches": gpu_launches,
     }
     print(json.dumps(line), flush=True)
@@ -345,6 +424,8 @@ def main():
     ap.add_argument("--workload", choices=["mlp", "qtip", "heavy", "l12", "tiny"], default="mlp")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip the short encode/decode timing of the other named workloads")
     ap.add_argument("--cpu-blocks-per-core", type=int, default=4)
     ap.add_argument("--blocks", type=int, default=0,
                     help="encode only the first N blocks of the workload (a smaller profiling "

@@ -12,7 +12,7 @@
  *     trellis-coded quantization and the Viterbi search): the state picks the
  *     coset for the next weight, the written bits pick the value and set the
  *     next state; the encoder is the Viterbi dynamic program, linear in length;
- *     decoding is "read bits, update state, look up values".
+ *     decoding walks the bits, advancing the state and fetching the codeword.
  *   - CurveTQ abstract (aggregator page for paper 2610.09212): the Viterbi
  *     branch metric weighted per coordinate by the diagonal d_j of the
  *     Hessian's LDL factor, and a start state stored per coding block.
@@ -117,7 +117,7 @@ tcq_status tcq_encode(const float* x, const float* d, const void* codebook, tcq_
                       tcq_stream_t stream);
 
 /*
- * Decode (the 2-bit post's "read bits, update state, look up values"; QTIP's
+ * Decode (the 2-bit post's state-tracking table-lookup decoder; QTIP's
  * stateful bitshift decoder): y[b, t-1] = c[s_t] with s_t the last L bits of
  * (start_state[b] || stream[0, tk)).  Bit-exact: y is the exact fp32 widening
  * of the codebook entry.
@@ -131,6 +131,30 @@ tcq_status tcq_encode(const float* x, const float* d, const void* codebook, tcq_
 tcq_status tcq_decode(const uint32_t* bits, const uint32_t* start_state, const void* codebook,
                       tcq_dtype cb_dtype, int L, int k, int T, int64_t n_blocks, float* y,
                       tcq_stream_t stream);
+
+/*
+ * Matrix-vector product with a trellis-coded matrix, decoding on the fly (the
+ * 2-bit post's Pingala-8 section: the decoder, which advances the state from the
+ * bits and fetches each codeword, runs inside the matrix-vector product, so the
+ * weights are never materialised).
+ *
+ * The rows x cols matrix is stored as rows * (cols / T) coding blocks of T
+ * consecutive columns, block (r, j) = r * (cols / T) + j covering columns
+ * [jT, jT + T) of row r -- what tcq_encode returns for the row-major matrix
+ * viewed as [rows * cols / T, T] -- each with optional fp32 scale:
+ *     y[r] = sum_j scale[r, j] * sum_t c[s_{r,j,t}] * x[jT + t]
+ * accumulated in fp32.
+ *
+ *   bits, start_state  as tcq_decode, for rows * (cols / T) blocks.
+ *   scale              fp32 [rows * cols / T] or NULL (all 1).
+ *   x                  fp32 [cols], 16-byte aligned.   y  out: fp32 [rows].
+ * Requires T % 4 == 0 and cols % T == 0 (else TCQ_ERR_UNSUPPORTED /
+ * TCQ_ERR_INVALID_ARG), and a binary16 codebook when L >= 15 (the table lives
+ * in shared memory).  rows == 0 is a no-op.
+ */
+tcq_status tcq_gemv(const uint32_t* bits, const uint32_t* start_state, const float* scale,
+                    const void* codebook, tcq_dtype cb_dtype, int L, int k, int T, int64_t rows,
+                    int64_t cols, const float* x, float* y, tcq_stream_t stream);
 
 /* Static, human-readable name of a status code. */
 const char* tcq_status_string(tcq_status status);

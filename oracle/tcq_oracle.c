@@ -12,8 +12,8 @@
  *     trellis: "QTIP: Quantization with Trellises and Incoherence Processing"
  *     (abstract).  The state is the last L bits written, k new bits are shifted
  *     in per weight, and the reconstruction is a codebook lookup by state.
- *   - The search is the Viterbi dynamic program that keeps the cheapest path
- *     into every state, linear in length: "How do you fit a 4B LLM in 1.24 GB:
+ *   - The search is the Viterbi dynamic program that retains, per state, the
+ *     lowest-cost path reaching it, with work linear in the block length: "How do you fit a 4B LLM in 1.24 GB:
  *     trellis-coded 2-bit" (section on trellis memory and the Viterbi search).
  *   - The branch metric is the per-coordinate weighted error d_j (x_j - c)^2,
  *     with d_j the diagonal of the Hessian's LDL factor, and a start state is
@@ -264,5 +264,39 @@ int oracle_greedy(const double* x, const double* d, const double* cb, int L, int
         }
         cost[blk] = acc;
     }
+    return ORACLE_OK;
+}
+
+/*
+ * Matrix-vector product with a trellis-coded matrix: rows x cols weights stored
+ * as rows * (cols / T) coding blocks of T consecutive columns (block (r, j) =
+ * index r * (cols/T) + j covers columns [jT, jT + T) of row r), each scaled by
+ * scale[block] (NULL: 1).  y[r] = sum_j scale[r, j] * sum_t c[s_{r,j,t}] * x[jT + t],
+ * i.e. decode every block, then the dense product, accumulated in fp64.
+ */
+int oracle_gemv(const uint32_t* bits, const uint32_t* start_state, const double* scale,
+                const double* cb, int L, int k, int T, int64_t rows, int64_t cols,
+                const double* x, double* y)
+{
+    if (!valid_shape(L, k, T) || rows < 0 || cols < 0 || cols % T != 0) return ORACLE_EINVAL;
+    if (rows == 0) return ORACLE_OK;
+    if (!bits || !start_state || !cb || !x || !y) return ORACLE_EINVAL;
+    const int64_t nb = cols / T;
+    const int W = oracle_words_per_block(k, T);
+    double* vals = (double*)malloc(sizeof(double) * (size_t)T);
+    if (!vals) return ORACLE_ENOMEM;
+    for (int64_t r = 0; r < rows; ++r) {
+        double acc = 0.0;
+        for (int64_t j = 0; j < nb; ++j) {
+            const int64_t b = r * nb + j;
+            int rc = oracle_decode(bits + b * W, start_state + b, cb, L, k, T, 1, vals);
+            if (rc != ORACLE_OK) { free(vals); return rc; }
+            double part = 0.0;
+            for (int t = 0; t < T; ++t) part += vals[t] * x[j * T + t];
+            acc += (scale ? scale[b] : 1.0) * part;
+        }
+        y[r] = acc;
+    }
+    free(vals);
     return ORACLE_OK;
 }

@@ -48,6 +48,8 @@ def _load():
         lib.oracle_path_cost.restype = ci
         lib.oracle_greedy.argtypes = [dp, dp, dp, ci, ci, ci, i64, up, up, dp]
         lib.oracle_greedy.restype = ci
+        lib.oracle_gemv.argtypes = [up, up, dp, dp, ci, ci, ci, i64, i64, dp, dp]
+        lib.oracle_gemv.restype = ci
         _lib = lib
     return _lib
 
@@ -160,3 +162,21 @@ def oracle_greedy(x, d, codebook, L: int, k: int, start_state):
     if rc != 0:
         raise ValueError(f"oracle_greedy failed with code {rc}")
     return bits, cost
+
+
+def oracle_gemv(bits, start_state, scale, codebook, L: int, k: int, T: int, rows: int, cols: int, x):
+    """y = (decoded, block-scaled matrix) @ x in fp64; blocks row-major [rows, cols/T]."""
+    bits = _u32(bits).reshape(-1)
+    start = _u32(start_state).reshape(-1)
+    sc = None if scale is None else _f64(scale).reshape(-1)
+    cb = _f64(codebook).reshape(-1)
+    xv = _f64(x).reshape(-1)
+    y = np.zeros(rows, dtype=np.float64)
+    rc = _load().oracle_gemv(
+        _ptr(bits, ctypes.c_uint32), _ptr(start, ctypes.c_uint32), _ptr(sc, ctypes.c_double),
+        _ptr(cb, ctypes.c_double), L, k, T, rows, cols, _ptr(xv, ctypes.c_double),
+        _ptr(y, ctypes.c_double),
+    )
+    if rc != 0:
+        raise ValueError(f"oracle_gemv failed with code {rc}")
+    return y

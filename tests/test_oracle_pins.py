@@ -235,3 +235,33 @@ def test_rejects_bad_shapes():
         oracle_encode(np.zeros((1, 4)), None, np.zeros(8), 3, 4)  # k > L
     with pytest.raises(ValueError):
         oracle_encode(np.zeros((1, 4)), None, np.zeros(7), 3, 1)  # codebook size
+
+
+# --------------------------------------------------------------------------
+# decode-in-matvec: the oracle GEMV is decode followed by a dense product
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("L,k,T,rows,nb", [(4, 2, 8, 5, 3), (6, 3, 4, 3, 4), (8, 2, 16, 4, 2)])
+@pytest.mark.parametrize("scaled", [False, True])
+def test_oracle_gemv_is_decode_then_dense_product(L, k, T, rows, nb, scaled):
+    from oracle import oracle_gemv
+
+    rng = _rng(L * 13 + k + T)
+    cols = nb * T
+    W = oracle_words_per_block(k, T)
+    n = rows * nb
+    bits = rng.integers(0, 2**32, size=(n, W), dtype=np.uint64).astype(np.uint32)
+    used = T * k - 32 * (W - 1)
+    if used < 32:
+        bits[:, -1] &= np.uint32(((1 << used) - 1) << (32 - used))
+    start = rng.integers(0, 2**32, size=n, dtype=np.uint64).astype(np.uint32)
+    cb = rng.standard_normal(1 << L)
+    scale = rng.lognormal(0.0, 0.5, n) if scaled else None
+    x = rng.standard_normal(cols)
+    dense = np.zeros((rows, cols))
+    for r in range(rows):
+        for j in range(nb):
+            b = r * nb + j
+            vals = decode_window(bits[b], int(start[b]), cb, L, k, T)
+            dense[r, j * T:(j + 1) * T] = vals * (scale[b] if scaled else 1.0)
+    y = oracle_gemv(bits, start, scale, cb, L, k, T, rows, cols, x)
+    np.testing.assert_allclose(y, dense @ x, rtol=1e-12, atol=1e-12)

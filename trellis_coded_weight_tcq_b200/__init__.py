@@ -11,11 +11,13 @@ from .tcq import (  # noqa: F401
     Workspace,
     decode,
     encode,
+    gemv,
     load_library,
     tcq_decode,
     tcq_encode,
     tcq_encode_path,
     tcq_encode_workspace_bytes,
+    tcq_gemv,
     tcq_status_string,
     tcq_words_per_block,
 )

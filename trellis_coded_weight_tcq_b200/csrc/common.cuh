@@ -36,6 +36,18 @@ struct DecodeArgs {
     float* y;
 };
 
+struct GemvArgs {
+    const uint32_t* bits;         // [rows * cols / T, W]
+    const uint32_t* start_state;  // [rows * cols / T]
+    const float* scale;           // [rows * cols / T] or nullptr
+    const void* cb;
+    int cb_f16;
+    int L, K, T, W;
+    long long rows, cols;
+    const float* x;               // [cols]
+    float* y;                     // [rows]
+};
+
 // One codebook entry, widened exactly to fp32.
 __device__ __forceinline__ float load_codeword(const void* cb, int f16, uint32_t s)
 {
@@ -112,5 +124,6 @@ const EncodeKernelInfo* find_grouped_kernel(int L, int K, int cb_f16);
 const EncodeKernelInfo* generic_kernel_info(int L, int K);
 
 cudaError_t launch_decode(const DecodeArgs& a, int num_sms, cudaStream_t stream);
+cudaError_t launch_gemv(const GemvArgs& a, int num_sms, cudaStream_t stream);
 
 }  // namespace tcq

@@ -1,7 +1,7 @@
 // decode.cu -- bitstream -> values for the bitshift trellis.
 //
-// The 2-bit post describes decoding as "read bits, update state, look up
-// values"; with the bitshift trellis of QTIP the state after symbol t is just
+// The 2-bit post's decoder advances the state from the bits and fetches each
+// codeword; with the bitshift trellis of QTIP the state after symbol t is just
 // the last L bits of (start || stream[0, tk)), so every output is independent:
 // one window extract and one codebook gather, no serial state.
 //

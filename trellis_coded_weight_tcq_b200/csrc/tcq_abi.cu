@@ -173,6 +173,46 @@ tcq_status tcq_decode(const uint32_t* bits, const uint32_t* start_state, const v
     return e == cudaSuccess ? TCQ_OK : TCQ_ERR_CUDA;
 }
 
+tcq_status tcq_gemv(const uint32_t* bits, const uint32_t* start_state, const float* scale,
+                    const void* codebook, tcq_dtype cb_dtype, int L, int k, int T, int64_t rows,
+                    int64_t cols, const float* x, float* y, tcq_stream_t stream)
+{
+    if (rows < 0 || cols < 0) return TCQ_ERR_INVALID_ARG;
+    if (!valid_dtype(cb_dtype)) return TCQ_ERR_INVALID_ARG;
+    const tcq_status shape = check_shape(L, k, T);
+    if (shape != TCQ_OK) return shape;
+    if (T % 4 != 0) return TCQ_ERR_UNSUPPORTED;
+    if (cb_dtype == TCQ_F32 && L >= 15) return TCQ_ERR_UNSUPPORTED;  // table must fit in smem
+    if (cols % T != 0) return TCQ_ERR_INVALID_ARG;
+    if (rows == 0) return TCQ_OK;
+    if (cols > ((int64_t)1 << 31)) return TCQ_ERR_INVALID_ARG;
+    if (!bits || !start_state || !codebook || !x || !y) return TCQ_ERR_INVALID_ARG;
+    const size_t entry = cb_dtype == TCQ_F16 ? 2 : 4;
+    if (!aligned(bits, 4) || !aligned(start_state, 4) || (scale && !aligned(scale, 4)) ||
+        !aligned(codebook, entry) || !aligned(x, 16) || !aligned(y, 4))
+        return TCQ_ERR_INVALID_ARG;
+    if ((unsigned long long)rows * (unsigned long long)(cols / T) > (1ull << 40))
+        return TCQ_ERR_INVALID_ARG;
+    const int sms = current_sms();
+    if (sms <= 0) return TCQ_ERR_CUDA;
+    GemvArgs a;
+    a.bits = bits;
+    a.start_state = start_state;
+    a.scale = scale;
+    a.cb = codebook;
+    a.cb_f16 = cb_dtype == TCQ_F16 ? 1 : 0;
+    a.L = L;
+    a.K = k;
+    a.T = T;
+    a.W = tcq_words_per_block(k, T);
+    a.rows = rows;
+    a.cols = cols;
+    a.x = x;
+    a.y = y;
+    const cudaError_t e = launch_gemv(a, sms, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TCQ_OK : TCQ_ERR_CUDA;
+}
+
 const char* tcq_status_string(tcq_status status)
 {
     switch (status) {

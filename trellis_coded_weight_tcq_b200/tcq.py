@@ -64,6 +64,8 @@ def load_library() -> ctypes.CDLL:
     lib.tcq_status_string.restype = ctypes.c_char_p
     lib.tcq_encode_path.argtypes = [ci, ci, ci]
     lib.tcq_encode_path.restype = ctypes.c_char_p
+    lib.tcq_gemv.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, i64, i64, vp, vp, vp]
+    lib.tcq_gemv.restype = ci
     _lib = lib
     return lib
 
@@ -95,6 +97,11 @@ def tcq_encode(x, d, codebook, cb_dtype, L, k, T, n_blocks, start_state, bits, p
 def tcq_decode(bits, start_state, codebook, cb_dtype, L, k, T, n_blocks, y, stream) -> int:
     return int(load_library().tcq_decode(bits, start_state, codebook, cb_dtype, L, k, T, n_blocks,
                                           y, stream))
+
+
+def tcq_gemv(bits, start_state, scale, codebook, cb_dtype, L, k, T, rows, cols, x, y, stream) -> int:
+    return int(load_library().tcq_gemv(bits, start_state, scale, codebook, cb_dtype, L, k, T, rows,
+                                        cols, x, y, stream))
 
 
 def tcq_status_string(status: int) -> str:
@@ -188,6 +195,18 @@ def decode(bits, start_state, codebook, L: int, k: int, T: int, out=None, stream
         out = torch.empty((n, T), dtype=torch.float32, device=bits.device)
     _check(tcq_decode(_ptr(bits), _ptr(start_state), _ptr(codebook), cb_dtype_of(codebook), L, k,
                       T, n, _ptr(out), _stream_handle(stream)), "tcq_decode")
+    return out
+
+
+def gemv(bits, start_state, scale, codebook, L: int, k: int, T: int, rows: int, cols: int, x,
+         out=None, stream=None):
+    """y = (trellis-coded matrix) @ x, decoding on the fly; blocks row-major [rows, cols/T]."""
+    torch = _torch()
+    if out is None:
+        out = torch.empty(rows, dtype=torch.float32, device=x.device)
+    _check(tcq_gemv(_ptr(bits), _ptr(start_state), _ptr(scale), _ptr(codebook),
+                    cb_dtype_of(codebook), L, k, T, rows, cols, _ptr(x), _ptr(out),
+                    _stream_handle(stream)), "tcq_gemv")
     return out
 
 
