@@ -10,6 +10,7 @@ from .tcq_oracle import (  # noqa: F401
     oracle_encode,
     oracle_gemv,
     oracle_greedy,
+    oracle_ldlq,
     oracle_path_cost,
     oracle_words_per_block,
 )

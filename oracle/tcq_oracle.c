@@ -300,3 +300,51 @@ int oracle_gemv(const uint32_t* bits, const uint32_t* start_state, const double*
     free(vals);
     return ORACLE_OK;
 }
+
+/*
+ * Error-feedback (LDLQ) encode of a rows x cols matrix, column block by column
+ * block.  "How do you fit a 4B LLM in 1.24 GB? Trellis-coded 2-bit", section on
+ * error feedback and LDLQ: columns are quantised in order and each one's error
+ * is pushed onto the columns not yet quantised, in proportions set by
+ * H = E[x x^T]; CurveTQ abstract: the feedback runs between coding blocks and
+ * the Viterbi metric inside a block is weighted by the diagonal of H's LDL
+ * factorisation.
+ *
+ * With H = U diag(d) U^T, U unit upper triangular (cols x cols, row-major, only
+ * the strictly upper part is read) and w_r the r-th row:
+ *   for block B = [jT, jT + T):
+ *     x_r[c] = w_r[c] + sum_{i < jT} (w_r[i] - q_r[i]) U[i][c],   c in B
+ *     (q_r[B], bits, start) = Viterbi TCQ of x_r[B] with weights d[B]
+ * Outputs: q [rows, cols], the targets x [rows, cols], and per coding block
+ * (block (r, j) = r * cols/T + j) start state, bits and cost.
+ */
+int oracle_ldlq(const double* w, const double* u, const double* dd, const double* cb, int L,
+                int k, int T, int64_t rows, int64_t cols, double* q, double* xt,
+                uint32_t* start_state, uint32_t* bits, double* cost)
+{
+    if (!valid_shape(L, k, T) || rows < 0 || cols < 0 || cols % T != 0) return ORACLE_EINVAL;
+    if (rows == 0 || cols == 0) return ORACLE_OK;
+    if (!w || !u || !dd || !cb || !q || !xt || !start_state || !bits || !cost)
+        return ORACLE_EINVAL;
+    const int64_t nb = cols / T;
+    const int W = oracle_words_per_block(k, T);
+    for (int64_t r = 0; r < rows; ++r) {
+        const double* wr = w + r * cols;
+        double* qr = q + r * cols;
+        double* xr = xt + r * cols;
+        for (int64_t j = 0; j < nb; ++j) {
+            for (int64_t c = j * T; c < (j + 1) * T; ++c) {
+                double acc = wr[c];
+                for (int64_t i = 0; i < j * T; ++i) acc += (wr[i] - qr[i]) * u[i * cols + c];
+                xr[c] = acc;
+            }
+            const int64_t b = r * nb + j;
+            int rc = oracle_encode(xr + j * T, dd + j * T, cb, L, k, T, 1, -1, start_state + b,
+                                   bits + b * W, cost + b);
+            if (rc != ORACLE_OK) return rc;
+            rc = oracle_decode(bits + b * W, start_state + b, cb, L, k, T, 1, qr + j * T);
+            if (rc != ORACLE_OK) return rc;
+        }
+    }
+    return ORACLE_OK;
+}

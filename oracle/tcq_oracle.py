@@ -50,6 +50,8 @@ def _load():
         lib.oracle_greedy.restype = ci
         lib.oracle_gemv.argtypes = [up, up, dp, dp, ci, ci, ci, i64, i64, dp, dp]
         lib.oracle_gemv.restype = ci
+        lib.oracle_ldlq.argtypes = [dp, dp, dp, dp, ci, ci, ci, i64, i64, dp, dp, up, up, dp]
+        lib.oracle_ldlq.restype = ci
         _lib = lib
     return _lib
 
@@ -180,3 +182,33 @@ def oracle_gemv(bits, start_state, scale, codebook, L: int, k: int, T: int, rows
     if rc != 0:
         raise ValueError(f"oracle_gemv failed with code {rc}")
     return y
+
+
+def oracle_ldlq(w, u, d, codebook, L: int, k: int, T: int):
+    """Error-feedback TCQ of the matrix ``w`` ([rows, cols]) by column blocks of T.
+
+    ``u`` is the unit upper factor and ``d`` the diagonal of H = U diag(d) U^T.
+    Returns (q [rows, cols], x targets [rows, cols], start [rows*nb],
+    bits [rows*nb, W], cost [rows*nb]), blocks indexed r * (cols/T) + j.
+    """
+    w = _f64(w)
+    rows, cols = w.shape
+    u = _f64(u).reshape(cols, cols)
+    d = _f64(d).reshape(cols)
+    cb = _f64(codebook).reshape(-1)
+    nb = cols // T
+    W = oracle_words_per_block(k, T)
+    q = np.zeros((rows, cols))
+    xt = np.zeros((rows, cols))
+    start = np.zeros(rows * nb, dtype=np.uint32)
+    bits = np.zeros((rows * nb, W), dtype=np.uint32)
+    cost = np.zeros(rows * nb)
+    rc = _load().oracle_ldlq(
+        _ptr(w, ctypes.c_double), _ptr(u, ctypes.c_double), _ptr(d, ctypes.c_double),
+        _ptr(cb, ctypes.c_double), L, k, T, rows, cols, _ptr(q, ctypes.c_double),
+        _ptr(xt, ctypes.c_double), _ptr(start, ctypes.c_uint32), _ptr(bits, ctypes.c_uint32),
+        _ptr(cost, ctypes.c_double),
+    )
+    if rc != 0:
+        raise ValueError(f"oracle_ldlq failed with code {rc}")
+    return q, xt, start, bits, cost
