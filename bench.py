@@ -299,8 +299,10 @@ def run_ours(args, rank, world, local_rank):
     # block row: rows = blocks * T / cols)
     gemv = None
     mat = wl.meta.get("matrix")
-    if mat and rank == 0:
-        rows_m, cols_m = int(mat[0]), int(mat[1])
+    if mat and rank == 0 and (n * T) % int(mat[1]) == 0:
+        # the rows the encoded blocks cover (all of the matrix unless --blocks cut it)
+        cols_m = int(mat[1])
+        rows_m = n * T // cols_m
         xv = torch.randn(cols_m, device=dev)
         scale = torch.ones(n, device=dev)
         ym = torch.empty(rows_m, device=dev)
@@ -359,6 +361,40 @@ def run_ours(args, rank, world, local_rank):
                              "alu_frac": wl.nodes * ALGO_OPS_PER_NODE / (acs_ms / 1e3) / peaks_ops(),
                              "kernel": tcq.tcq_encode_path(L, k, tcq.cb_dtype_of(cb))})
 
+    # ---- error-feedback (LDLQ) encode of the MLP matrix: 16 column blocks, each
+    # a feedback product, an encode of 14336 blocks and a decode
+    ldlq = None
+    if rank == 0 and world == 1 and not args.no_ldlq:
+        torch.cuda.empty_cache()
+        lw = workloads.ldlq_mlp()
+        w_t = torch.from_numpy(lw.w).to(dev)
+        u_t = torch.from_numpy(lw.u).to(dev)
+        d_t = torch.from_numpy(lw.d).to(dev)
+        cb_t = torch.from_numpy(lw.codebook).to(dev)
+        lws = torch.empty(tcq.tcq_ldlq_workspace_bytes(lw.L, lw.k, lw.T, lw.rows, lw.cols,
+                                                       tcq.cb_dtype_of(cb_t)),
+                          dtype=torch.uint8, device=dev)
+        tcq.ldlq(w_t, u_t, d_t, cb_t, lw.L, lw.k, lw.T, keep_targets=False, workspace=lws)
+        l_ev = []
+        for _ in range(2):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            res = tcq.ldlq(w_t, u_t, d_t, cb_t, lw.L, lw.k, lw.T, keep_targets=False, workspace=lws)
+            b.record(stream)
+            l_ev.append((a, b))
+        torch.cuda.synchronize()
+        l_ms = sum(a.elapsed_time(b) for a, b in l_ev) / len(l_ev)
+        costs = res.coded.path_cost.cpu().numpy()
+        assert np.all(np.isfinite(costs)) and np.all(costs >= 0)
+        nbc = lw.cols // lw.T
+        ldlq = {"workload": lw.name, "ms": l_ms, "nodes_per_s": lw.nodes / (l_ms / 1e3),
+                "weights_per_s": lw.rows * lw.cols / (l_ms / 1e3),
+                "feedback_flops": lw.rows * lw.T * lw.T * nbc * (nbc - 1),
+                "launches_per_call": 3 * nbc,
+                "alu_frac": lw.nodes * ALGO_OPS_PER_NODE / (l_ms / 1e3) / peaks_ops(),
+                "proxy_loss_per_weight": float(costs.astype(np.float64).sum()) / (lw.rows * lw.cols)}
+        del w_t, u_t, d_t, lws, res
+
     # sanity: the last step's result is a valid encode of the workload (cheap host check)
     cost_h = cost_last
     assert np.all(np.isfinite(cost_h)) and np.all(cost_h >= 0)
@@ -409,7 +445,7 @@ def run_ours(args, rank, world, local_rank):
         "weights_per_s": world * wl.weights / (ms / 1e3),
         "encode_ms_per_step": acs_ms, "decode_ms_per_step": dec_ms,
         "roofline": roofline, "decode_roofline": decode_roofline, "cpu_baseline": cpu_baseline, "e2e": e2e,
-        "per_workload": per_workload, "gemv": gemv,
+        "per_workload": per_workload, "gemv": gemv, "ldlq": ldlq,
         "clocks": clocks.summary(), "gpu_launches": gpu_launches,
     }
     print(json.dumps(line), flush=True)
@@ -426,6 +462,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-workload", action="store_true",
                     help="skip the short encode/decode timing of the other named workloads")
+    ap.add_argument("--no-ldlq", action="store_true",
+                    help="skip the error-feedback encode of the MLP matrix")
     ap.add_argument("--cpu-blocks-per-core", type=int, default=4)
     ap.add_argument("--blocks", type=int, default=0,
                     help="encode only the first N blocks of the workload (a smaller profiling "

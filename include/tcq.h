@@ -156,6 +156,50 @@ tcq_status tcq_gemv(const uint32_t* bits, const uint32_t* start_state, const flo
                     const void* codebook, tcq_dtype cb_dtype, int L, int k, int T, int64_t rows,
                     int64_t cols, const float* x, float* y, tcq_stream_t stream);
 
+/*
+ * Error-feedback quantisation of a matrix, one column block at a time (the 2-bit
+ * post's section on error feedback and LDLQ: each quantised column's error is
+ * pushed onto the columns not yet quantised, in proportions set by
+ * H = E[x x^T]; CurveTQ's abstract: the feedback runs between coding blocks and
+ * the Viterbi metric of a block is weighted by the diagonal of H's LDL
+ * factorisation).
+ *
+ * With H = U diag(d) U^T, U unit upper triangular, and W the rows x cols weight
+ * matrix, for each column block B = [jT, jT + T) in order and every row r:
+ *     X[r, c] = W[r, c] + sum_{i < jT} (W[r, i] - Q[r, i]) U[i, c]      c in B
+ *     coding block (r, j) = tcq_encode of X[r, B] with weights d[B]
+ *     Q[r, B] = tcq_decode of that block
+ * Only U's entries above its T x T diagonal blocks are read: feedback inside a
+ * block is not applied (the Viterbi search codes the block jointly).  The
+ * factorisation H -> (U, d) is the caller's.
+ *
+ *   w           fp32 [rows, cols] row-major.
+ *   u           fp32 [cols, cols] row-major.
+ *   d           fp32 [cols], or NULL for d = 1.
+ *   codebook    as tcq_encode.
+ *   q           out: fp32 [rows, cols], the reconstruction Q.
+ *   x           out: fp32 [rows, cols], the targets X, or NULL if not wanted.
+ *   start_state out: uint32 [rows * cols / T]; bits out: uint32 [rows * cols / T, W];
+ *   path_cost   out: fp32 [rows * cols / T]; block (r, j) at index r * (cols / T) + j,
+ *               the layout tcq_gemv reads.
+ *   workspace   device scratch, 256-byte aligned, at least
+ *               tcq_ldlq_workspace_bytes(...) for full speed (it holds one column
+ *               block's targets plus an encode workspace for `rows` blocks).
+ * Every pointer except d and x must be non-NULL and 4-byte aligned (the codebook
+ * to its entry size).  Requires cols % T == 0 and rows <= 65535 * 128, else
+ * TCQ_ERR_INVALID_ARG; a workspace too small for the targets and one CTA's
+ * encode share returns TCQ_ERR_WORKSPACE.  Launches 3 kernels per column block
+ * on `stream`; rows == 0 or cols == 0 is a no-op.  Each block's path and cost
+ * have tcq_encode's guarantees for that block's targets.
+ */
+size_t tcq_ldlq_workspace_bytes(int L, int k, int T, int64_t rows, int64_t cols,
+                                tcq_dtype cb_dtype);
+
+tcq_status tcq_ldlq(const float* w, const float* u, const float* d, const void* codebook,
+                    tcq_dtype cb_dtype, int L, int k, int T, int64_t rows, int64_t cols, float* q,
+                    float* x, uint32_t* start_state, uint32_t* bits, float* path_cost,
+                    void* workspace, size_t workspace_bytes, tcq_stream_t stream);
+
 /* Static, human-readable name of a status code. */
 const char* tcq_status_string(tcq_status status);
 

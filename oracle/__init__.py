@@ -8,6 +8,7 @@ from .tcq_oracle import (  # noqa: F401
     build_oracle,
     oracle_decode,
     oracle_encode,
+    oracle_feedback_targets,
     oracle_gemv,
     oracle_greedy,
     oracle_ldlq,

@@ -302,6 +302,29 @@ int oracle_gemv(const uint32_t* bits, const uint32_t* start_state, const double*
 }
 
 /*
+ * The targets of column block j given the reconstruction of the blocks before
+ * it (the feedback step of the error-feedback encode below):
+ *   x[r][c] = w[r][c] + sum_{i < jT} (w[r][i] - q[r][i]) u[i][c],  c in [jT, jT + T).
+ * Only x's columns of block j are written.
+ */
+int oracle_feedback(const double* w, const double* u, const double* q, int T, int64_t rows,
+                    int64_t cols, int64_t j, double* xt)
+{
+    if (T < 1 || rows < 0 || cols < 0 || cols % T != 0 || j < 0 || j * T >= cols)
+        return ORACLE_EINVAL;
+    for (int64_t r = 0; r < rows; ++r) {
+        const double* wr = w + r * cols;
+        const double* qr = q + r * cols;
+        for (int64_t c = j * T; c < (j + 1) * T; ++c) {
+            double acc = wr[c];
+            for (int64_t i = 0; i < j * T; ++i) acc += (wr[i] - qr[i]) * u[i * cols + c];
+            xt[r * cols + c] = acc;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/*
  * Error-feedback (LDLQ) encode of a rows x cols matrix, column block by column
  * block.  "How do you fit a 4B LLM in 1.24 GB? Trellis-coded 2-bit", section on
  * error feedback and LDLQ: columns are quantised in order and each one's error
@@ -333,11 +356,7 @@ int oracle_ldlq(const double* w, const double* u, const double* dd, const double
         double* qr = q + r * cols;
         double* xr = xt + r * cols;
         for (int64_t j = 0; j < nb; ++j) {
-            for (int64_t c = j * T; c < (j + 1) * T; ++c) {
-                double acc = wr[c];
-                for (int64_t i = 0; i < j * T; ++i) acc += (wr[i] - qr[i]) * u[i * cols + c];
-                xr[c] = acc;
-            }
+            oracle_feedback(wr, u, qr, T, 1, cols, j, xr);
             const int64_t b = r * nb + j;
             int rc = oracle_encode(xr + j * T, dd + j * T, cb, L, k, T, 1, -1, start_state + b,
                                    bits + b * W, cost + b);

@@ -52,6 +52,8 @@ def _load():
         lib.oracle_gemv.restype = ci
         lib.oracle_ldlq.argtypes = [dp, dp, dp, dp, ci, ci, ci, i64, i64, dp, dp, up, up, dp]
         lib.oracle_ldlq.restype = ci
+        lib.oracle_feedback.argtypes = [dp, dp, dp, ci, i64, i64, i64, dp]
+        lib.oracle_feedback.restype = ci
         _lib = lib
     return _lib
 
@@ -212,3 +214,21 @@ def oracle_ldlq(w, u, d, codebook, L: int, k: int, T: int):
     if rc != 0:
         raise ValueError(f"oracle_ldlq failed with code {rc}")
     return q, xt, start, bits, cost
+
+
+def oracle_feedback_targets(w, u, q, T: int):
+    """Targets of every column block given the reconstruction ``q`` ([rows, cols]):
+    block j's targets use only q's columns before jT."""
+    w = _f64(w)
+    q = _f64(q)
+    rows, cols = w.shape
+    u = _f64(u).reshape(cols, cols)
+    xt = np.zeros((rows, cols))
+    lib = _load()
+    for j in range(cols // T):
+        rc = lib.oracle_feedback(_ptr(w, ctypes.c_double), _ptr(u, ctypes.c_double),
+                                 _ptr(q, ctypes.c_double), T, rows, cols, j,
+                                 _ptr(xt, ctypes.c_double))
+        if rc != 0:
+            raise ValueError(f"oracle_feedback failed with code {rc}")
+    return xt

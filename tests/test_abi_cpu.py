@@ -121,3 +121,22 @@ def test_rejections_happen_before_cuda(lib):
     assert dec(dt=1, cb=ctypes.c_void_p(0x10001)) == tcq.TCQ_ERR_INVALID_ARG
     assert dec(L=0) == tcq.TCQ_ERR_UNSUPPORTED
     assert dec(n=-5) == tcq.TCQ_ERR_INVALID_ARG
+
+
+def test_binding_rejects_undersized_tensors_before_any_launch():
+    """The Python wrappers check tensor sizes against the shape they are given,
+    so a call can never hand the library a buffer smaller than the matrix."""
+    import torch
+    from trellis_coded_weight_tcq_b200 import tcq
+
+    W = tcq.tcq_words_per_block(2, 256)
+    bits = torch.zeros((10, W), dtype=torch.int32)
+    start = torch.zeros(10, dtype=torch.int32)
+    cb = torch.zeros(1 << 16, dtype=torch.float16)
+    x = torch.zeros(4096)
+    with pytest.raises(ValueError):  # 74 x 4096 needs 1184 blocks
+        tcq.gemv(bits, start, None, cb, 16, 2, 256, 74, 4096, x)
+    with pytest.raises(ValueError):
+        tcq.decode(bits[:5], start, cb, 16, 2, 256)
+    with pytest.raises(ValueError):
+        tcq.decode(bits, start, cb, 16, 2, 256, out=torch.empty((9, 256)))

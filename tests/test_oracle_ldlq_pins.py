@@ -144,3 +144,18 @@ def test_rejects_bad_shapes():
     cb = np.zeros(16)
     with pytest.raises(ValueError):
         oracle_ldlq(np.zeros((2, 10)), np.eye(10), np.ones(10), cb, 4, 2, 4)  # cols % T != 0
+
+
+def test_feedback_targets_match_the_driver():
+    """The standalone feedback step, fed the driver's own reconstruction,
+    reproduces the driver's targets for every block."""
+    from oracle import oracle_feedback_targets
+
+    rng = np.random.default_rng(53)
+    L, k, T, rows, cols = 5, 1, 6, 3, 36
+    w = rng.standard_normal((rows, cols))
+    d = rng.lognormal(0.0, 0.5, cols)
+    cb = rng.standard_normal(1 << L)
+    U = np.triu(rng.standard_normal((cols, cols)) * 0.2, 1) + np.eye(cols)
+    q, xt, _, _, _ = oracle_ldlq(w, U, d, cb, L, k, T)
+    assert np.array_equal(oracle_feedback_targets(w, U, q, T), xt)

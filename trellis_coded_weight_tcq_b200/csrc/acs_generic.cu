@@ -54,8 +54,8 @@ __global__ void __launch_bounds__(kGenericThreads) acs_generic_kernel(EncodeArgs
                        : reinterpret_cast<float*>(slot + generic_bp_bytes(L, K, T));
 
     for (long long b = blockIdx.x; b < a.n_blocks; b += gridDim.x) {
-        const float* xb = a.x + b * T;
-        const float* db = a.d ? a.d + b * T : nullptr;
+        const float* xb = a.x + b * a.x_stride;
+        const float* db = a.d ? a.d + b * a.d_stride : nullptr;
         float bestv = __int_as_float(0x7f800000);
         uint32_t bests = 0xffffffffu;
         for (int t = 1; t <= T; ++t) {
@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(kGenericThreads) acs_generic_kernel(EncodeArgs
             for (int w = 1; w < (int)(blockDim.x >> 5); ++w) keep_best(redv[w], reds[w], bv, bs);
             fin = bs;
             // traceback, bit packing and the fp64 cost along the path
-            BackwardBitWriter bw(a.bits + b * a.W, a.W);
+            BackwardBitWriter bw(a.bits + b * a.out_stride * a.W, a.W);
             uint32_t s = fin;
             double cost = 0.0;
             for (int t = T; t >= 1; --t) {
@@ -116,8 +116,8 @@ __global__ void __launch_bounds__(kGenericThreads) acs_generic_kernel(EncodeArgs
                 }
             }
             bw.finish();
-            a.start_state[b] = s >> K;
-            a.path_cost[b] = (float)cost;
+            a.start_state[b * a.out_stride] = s >> K;
+            a.path_cost[b * a.out_stride] = (float)cost;
         }
         __syncthreads();
     }

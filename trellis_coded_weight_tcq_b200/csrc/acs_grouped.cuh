@@ -374,8 +374,8 @@ __device__ __forceinline__ void finish_block(const EncodeArgs& a, long long b,
     const int T = a.T;
     double acc = 0.0;
     if (b >= 0) {
-        const float* xb = a.x + b * T;
-        const float* db = a.d ? a.d + b * T : nullptr;
+        const float* xb = a.x + b * opaque(a.x_stride);
+        const float* db = a.d ? a.d + b * opaque(a.d_stride) : nullptr;
         for (int t = tid; t < T; t += C::NT) {
             const double e = (double)xb[t] - (double)load_codeword(a.cb, a.cb_f16, path[t]);
             acc += (double)(db ? db[t] : 1.f) * e * e;
@@ -389,13 +389,13 @@ __device__ __forceinline__ void finish_block(const EncodeArgs& a, long long b,
                 const uint32_t sym = path[p / C::K] & (C::H - 1);
                 word |= ((sym >> (C::K - 1 - p % C::K)) & 1u) << (31 - i);
             }
-            a.bits[b * a.W + w] = word;
+            a.bits[b * opaque(a.out_stride) * a.W + w] = word;
         }
     }
     const double total = team_sum<C>(acc, redd, m, tid);
     if (b >= 0 && tid == 0) {
-        a.start_state[b] = (uint32_t)path[0] >> C::K;
-        a.path_cost[b] = (float)total;
+        a.start_state[b * opaque(a.out_stride)] = (uint32_t)path[0] >> C::K;
+        a.path_cost[b * opaque(a.out_stride)] = (float)total;
     }
 }
 
@@ -458,8 +458,8 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB) acs_grouped_kernel(Encod
         const long long b = first + (long long)r * stride + m;
         const bool valid = b < nb;
         unit_t* bp = reinterpret_cast<unit_t*>(slot + (size_t)(par * C::NTEAM + m) * team_bytes);
-        const float* xb = a.x + (valid ? b : 0) * T;
-        const float* db = a.d ? a.d + (valid ? b : 0) * T : nullptr;
+        const float* xb = a.x + (valid ? b : 0) * opaque(a.x_stride);
+        const float* db = a.d ? a.d + (valid ? b : 0) * opaque(a.d_stride) : nullptr;
         float dfloor = 0.f;
         if constexpr (C::CB16 && WEIGHTED) {
             float dm = 0.f;

@@ -84,9 +84,9 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a)
             const int p0 = (4 * q + 1) * K - L;
             f.off[u] = p0 & 31;
             if (b < a.n_blocks) {
-                const uint32_t* wb = a.bits + b * W;
+                const uint32_t* wb = a.bits + b * a.in_stride * W;
                 const int wi = p0 >> 5;  // -1 for the first windows
-                const unsigned long long hi = wi < 0 ? a.start_state[b] : wb[wi];
+                const unsigned long long hi = wi < 0 ? a.start_state[b * a.in_stride] : wb[wi];
                 const unsigned long long lo = wi + 1 < W ? wb[wi + 1] : 0ull;
                 f.win[u] = (hi << 32) | lo;
             }
@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a)
 #pragma unroll
             for (int e = 0; e < 4; ++e)
                 v[e] = lookup((uint32_t)(f.win[u] >> (64 - f.off[u] - e * K - L)) & mask);
-            float* yb = a.y + b * T;
+            float* yb = a.y + b * a.y_stride;
             if constexpr (VEC) {
                 __stcs(reinterpret_cast<float4*>(yb + 4 * q), make_float4(v[0], v[1], v[2], v[3]));
             } else {
@@ -172,7 +172,8 @@ cudaError_t launch_decode(const DecodeArgs& a, int num_sms, cudaStream_t stream)
     const long long cap = (long long)num_sms * ctas_per_sm;
     if (grid > cap) grid = cap;
     if (grid < 1) grid = 1;
-    const bool vec = (a.T % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.y) & 15) == 0);
+    const bool vec = (a.T % 4 == 0) && (a.y_stride % 4 == 0) &&
+                     ((reinterpret_cast<uintptr_t>(a.y) & 15) == 0);
     switch (mode * 2 + (vec ? 1 : 0)) {
     case 0: return launch_mode<kTableF32, false>(a, (int)grid, smem, stream);
     case 1: return launch_mode<kTableF32, true>(a, (int)grid, smem, stream);

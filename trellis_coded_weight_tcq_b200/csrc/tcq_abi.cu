@@ -65,6 +65,29 @@ long long wanted_ctas(const EncodeKernelInfo* info, int L, int k, int T, long lo
     return by_blocks < resident ? by_blocks : resident;
 }
 
+// Plans the grid for an encode whose arguments are filled in (all but the
+// workspace) and launches it.
+tcq_status run_encode(EncodeArgs& a, tcq_dtype cb_dtype, void* workspace, size_t workspace_bytes,
+                      cudaStream_t stream)
+{
+    const EncodeKernelInfo* info = select_kernel(a.L, a.K, cb_dtype);
+    if (!info) return TCQ_ERR_INTERNAL;
+    const size_t slot = info->slot_bytes(a.L, a.K, a.T);
+    const int sms = current_sms();
+    if (sms <= 0) return TCQ_ERR_CUDA;
+    long long grid = wanted_ctas(info, a.L, a.K, a.T, a.n_blocks, sms);
+    if (slot > 0) {
+        const long long fit = (long long)(workspace_bytes / slot);
+        if (fit < 1) return TCQ_ERR_WORKSPACE;
+        if (grid > fit) grid = fit;
+    }
+    if (grid < 1) grid = 1;
+    a.ws = static_cast<unsigned char*>(workspace);
+    a.slot_bytes = slot;
+    const cudaError_t e = info->launch(a, (int)grid, stream);
+    return e == cudaSuccess ? TCQ_OK : TCQ_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -108,19 +131,6 @@ tcq_status tcq_encode(const float* x, const float* d, const void* codebook, tcq_
         return TCQ_ERR_INVALID_ARG;
     if ((unsigned long long)n_blocks > (1ull << 40)) return TCQ_ERR_INVALID_ARG;
 
-    const EncodeKernelInfo* info = select_kernel(L, k, cb_dtype);
-    if (!info) return TCQ_ERR_INTERNAL;
-    const size_t slot = info->slot_bytes(L, k, T);
-    const int sms = current_sms();
-    if (sms <= 0) return TCQ_ERR_CUDA;
-    long long grid = wanted_ctas(info, L, k, T, n_blocks, sms);
-    if (slot > 0) {
-        const long long fit = (long long)(workspace_bytes / slot);
-        if (fit < 1) return TCQ_ERR_WORKSPACE;
-        if (grid > fit) grid = fit;
-    }
-    if (grid < 1) grid = 1;
-
     EncodeArgs a;
     a.x = x;
     a.d = d;
@@ -134,10 +144,11 @@ tcq_status tcq_encode(const float* x, const float* d, const void* codebook, tcq_
     a.start_state = start_state;
     a.bits = bits;
     a.path_cost = path_cost;
-    a.ws = static_cast<unsigned char*>(workspace);
-    a.slot_bytes = slot;
-    const cudaError_t e = info->launch(a, (int)grid, reinterpret_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? TCQ_OK : TCQ_ERR_CUDA;
+    a.x_stride = T;
+    a.d_stride = T;
+    a.out_stride = 1;
+    return run_encode(a, cb_dtype, workspace, workspace_bytes,
+                      reinterpret_cast<cudaStream_t>(stream));
 }
 
 tcq_status tcq_decode(const uint32_t* bits, const uint32_t* start_state, const void* codebook,
@@ -169,6 +180,8 @@ tcq_status tcq_decode(const uint32_t* bits, const uint32_t* start_state, const v
     a.W = tcq_words_per_block(k, T);
     a.n_blocks = n_blocks;
     a.y = y;
+    a.in_stride = 1;
+    a.y_stride = T;
     const cudaError_t e = launch_decode(a, sms, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TCQ_OK : TCQ_ERR_CUDA;
 }
@@ -211,6 +224,101 @@ tcq_status tcq_gemv(const uint32_t* bits, const uint32_t* start_state, const flo
     a.y = y;
     const cudaError_t e = launch_gemv(a, sms, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TCQ_OK : TCQ_ERR_CUDA;
+}
+
+size_t tcq_ldlq_workspace_bytes(int L, int k, int T, int64_t rows, int64_t cols,
+                                tcq_dtype cb_dtype)
+{
+    if (check_shape(L, k, T) != TCQ_OK || rows <= 0 || cols <= 0 || cols % T != 0 ||
+        !valid_dtype(cb_dtype))
+        return 0;
+    const size_t enc = tcq_encode_workspace_bytes(L, k, T, rows, cb_dtype);
+    const size_t targets = ((size_t)rows * (size_t)T * sizeof(float) + 255) & ~(size_t)255;
+    return targets + enc;
+}
+
+tcq_status tcq_ldlq(const float* w, const float* u, const float* d, const void* codebook,
+                    tcq_dtype cb_dtype, int L, int k, int T, int64_t rows, int64_t cols, float* q,
+                    float* x, uint32_t* start_state, uint32_t* bits, float* path_cost,
+                    void* workspace, size_t workspace_bytes, tcq_stream_t stream)
+{
+    if (rows < 0 || cols < 0) return TCQ_ERR_INVALID_ARG;
+    if (!valid_dtype(cb_dtype)) return TCQ_ERR_INVALID_ARG;
+    const tcq_status shape = check_shape(L, k, T);
+    if (shape != TCQ_OK) return shape;
+    if (cols % T != 0) return TCQ_ERR_INVALID_ARG;
+    if (rows == 0 || cols == 0) return TCQ_OK;
+    if (!w || !u || !codebook || !q || !start_state || !bits || !path_cost || !workspace)
+        return TCQ_ERR_INVALID_ARG;
+    const size_t entry = cb_dtype == TCQ_F16 ? 2 : 4;
+    if (!aligned(w, 4) || !aligned(u, 4) || (d && !aligned(d, 4)) || !aligned(codebook, entry) ||
+        !aligned(q, 4) || (x && !aligned(x, 4)) || !aligned(start_state, 4) ||
+        !aligned(bits, 4) || !aligned(path_cost, 4) || !aligned(workspace, 256))
+        return TCQ_ERR_INVALID_ARG;
+    // grid rows of the feedback product, and the block count of the code
+    if (rows > 65535LL * 128 || cols > ((int64_t)1 << 31)) return TCQ_ERR_INVALID_ARG;
+    const size_t targets = ((size_t)rows * (size_t)T * sizeof(float) + 255) & ~(size_t)255;
+    if (workspace_bytes <= targets) return TCQ_ERR_WORKSPACE;
+    const int sms = current_sms();
+    if (sms <= 0) return TCQ_ERR_CUDA;
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    const int64_t nb = cols / T;
+    const int W = tcq_words_per_block(k, T);
+    // targets of the current column block: x[:, B] when the caller keeps them,
+    // else the front of the workspace
+    float* xbuf = x ? x : reinterpret_cast<float*>(ws);
+    const long long x_ld = x ? cols : T;
+
+    for (int64_t j = 0; j < nb; ++j) {
+        const long long c0 = j * (long long)T;
+        FeedbackArgs f;
+        f.w = w;
+        f.q = q;
+        f.u = u;
+        f.rows = rows;
+        f.cols = cols;
+        f.c0 = c0;
+        f.n = T;
+        f.x = x ? xbuf + c0 : xbuf;
+        f.x_ld = x_ld;
+        if (launch_feedback(f, st) != cudaSuccess) return TCQ_ERR_CUDA;
+
+        EncodeArgs a;
+        a.x = f.x;
+        a.d = d ? d + c0 : nullptr;
+        a.cb = codebook;
+        a.cb_f16 = cb_dtype == TCQ_F16 ? 1 : 0;
+        a.L = L;
+        a.K = k;
+        a.T = T;
+        a.W = W;
+        a.n_blocks = rows;
+        a.start_state = start_state + j;
+        a.bits = bits + j * W;
+        a.path_cost = path_cost + j;
+        a.x_stride = x_ld;
+        a.d_stride = 0;
+        a.out_stride = nb;
+        const tcq_status es = run_encode(a, cb_dtype, ws + targets, workspace_bytes - targets, st);
+        if (es != TCQ_OK) return es;
+
+        DecodeArgs dq;
+        dq.bits = bits + j * W;
+        dq.start_state = start_state + j;
+        dq.cb = codebook;
+        dq.cb_f16 = a.cb_f16;
+        dq.L = L;
+        dq.K = k;
+        dq.T = T;
+        dq.W = W;
+        dq.n_blocks = rows;
+        dq.y = q + c0;
+        dq.in_stride = nb;
+        dq.y_stride = cols;
+        if (launch_decode(dq, sms, st) != cudaSuccess) return TCQ_ERR_CUDA;
+    }
+    return TCQ_OK;
 }
 
 const char* tcq_status_string(tcq_status status)

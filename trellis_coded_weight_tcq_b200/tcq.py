@@ -66,6 +66,11 @@ def load_library() -> ctypes.CDLL:
     lib.tcq_encode_path.restype = ctypes.c_char_p
     lib.tcq_gemv.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, i64, i64, vp, vp, vp]
     lib.tcq_gemv.restype = ci
+    lib.tcq_ldlq_workspace_bytes.argtypes = [ci, ci, ci, i64, i64, ci]
+    lib.tcq_ldlq_workspace_bytes.restype = sz
+    lib.tcq_ldlq.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, i64, i64, vp, vp, vp, vp, vp, vp,
+                             sz, vp]
+    lib.tcq_ldlq.restype = ci
     _lib = lib
     return lib
 
@@ -102,6 +107,17 @@ def tcq_decode(bits, start_state, codebook, cb_dtype, L, k, T, n_blocks, y, stre
 def tcq_gemv(bits, start_state, scale, codebook, cb_dtype, L, k, T, rows, cols, x, y, stream) -> int:
     return int(load_library().tcq_gemv(bits, start_state, scale, codebook, cb_dtype, L, k, T, rows,
                                         cols, x, y, stream))
+
+
+def tcq_ldlq_workspace_bytes(L: int, k: int, T: int, rows: int, cols: int, cb_dtype: int) -> int:
+    return int(load_library().tcq_ldlq_workspace_bytes(L, k, T, rows, cols, cb_dtype))
+
+
+def tcq_ldlq(w, u, d, codebook, cb_dtype, L, k, T, rows, cols, q, x, start_state, bits, path_cost,
+             workspace, workspace_bytes, stream) -> int:
+    return int(load_library().tcq_ldlq(w, u, d, codebook, cb_dtype, L, k, T, rows, cols, q, x,
+                                       start_state, bits, path_cost, workspace, workspace_bytes,
+                                       stream))
 
 
 def tcq_status_string(status: int) -> str:
@@ -191,8 +207,13 @@ def decode(bits, start_state, codebook, L: int, k: int, T: int, out=None, stream
     """Values [n_blocks, T] (fp32) of packed ``bits`` from ``start_state``."""
     torch = _torch()
     n = start_state.shape[0]
+    W = tcq_words_per_block(k, T)
+    if bits.numel() < n * max(W, 0):
+        raise ValueError("decode: bits holds fewer than n_blocks * W words")
     if out is None:
         out = torch.empty((n, T), dtype=torch.float32, device=bits.device)
+    if out.numel() < n * T:
+        raise ValueError("decode: out holds fewer than n_blocks * T values")
     _check(tcq_decode(_ptr(bits), _ptr(start_state), _ptr(codebook), cb_dtype_of(codebook), L, k,
                       T, n, _ptr(out), _stream_handle(stream)), "tcq_decode")
     return out
@@ -202,12 +223,61 @@ def gemv(bits, start_state, scale, codebook, L: int, k: int, T: int, rows: int, 
          out=None, stream=None):
     """y = (trellis-coded matrix) @ x, decoding on the fly; blocks row-major [rows, cols/T]."""
     torch = _torch()
+    nb = rows * (cols // T) if T > 0 else 0
+    W = tcq_words_per_block(k, T)
+    if bits.numel() < nb * max(W, 0) or start_state.numel() < nb or x.numel() < cols or (
+            scale is not None and scale.numel() < nb):
+        raise ValueError(f"gemv: tensors too small for a {rows} x {cols} matrix of T={T} blocks")
     if out is None:
         out = torch.empty(rows, dtype=torch.float32, device=x.device)
+    if out.numel() < rows:
+        raise ValueError("gemv: out holds fewer than rows values")
     _check(tcq_gemv(_ptr(bits), _ptr(start_state), _ptr(scale), _ptr(codebook),
                     cb_dtype_of(codebook), L, k, T, rows, cols, _ptr(x), _ptr(out),
                     _stream_handle(stream)), "tcq_gemv")
     return out
+
+
+@dataclass
+class LdlqResult:
+    q: "object"            # float32 [rows, cols], the reconstruction
+    x: "object"            # float32 [rows, cols], the targets, or None
+    coded: Encoded         # blocks (r, j) at r * (cols / T) + j
+
+
+def ldlq(w, u, d, codebook, L: int, k: int, T: int, keep_targets: bool = True, workspace=None,
+         stream=None) -> LdlqResult:
+    """Error-feedback TCQ of the matrix ``w`` (fp32 CUDA [rows, cols]) by column
+    blocks of T, with H = U diag(d) U^T (``u`` fp32 [cols, cols], ``d`` fp32 [cols]
+    or None)."""
+    torch = _torch()
+    if w.dim() != 2 or w.dtype != torch.float32 or not w.is_cuda or not w.is_contiguous():
+        raise ValueError("w must be a contiguous float32 CUDA tensor [rows, cols]")
+    rows, cols = w.shape
+    if u.shape != (cols, cols) or u.dtype != torch.float32 or not u.is_contiguous():
+        raise ValueError("u must be a contiguous float32 tensor [cols, cols]")
+    if d is not None and (d.shape != (cols,) or d.dtype != torch.float32 or not d.is_contiguous()):
+        raise ValueError("d must be None or a contiguous float32 tensor [cols]")
+    W = tcq_words_per_block(k, T)
+    if W < 0:
+        raise TCQError(TCQ_ERR_UNSUPPORTED, "tcq_words_per_block")
+    nb = cols // T if T > 0 else 0
+    dev = w.device
+    q = torch.empty((rows, cols), dtype=torch.float32, device=dev)
+    x = torch.empty((rows, cols), dtype=torch.float32, device=dev) if keep_targets else None
+    coded = Encoded(
+        torch.empty(rows * nb, dtype=torch.int32, device=dev),
+        torch.empty((rows * nb, W), dtype=torch.int32, device=dev),
+        torch.empty(rows * nb, dtype=torch.float32, device=dev),
+    )
+    if workspace is None:
+        nbytes = max(tcq_ldlq_workspace_bytes(L, k, T, rows, cols, cb_dtype_of(codebook)), 256)
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    _check(tcq_ldlq(_ptr(w), _ptr(u), _ptr(d), _ptr(codebook), cb_dtype_of(codebook), L, k, T,
+                    rows, cols, _ptr(q), _ptr(x), _ptr(coded.start_state), _ptr(coded.bits),
+                    _ptr(coded.path_cost), ctypes.c_void_p(workspace.data_ptr()),
+                    workspace.numel(), _stream_handle(stream)), "tcq_ldlq")
+    return LdlqResult(q, x, coded)
 
 
 class HostPipeline:

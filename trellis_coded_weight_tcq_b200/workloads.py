@@ -147,3 +147,74 @@ def dyadic_exact(L: int, k: int, T: int, n_blocks: int, weighted: bool, cb_dtype
     x = (rng.integers(-16, 17, (n_blocks, T)) / 8.0).astype(np.float32)
     d = (4.0 ** rng.integers(-1, 2, (n_blocks, T))).astype(np.float32) if weighted else None
     return Workload(f"dyadic_L{L}_k{k}_T{T}_B{n_blocks}", L, k, T, x, d, cb)
+
+
+@dataclass
+class LdlqWorkload:
+    """A matrix for the error-feedback encode, with the factor of its Hessian.
+
+    H = U diag(d) U^T is implied by (u, d): u is unit upper triangular, so H is
+    symmetric positive definite whenever d > 0.
+    """
+    name: str
+    L: int
+    k: int
+    T: int
+    w: np.ndarray                 # float32 [rows, cols]
+    u: np.ndarray                 # float32 [cols, cols], unit upper triangular
+    d: np.ndarray | None          # float32 [cols] or None (d = 1)
+    codebook: np.ndarray          # float32 or float16 [2^L]
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def rows(self) -> int:
+        return self.w.shape[0]
+
+    @property
+    def cols(self) -> int:
+        return self.w.shape[1]
+
+    @property
+    def n_blocks(self) -> int:
+        return self.rows * (self.cols // self.T)
+
+    @property
+    def nodes(self) -> int:
+        return self.n_blocks * self.T * (1 << self.L)
+
+
+def unit_upper_factor(cols: int, T: int, rho: float, seed: int, block_free: bool = False) -> np.ndarray:
+    """I plus strictly upper entries ~ N(0, rho^2 / cols); with ``block_free`` the
+    entries inside the T x T diagonal blocks are zero as well."""
+    rng = np.random.default_rng(seed)
+    u = np.triu(rng.standard_normal((cols, cols)).astype(np.float32) * np.float32(rho / np.sqrt(cols)), 1)
+    if block_free:
+        for j in range(cols // T):
+            u[j * T:(j + 1) * T, j * T:(j + 1) * T] = 0.0
+    u[np.arange(cols), np.arange(cols)] = 1.0
+    return u
+
+
+def ldlq_random(L: int, k: int, T: int, rows: int, cols: int, weighted: bool, cb_dtype: str,
+                seed: int, rho: float = 0.5, block_free: bool = False) -> LdlqWorkload:
+    """A small seeded case: w ~ N(0,1); U as unit_upper_factor; d ~ LogNormal(0,1)
+    per column; codebook N(0,1) in fp32 or fp16."""
+    rng = np.random.default_rng(seed)
+    w = rng.standard_normal((rows, cols)).astype(np.float32)
+    d = rng.lognormal(0.0, 1.0, cols).astype(np.float32) if weighted else None
+    cb = rng.standard_normal(1 << L)
+    cb = cb.astype(np.float16) if cb_dtype == "f16" else cb.astype(np.float32)
+    u = unit_upper_factor(cols, T, rho, seed + 1, block_free)
+    tag = "_blockfree" if block_free else ""
+    return LdlqWorkload(f"ldlq_L{L}_k{k}_T{T}_{rows}x{cols}{tag}", L, k, T, w, u, d, cb)
+
+
+def ldlq_mlp(shard: int = 0) -> LdlqWorkload:
+    """The MLP matrix (14336x4096 N(0, 0.02^2), bf16) divided by 0.02, with
+    U = I + N(0, 0.25/4096) strictly upper and d ~ LogNormal(0,1) per column;
+    L=16, k=2, T=256; fp16 N(0,1) codebook."""
+    W = _weight_matrix_gaussian(14336, 4096, SEED_X + 7919 * shard) / np.float32(0.02)
+    d = np.random.default_rng(SEED_D + 7919 * shard).lognormal(0.0, 1.0, 4096).astype(np.float32)
+    u = unit_upper_factor(4096, 256, 0.5, SEED_PERM + 1 + 7919 * shard)
+    return LdlqWorkload("ldlq_mlp_14336x4096_L16_k2_T256_weighted", 16, 2, 256, W.astype(np.float32),
+                        u, d, gaussian_sample_codebook_f16(1 << 16), {"matrix": [14336, 4096]})
