@@ -5,6 +5,7 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 path fails loudly when its extension is missing instead of falling back here.
 """
 from .tcq_oracle import (  # noqa: F401
+    oracle_bcjr,
     build_oracle,
     oracle_decode,
     oracle_encode,

@@ -367,3 +367,99 @@ int oracle_ldlq(const double* w, const double* u, const double* dd, const double
     }
     return ORACLE_OK;
 }
+
+/*
+ * Soft trellis quantization by the forward-backward (BCJR) sum-product
+ * recursion at temperature tau: "BCJR-QAT: A Differentiable Relaxation of
+ * Trellis-Coded Weight Quantization" (abstract, aggregator page).  The Viterbi
+ * minimum over paths is replaced by the Boltzmann distribution
+ *     P(path) = exp(-J(path) / tau) / Z,
+ * the soft codeword of position t is the expectation of c[s_t] under P, and it
+ * returns to the hard Viterbi code as tau -> 0.  A path is a state sequence
+ * s_1..s_T of the bitshift trellis with the first state free (each of the 2^L
+ * first states counted once) and J the weighted cost above.
+ *
+ * Per block, in natural-log units and double precision, per STATE:
+ *   la_1[s] = -d_1 (x_1 - c[s])^2 / tau
+ *   la_t[s] = -d_t (x_t - c[s])^2 / tau + lse_h la_{t-1}[(h << (L-k)) | (s >> k)]
+ *   lb_T[s] = 0
+ *   lb_t[s] = lse_b ( -d_{t+1} (x_{t+1} - c[s'])^2 / tau + lb_{t+1}[s'] ),
+ *             s' = ((s << k) | b) & mask
+ *   log Z   = lse_s la_T[s]
+ *   y_t     = sum_s exp(la_t[s] + lb_t[s] - log Z) c[s]
+ *   F       = -tau log Z                      (the free energy; F -> J_min)
+ * with lse the log-sum-exp.  Outputs y [n_blocks, T] and F [n_blocks].
+ */
+static double lse_add(double a, double b)
+{
+    if (a == -INFINITY) return b;
+    if (b == -INFINITY) return a;
+    const double m = a > b ? a : b;
+    return m + log(exp(a - m) + exp(b - m));
+}
+
+int oracle_bcjr(const double* x, const double* d, const double* cb, int L, int k, int T,
+                int64_t n_blocks, double tau, double* y, double* free_energy)
+{
+    if (!valid_shape(L, k, T) || n_blocks < 0 || !(tau > 0.0) || !isfinite(tau))
+        return ORACLE_EINVAL;
+    if (n_blocks == 0) return ORACLE_OK;
+    if (!x || !cb || !y || !free_energy) return ORACLE_EINVAL;
+    const int64_t S = (int64_t)1 << L;
+    const uint32_t mask = (uint32_t)(S - 1);
+    const int H = 1 << k;
+    double* la = (double*)malloc(sizeof(double) * (size_t)T * (size_t)S);
+    double* lb = (double*)malloc(sizeof(double) * (size_t)T * (size_t)S);
+    if (!la || !lb) {
+        free(la);
+        free(lb);
+        return ORACLE_EINVAL;
+    }
+    for (int64_t blk = 0; blk < n_blocks; ++blk) {
+        const double* xb = x + blk * T;
+        const int64_t base = blk * T;
+        /* forward */
+        for (int64_t s = 0; s < S; ++s) {
+            const double e = xb[0] - cb[s];
+            la[s] = -weight_at(d, base) * e * e / tau;
+        }
+        for (int t = 1; t < T; ++t) {
+            const double w = weight_at(d, base + t);
+            for (int64_t s = 0; s < S; ++s) {
+                double acc = -INFINITY;
+                for (int h = 0; h < H; ++h) {
+                    const uint32_t prev = (((uint32_t)h << (L - k)) | ((uint32_t)s >> k)) & mask;
+                    acc = lse_add(acc, la[(int64_t)(t - 1) * S + prev]);
+                }
+                const double e = xb[t] - cb[s];
+                la[(int64_t)t * S + s] = -w * e * e / tau + acc;
+            }
+        }
+        /* backward */
+        for (int64_t s = 0; s < S; ++s) lb[(int64_t)(T - 1) * S + s] = 0.0;
+        for (int t = T - 2; t >= 0; --t) {
+            const double w = weight_at(d, base + t + 1);
+            for (int64_t s = 0; s < S; ++s) {
+                double acc = -INFINITY;
+                for (int b = 0; b < H; ++b) {
+                    const uint32_t next = (((uint32_t)s << k) | (uint32_t)b) & mask;
+                    const double e = xb[t + 1] - cb[next];
+                    acc = lse_add(acc, -w * e * e / tau + lb[(int64_t)(t + 1) * S + next]);
+                }
+                lb[(int64_t)t * S + s] = acc;
+            }
+        }
+        double logz = -INFINITY;
+        for (int64_t s = 0; s < S; ++s) logz = lse_add(logz, la[(int64_t)(T - 1) * S + s]);
+        for (int t = 0; t < T; ++t) {
+            double acc = 0.0;
+            for (int64_t s = 0; s < S; ++s)
+                acc += exp(la[(int64_t)t * S + s] + lb[(int64_t)t * S + s] - logz) * cb[s];
+            y[base + t] = acc;
+        }
+        free_energy[blk] = -tau * logz;
+    }
+    free(la);
+    free(lb);
+    return ORACLE_OK;
+}

@@ -54,6 +54,8 @@ def _load():
         lib.oracle_ldlq.restype = ci
         lib.oracle_feedback.argtypes = [dp, dp, dp, ci, i64, i64, i64, dp]
         lib.oracle_feedback.restype = ci
+        lib.oracle_bcjr.argtypes = [dp, dp, dp, ci, ci, ci, i64, ctypes.c_double, dp, dp]
+        lib.oracle_bcjr.restype = ci
         _lib = lib
     return _lib
 
@@ -232,3 +234,24 @@ def oracle_feedback_targets(w, u, q, T: int):
         if rc != 0:
             raise ValueError(f"oracle_feedback failed with code {rc}")
     return xt
+
+
+def oracle_bcjr(x, d, codebook, L: int, k: int, tau: float):
+    """Soft codewords y [n, T] (expectation of c[s_t] under exp(-J/tau)/Z over
+    trellis paths) and free energies F = -tau log Z [n] for the blocks of ``x``."""
+    x = _f64(x)
+    if x.ndim == 1:
+        x = x[None, :]
+    n, T = x.shape
+    dd = None if d is None else _f64(d).reshape(n, T)
+    cb = _f64(codebook).reshape(-1)
+    y = np.zeros((n, T))
+    F = np.zeros(n)
+    rc = _load().oracle_bcjr(
+        _ptr(x, ctypes.c_double), None if dd is None else _ptr(dd, ctypes.c_double),
+        _ptr(cb, ctypes.c_double), L, k, T, n, float(tau), _ptr(y, ctypes.c_double),
+        _ptr(F, ctypes.c_double),
+    )
+    if rc != 0:
+        raise ValueError(f"oracle_bcjr failed with code {rc}")
+    return y, F

@@ -74,3 +74,33 @@ def decode_window(words, start: int, codebook, L: int, k: int, T: int) -> np.nda
     mask = (1 << L) - 1
     st = [((s0 << (t * k)) | (n >> ((T - t) * k))) & mask for t in range(1, T + 1)]
     return np.asarray(codebook, dtype=np.float64)[np.array(st, dtype=np.int64)]
+
+
+def path_table(x, d, codebook, L: int, k: int):
+    """Every distinct path of one block (first state free, counted once) with its
+    states [P, T] and cost J [P].  A path is fixed by s_0 in [0, 2^(L-k)) and the
+    bitstream, since the top k bits of s_0 never reach s_1."""
+    x = np.asarray(x, dtype=np.float64).reshape(-1)
+    T = x.size
+    d = np.ones(T) if d is None else np.asarray(d, dtype=np.float64).reshape(-1)
+    c = np.asarray(codebook, dtype=np.float64).reshape(-1)
+    assert c.size == 1 << L
+    assert (L - k) + T * k <= 20, "keep the enumeration small"
+    s0 = np.arange(1 << (L - k), dtype=np.int64)
+    n = np.arange(1 << (T * k), dtype=np.int64)
+    st = states_for(L, k, T, s0[:, None], n[None, :]).reshape(-1, T)
+    J = (d * (x - c[st]) ** 2).sum(axis=-1)
+    return st, J
+
+
+def boltzmann_brute_force(x, d, codebook, L: int, k: int, tau: float):
+    """Soft codewords E[c[s_t]] and free energy -tau log Z under P ~ exp(-J/tau),
+    summed over every path."""
+    st, J = path_table(x, d, codebook, L, k)
+    c = np.asarray(codebook, dtype=np.float64).reshape(-1)
+    a = -J / tau
+    m = a.max()
+    logz = m + np.log(np.exp(a - m).sum())
+    p = np.exp(a - logz)
+    y = (p[:, None] * c[st]).sum(axis=0)
+    return y, -tau * logz
