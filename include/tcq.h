@@ -200,6 +200,40 @@ tcq_status tcq_ldlq(const float* w, const float* u, const float* d, const void* 
                     float* x, uint32_t* start_state, uint32_t* bits, float* path_cost,
                     void* workspace, size_t workspace_bytes, tcq_stream_t stream);
 
+/*
+ * Soft trellis quantization (BCJR-QAT abstract: the Viterbi argmax replaced by
+ * the BCJR forward-backward sum-product recursion at temperature tau, giving
+ * the Boltzmann expectation of the codeword over trellis paths, which returns
+ * to the hard code as tau -> 0).
+ *
+ * Over the paths s_1..s_T of the bitshift trellis (first state free, each of
+ * the 2^L first states counted once) with cost J = sum_t d_t (x_t - c[s_t])^2:
+ *     P(path)      = exp(-J / tau) / Z
+ *     y_soft[b, t] = E_P[c[s_t]]            (the soft codeword)
+ *     free_energy[b] = -tau ln Z            (F <= J_min, F -> J_min as tau -> 0)
+ * computed in fp32 with the normalising constants summed in fp64.
+ *
+ *   x, d, codebook  as tcq_encode.
+ *   tau             > 0 and finite, with d_t (x_t - c)^2 / tau finite in fp32
+ *                   for every t and codeword (else TCQ_ERR_INVALID_ARG for tau
+ *                   itself, undefined values otherwise).
+ *   y_soft          out: fp32 [n_blocks, T], 4-byte aligned.
+ *   free_energy     out: fp32 [n_blocks], or NULL.
+ *   workspace       device scratch, 256-byte aligned, at least
+ *                   tcq_bcjr_workspace_bytes(...) for full speed; it holds the
+ *                   forward values of every step of a block (T * 2^(L-k) fp32)
+ *                   per concurrently processed block.  Smaller workspaces run
+ *                   fewer blocks at a time; one block's share is the minimum
+ *                   (else TCQ_ERR_WORKSPACE).
+ * n_blocks == 0 is a no-op.  One kernel launch on `stream`.
+ */
+size_t tcq_bcjr_workspace_bytes(int L, int k, int T, int64_t n_blocks, tcq_dtype cb_dtype);
+
+tcq_status tcq_bcjr(const float* x, const float* d, const void* codebook, tcq_dtype cb_dtype,
+                    int L, int k, int T, int64_t n_blocks, float tau, float* y_soft,
+                    float* free_energy, void* workspace, size_t workspace_bytes,
+                    tcq_stream_t stream);
+
 /* Static, human-readable name of a status code. */
 const char* tcq_status_string(tcq_status status);
 

@@ -74,6 +74,22 @@ struct GemvArgs {
     float* y;                     // [rows]
 };
 
+// Soft (forward-backward) quantization of n_blocks blocks at temperature tau.
+struct BcjrArgs {
+    const float* x;        // [n_blocks, T]
+    const float* d;        // [n_blocks, T] or nullptr (d_t = 1)
+    const void* cb;
+    int cb_f16;
+    int L, K, T;
+    long long n_blocks;
+    float w_scale;         // log2(e) / tau: branch metrics in log2 units of exp(-J / tau)
+    double tau_ln2;        // tau * ln 2: F = -tau_ln2 * log2 Z
+    float* y;              // [n_blocks, T] soft codewords
+    float* free_energy;    // [n_blocks] or nullptr
+    unsigned char* ws;     // gridDim.x slots of slot_bytes
+    size_t slot_bytes;
+};
+
 // One codebook entry, widened exactly to fp32.
 __device__ __forceinline__ float load_codeword(const void* cb, int f16, uint32_t s)
 {
@@ -150,6 +166,9 @@ const EncodeKernelInfo* find_grouped_kernel(int L, int K, int cb_f16);
 const EncodeKernelInfo* generic_kernel_info(int L, int K);
 
 cudaError_t launch_feedback(const FeedbackArgs& a, cudaStream_t stream);
+size_t bcjr_slot_bytes(int L, int K, int T);
+int bcjr_ctas_per_sm(int L, int K, int cb_f16);
+cudaError_t launch_bcjr(const BcjrArgs& a, int grid, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, int num_sms, cudaStream_t stream);
 cudaError_t launch_gemv(const GemvArgs& a, int num_sms, cudaStream_t stream);
 

@@ -65,6 +65,13 @@ long long wanted_ctas(const EncodeKernelInfo* info, int L, int k, int T, long lo
     return by_blocks < resident ? by_blocks : resident;
 }
 
+long long bcjr_grid(int L, int k, long long n_blocks, tcq_dtype dt, int sms)
+{
+    const long long resident =
+        (long long)(sms > 0 ? sms : 148) * bcjr_ctas_per_sm(L, k, dt == TCQ_F16 ? 1 : 0);
+    return n_blocks < resident ? n_blocks : resident;
+}
+
 // Plans the grid for an encode whose arguments are filled in (all but the
 // workspace) and launches it.
 tcq_status run_encode(EncodeArgs& a, tcq_dtype cb_dtype, void* workspace, size_t workspace_bytes,
@@ -319,6 +326,58 @@ tcq_status tcq_ldlq(const float* w, const float* u, const float* d, const void* 
         if (launch_decode(dq, sms, st) != cudaSuccess) return TCQ_ERR_CUDA;
     }
     return TCQ_OK;
+}
+
+size_t tcq_bcjr_workspace_bytes(int L, int k, int T, int64_t n_blocks, tcq_dtype cb_dtype)
+{
+    if (check_shape(L, k, T) != TCQ_OK || n_blocks <= 0 || !valid_dtype(cb_dtype)) return 0;
+    return (size_t)bcjr_grid(L, k, n_blocks, cb_dtype, current_sms()) * bcjr_slot_bytes(L, k, T);
+}
+
+tcq_status tcq_bcjr(const float* x, const float* d, const void* codebook, tcq_dtype cb_dtype,
+                    int L, int k, int T, int64_t n_blocks, float tau, float* y_soft,
+                    float* free_energy, void* workspace, size_t workspace_bytes,
+                    tcq_stream_t stream)
+{
+    if (n_blocks < 0) return TCQ_ERR_INVALID_ARG;
+    if (!valid_dtype(cb_dtype)) return TCQ_ERR_INVALID_ARG;
+    const tcq_status shape = check_shape(L, k, T);
+    if (shape != TCQ_OK) return shape;
+    if (!(tau > 0.f) || !(tau < INFINITY)) return TCQ_ERR_INVALID_ARG;
+    if (n_blocks == 0) return TCQ_OK;
+    if (!x || !codebook || !y_soft || !workspace) return TCQ_ERR_INVALID_ARG;
+    const size_t entry = cb_dtype == TCQ_F16 ? 2 : 4;
+    if (!aligned(x, 4) || (d && !aligned(d, 4)) || !aligned(codebook, entry) ||
+        !aligned(y_soft, 4) || (free_energy && !aligned(free_energy, 4)) ||
+        !aligned(workspace, 256))
+        return TCQ_ERR_INVALID_ARG;
+    if ((unsigned long long)n_blocks > (1ull << 40)) return TCQ_ERR_INVALID_ARG;
+    const int sms = current_sms();
+    if (sms <= 0) return TCQ_ERR_CUDA;
+    const size_t slot = bcjr_slot_bytes(L, k, T);
+    long long grid = bcjr_grid(L, k, n_blocks, cb_dtype, sms);
+    const long long fit = (long long)(workspace_bytes / slot);
+    if (fit < 1) return TCQ_ERR_WORKSPACE;
+    if (grid > fit) grid = fit;
+    if (grid < 1) grid = 1;
+    BcjrArgs a;
+    a.x = x;
+    a.d = d;
+    a.cb = codebook;
+    a.cb_f16 = cb_dtype == TCQ_F16 ? 1 : 0;
+    a.L = L;
+    a.K = k;
+    a.T = T;
+    a.n_blocks = n_blocks;
+    a.w_scale = (float)(1.4426950408889634 / (double)tau);
+    if (!(a.w_scale < INFINITY)) return TCQ_ERR_INVALID_ARG;
+    a.tau_ln2 = (double)tau * 0.6931471805599453;
+    a.y = y_soft;
+    a.free_energy = free_energy;
+    a.ws = static_cast<unsigned char*>(workspace);
+    a.slot_bytes = slot;
+    const cudaError_t e = launch_bcjr(a, (int)grid, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TCQ_OK : TCQ_ERR_CUDA;
 }
 
 const char* tcq_status_string(tcq_status status)

@@ -71,6 +71,10 @@ def load_library() -> ctypes.CDLL:
     lib.tcq_ldlq.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, i64, i64, vp, vp, vp, vp, vp, vp,
                              sz, vp]
     lib.tcq_ldlq.restype = ci
+    lib.tcq_bcjr_workspace_bytes.argtypes = [ci, ci, ci, i64, ci]
+    lib.tcq_bcjr_workspace_bytes.restype = sz
+    lib.tcq_bcjr.argtypes = [vp, vp, vp, ci, ci, ci, ci, i64, ctypes.c_float, vp, vp, vp, sz, vp]
+    lib.tcq_bcjr.restype = ci
     _lib = lib
     return lib
 
@@ -118,6 +122,16 @@ def tcq_ldlq(w, u, d, codebook, cb_dtype, L, k, T, rows, cols, q, x, start_state
     return int(load_library().tcq_ldlq(w, u, d, codebook, cb_dtype, L, k, T, rows, cols, q, x,
                                        start_state, bits, path_cost, workspace, workspace_bytes,
                                        stream))
+
+
+def tcq_bcjr_workspace_bytes(L: int, k: int, T: int, n_blocks: int, cb_dtype: int) -> int:
+    return int(load_library().tcq_bcjr_workspace_bytes(L, k, T, n_blocks, cb_dtype))
+
+
+def tcq_bcjr(x, d, codebook, cb_dtype, L, k, T, n_blocks, tau, y_soft, free_energy, workspace,
+             workspace_bytes, stream) -> int:
+    return int(load_library().tcq_bcjr(x, d, codebook, cb_dtype, L, k, T, n_blocks, tau, y_soft,
+                                       free_energy, workspace, workspace_bytes, stream))
 
 
 def tcq_status_string(status: int) -> str:
@@ -278,6 +292,30 @@ def ldlq(w, u, d, codebook, L: int, k: int, T: int, keep_targets: bool = True, w
                     _ptr(coded.path_cost), ctypes.c_void_p(workspace.data_ptr()),
                     workspace.numel(), _stream_handle(stream)), "tcq_ldlq")
     return LdlqResult(q, x, coded)
+
+
+def bcjr(x, d, codebook, L: int, k: int, tau: float, workspace=None, out=None, stream=None):
+    """Soft codewords [n_blocks, T] and free energies -tau ln Z [n_blocks] of the
+    rows of ``x`` (fp32 CUDA [n_blocks, T]) at temperature ``tau``."""
+    torch = _torch()
+    if x.dim() != 2 or x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous float32 CUDA tensor [n_blocks, T]")
+    n, T = x.shape
+    if d is not None and (d.shape != x.shape or d.dtype != torch.float32 or not d.is_contiguous()):
+        raise ValueError("d must be None or a contiguous float32 tensor shaped like x")
+    if out is None:
+        out = (torch.empty((n, T), dtype=torch.float32, device=x.device),
+               torch.empty(n, dtype=torch.float32, device=x.device))
+    y, F = out
+    if y.numel() < n * T or (F is not None and F.numel() < n):
+        raise ValueError("bcjr: output tensors too small")
+    if workspace is None:
+        nbytes = max(tcq_bcjr_workspace_bytes(L, k, T, n, cb_dtype_of(codebook)), 256)
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
+    _check(tcq_bcjr(_ptr(x), _ptr(d), _ptr(codebook), cb_dtype_of(codebook), L, k, T, n,
+                    float(tau), _ptr(y), _ptr(F), ctypes.c_void_p(workspace.data_ptr()),
+                    workspace.numel(), _stream_handle(stream)), "tcq_bcjr")
+    return y, F
 
 
 class HostPipeline:
