@@ -46,6 +46,11 @@ CASES = [
     (2, 1, 7, 8, "f32", True, 0.05),      # the 2-bit post's toy trellis
     (3, 1, 1, 5, "f32", True, 0.7),       # T = 1
     (10, 2, 300, 3, "f32", True, 0.02),   # cold: close to the hard code
+    # the register-resident kernel (L=16, k=2, binary16 codebook, T <= 1024)
+    (16, 2, 256, 3, "f16", True, 0.1),
+    (16, 2, 7, 5, "f16", False, 0.5),
+    (16, 2, 1, 4, "f16", True, 0.3),
+    (16, 2, 64, 2, "f16", True, 0.003),
 ]
 
 
@@ -120,3 +125,27 @@ def test_bcjr_small_workspace_and_rejections(cuda_device):
                                                                  device=cuda_device))
     y0, F0 = tcq.bcjr(torch.zeros((0, T), device=cuda_device), None, ct, L, k, 0.5)
     assert y0.shape == (0, T)
+
+
+def test_bcjr_register_kernel_loops_over_blocks(cuda_device):
+    """A workspace of one slot makes one CTA take every block in turn: the same
+    results as one CTA per block, and the oracle's on a sample."""
+    import torch
+    from oracle import oracle_bcjr
+    from trellis_coded_weight_tcq_b200 import tcq
+
+    L, k, T, n = 16, 2, 48, 5
+    rng = np.random.default_rng(79)
+    x = rng.standard_normal((n, T)).astype(np.float32)
+    d = rng.lognormal(0.0, 1.0, (n, T)).astype(np.float32)
+    cb = rng.standard_normal(1 << L).astype(np.float16)
+    y_ref, F_ref = _run(x, d, cb, L, k, 0.2, cuda_device)
+    one = tcq.tcq_bcjr_workspace_bytes(L, k, T, 1, tcq.TCQ_F16)
+    ws = torch.empty(one, dtype=torch.uint8, device=cuda_device)
+    y1, F1 = _run(x, d, cb, L, k, 0.2, cuda_device, workspace=ws)
+    np.testing.assert_array_equal(y1, y_ref)
+    np.testing.assert_array_equal(F1, F_ref)
+    y_o, F_o = oracle_bcjr(x[[0, 4]], d[[0, 4]], cb, L, k, 0.2)
+    y_tol, F_tol = _tolerances(T, cb.astype(np.float64), F_o, 0.2)
+    assert np.abs(y1[[0, 4]] - y_o).max() <= y_tol
+    assert np.all(np.abs(F1[[0, 4]] - F_o) <= F_tol)

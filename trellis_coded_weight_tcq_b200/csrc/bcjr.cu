@@ -272,6 +272,11 @@ cudaError_t launch_tab(const BcjrArgs& a, int grid, cudaStream_t stream)
 
 }  // namespace
 
+// bcjr_grouped.cu: the register-resident kernel for the shapes it is compiled for
+cudaError_t launch_bcjr_grouped(const BcjrArgs& a, int grid, cudaStream_t stream, bool* handled);
+
+// A slot serves either kernel (the register-resident one needs only the
+// forward values, the first part of this layout).
 size_t bcjr_slot_bytes(int L, int K, int T)
 {
     return s_bytes(L, K, T) + r_bytes(L, K) + round256((size_t)T * sizeof(double));
@@ -285,6 +290,9 @@ int bcjr_ctas_per_sm(int L, int, int cb_f16)
 
 cudaError_t launch_bcjr(const BcjrArgs& a, int grid, cudaStream_t stream)
 {
+    bool handled = false;
+    const cudaError_t eg = launch_bcjr_grouped(a, grid, stream, &handled);
+    if (handled || eg != cudaSuccess) return eg;
     int mode = table_mode(a.L, a.cb_f16);
     if (mode == kTabF16 && (reinterpret_cast<uintptr_t>(a.cb) & 15) != 0) mode = kTabGlobal;
     switch (mode) {
