@@ -29,6 +29,8 @@ sys.path.insert(0, ROOT)
 METRIC = "Viterbi trellis nodes/sec (blocks·T·2^L) and weights encoded/sec at L=16,k=2"
 ALGO_OPS_PER_NODE = 3  # error, square-accumulate, compare-select
 SMS, LANES_PER_SM = 148, 128
+SFU_PER_SM = 16  # ex2 / lg2 results per SM per clock (4 per sub-partition)
+BCJR_TAU = 0.1
 ROOFLINE_SRC = ["trellis_coded_weight_tcq_b200/csrc/acs_grouped.cuh",
                 "trellis_coded_weight_tcq_b200/csrc/acs_grouped.cu",
                 "trellis_coded_weight_tcq_b200/csrc/common.cuh"]
@@ -395,6 +397,38 @@ def run_ours(args, rank, world, local_rank):
                 "proxy_loss_per_weight": float(costs.astype(np.float64).sum()) / (lw.rows * lw.cols)}
         del w_t, u_t, d_t, lws, res
 
+    # ---- soft forward-backward quantization of the same blocks at tau = 0.1
+    bcjr = None
+    if rank == 0 and world == 1 and not args.no_bcjr:
+        torch.cuda.empty_cache()
+        xb_t = torch.from_numpy(wl.x).to(dev)
+        db_t = None if wl.d is None else torch.from_numpy(wl.d).to(dev)
+        bws = torch.empty(tcq.tcq_bcjr_workspace_bytes(L, k, T, n, tcq.cb_dtype_of(cb)),
+                          dtype=torch.uint8, device=dev)
+        yb = torch.empty((n, T), dtype=torch.float32, device=dev)
+        fb = torch.empty(n, dtype=torch.float32, device=dev)
+        tcq.bcjr(xb_t, db_t, cb, L, k, BCJR_TAU, workspace=bws, out=(yb, fb))
+        a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        tcq.bcjr(xb_t, db_t, cb, L, k, BCJR_TAU, workspace=bws, out=(yb, fb))
+        b2.record(stream)
+        torch.cuda.synchronize()
+        b_ms = a.elapsed_time(b2)
+        fe = fb.cpu().numpy()
+        assert np.all(np.isfinite(fe)) and bool(torch.isfinite(yb).all())
+        peaks_b, kind_b = _peaks()
+        sfu_peak = SMS * SFU_PER_SM * float(peaks_b.get("sm_max_mhz", 1965.0)) * 1e6
+        sfu_ops = wl.nodes * (2.0 + 3.0 / (1 << k))
+        bcjr = {"workload": wl.name, "tau": BCJR_TAU, "ms": b_ms,
+                "nodes_per_s": wl.nodes / (b_ms / 1e3), "weights_per_s": wl.weights / (b_ms / 1e3),
+                "bound": "sfu", "sfu_ops_per_node": 2.0 + 3.0 / (1 << k),
+                "achieved": sfu_ops / (b_ms / 1e3) / 1e12, "peak": sfu_peak / 1e12, "unit": "TOP/s",
+                "frac": sfu_ops / (b_ms / 1e3) / sfu_peak,
+                "peak_basis": f"{SMS} SMs x {SFU_PER_SM} ex2/lg2 per clock x "
+                              f"{peaks_b.get('sm_max_mhz', 1965.0)} MHz ({kind_b} max SM clock)",
+                "free_energy_mean": float(fe.astype(np.float64).mean())}
+        del xb_t, db_t, bws, yb, fb
+
     # sanity: the last step's result is a valid encode of the workload (cheap host check)
     cost_h = cost_last
     assert np.all(np.isfinite(cost_h)) and np.all(cost_h >= 0)
@@ -445,7 +479,7 @@ def run_ours(args, rank, world, local_rank):
         "weights_per_s": world * wl.weights / (ms / 1e3),
         "encode_ms_per_step": acs_ms, "decode_ms_per_step": dec_ms,
         "roofline": roofline, "decode_roofline": decode_roofline, "cpu_baseline": cpu_baseline, "e2e": e2e,
-        "per_workload": per_workload, "gemv": gemv, "ldlq": ldlq,
+        "per_workload": per_workload, "gemv": gemv, "ldlq": ldlq, "bcjr": bcjr,
         "clocks": clocks.summary(), "gpu_launches": gpu_launches,
     }
     print(json.dumps(line), flush=True)
@@ -462,6 +496,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-workload", action="store_true",
                     help="skip the short encode/decode timing of the other named workloads")
+    ap.add_argument("--no-bcjr", action="store_true",
+                    help="skip the soft forward-backward quantization of the workload")
     ap.add_argument("--no-ldlq", action="store_true",
                     help="skip the error-feedback encode of the MLP matrix")
     ap.add_argument("--cpu-blocks-per-core", type=int, default=4)
