@@ -117,6 +117,22 @@ tcq_status tcq_encode(const float* x, const float* d, const void* codebook, tcq_
                       tcq_stream_t stream);
 
 /*
+ * Encode with the start state of every block fixed instead of free (the 2-bit
+ * post's trellis toy starts in state 0; CurveTQ's free start per coding block
+ * is tcq_encode).  Block b minimises J over bitstreams alone from
+ * s_0 = fixed_start[b]; only the low L-k bits of fixed_start[b] matter, and the
+ * returned start_state[b] equals them.
+ *
+ *   fixed_start  uint32 [n_blocks], device, 4-byte aligned, not NULL.
+ * Everything else, including the workspace and the error codes, as tcq_encode.
+ */
+tcq_status tcq_encode_fixed_start(const float* x, const float* d, const void* codebook,
+                                  tcq_dtype cb_dtype, int L, int k, int T, int64_t n_blocks,
+                                  const uint32_t* fixed_start, uint32_t* start_state,
+                                  uint32_t* bits, float* path_cost, void* workspace,
+                                  size_t workspace_bytes, tcq_stream_t stream);
+
+/*
  * Decode (the 2-bit post's state-tracking table-lookup decoder; QTIP's
  * stateful bitshift decoder): y[b, t-1] = c[s_t] with s_t the last L bits of
  * (start_state[b] || stream[0, tk)).  Bit-exact: y is the exact fp32 widening

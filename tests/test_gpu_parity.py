@@ -54,7 +54,7 @@ def test_named_workload_full_size_sampled(name):
     dt = tcq.TCQ_F16 if wl.codebook.dtype == np.float16 else tcq.TCQ_F32
     assert tcq.tcq_encode_path(wl.L, wl.k, dt).startswith("grouped")
     start, bits, cost = gpu_encode(wl)
-    rows = _sample_rows(wl.n_blocks, 48, 7)
+    rows = _sample_rows(wl.n_blocks, 256, 7)  # first, last and 254 seeded
     check_encode(wl, start, bits, cost, rows=rows)
     y = gpu_decode(bits, start, wl.codebook, wl.L, wl.k, wl.T)
     y_o = oracle_decode(bits[rows], start[rows], wl.codebook, wl.L, wl.k, wl.T).astype(np.float32)

@@ -58,6 +58,8 @@ __global__ void __launch_bounds__(kGenericThreads) acs_generic_kernel(EncodeArgs
         const float* db = a.d ? a.d + b * a.d_stride : nullptr;
         float bestv = __int_as_float(0x7f800000);
         uint32_t bests = 0xffffffffu;
+        // a fixed start s_0 leaves only its successors reachable at step 1
+        const uint32_t s0 = a.fixed_start ? (a.fixed_start[b] & (NU - 1u)) : 0xffffffffu;
         for (int t = 1; t <= T; ++t) {
             const float sd = db ? sqrtf(db[t - 1]) : 1.f;
             const float ca = -sd, cx = sd * xb[t - 1];
@@ -69,7 +71,8 @@ __global__ void __launch_bounds__(kGenericThreads) acs_generic_kernel(EncodeArgs
                 for (int h = 0; h < H; ++h) {
                     const uint32_t s = ((uint32_t)h << LK) | u;
                     const float e = fmaf(ca, load_codeword(a.cb, a.cb_f16, s), cx);
-                    const float v = fmaf(e, e, t == 1 ? 0.f : Mp[s >> K]);
+                    const float m0 = (s0 == 0xffffffffu || (s >> K) == s0) ? 0.f : __int_as_float(0x7f800000);
+                    const float v = fmaf(e, e, t == 1 ? m0 : Mp[s >> K]);
                     if (v < best) {
                         best = v;
                         bh = (uint32_t)h;

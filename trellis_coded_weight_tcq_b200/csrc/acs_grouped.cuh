@@ -230,7 +230,9 @@ __device__ __forceinline__ void store_metrics(float* dst, const float (&v)[H])
     }
 }
 
-// One trellis step for one thread.  FIRST: M_0 = 0 (free start).  LAST: no
+// One trellis step for one thread.  FIRST: M_0 = 0 (free start), or, for a
+// start fixed at s_0 (s0 = its low L-k bits), 0 at u = s0 and +inf elsewhere,
+// so only the successors of s_0 are reachable at step 1.  LAST: no
 // metrics or backpointers are stored; the thread keeps its best final state.
 // (p0, p1) is the step's staged pair: (a, xs) for fp32 codewords,
 // (-x_t, d_{t-1} / d_t) for fp16 codewords.  Backpointers come back as K bit planes: bit P-1-q of
@@ -240,7 +242,7 @@ template <class C, bool WEIGHTED, bool FIRST, bool LAST>
 __device__ __forceinline__ void acs_step(const Codewords<C, C::CB16>& cw, float p0, float p1,
                                          const float* __restrict__ Mp, float* __restrict__ Mn,
                                          int tid, uint32_t (&planes)[C::K], float& bestv,
-                                         uint32_t& bests)
+                                         uint32_t& bests, uint32_t s0 = 0xffffffffu)
 {
 #pragma unroll
     for (int l = 0; l < C::K; ++l) planes[l] = 0;
@@ -250,7 +252,11 @@ __device__ __forceinline__ void acs_step(const Codewords<C, C::CB16>& cw, float 
         float Mh[C::H];
 #pragma unroll
         for (int h = 0; h < C::H; ++h) {
-            Mh[h] = FIRST ? 0.f : Mp[(h << (C::L - 2 * C::K)) | g];
+            if constexpr (FIRST)
+                Mh[h] = (s0 == 0xffffffffu || (uint32_t)((h << (C::L - 2 * C::K)) | g) == s0)
+                            ? 0.f : __int_as_float(0x7f800000);
+            else
+                Mh[h] = Mp[(h << (C::L - 2 * C::K)) | g];
             if constexpr (C::CB16 && WEIGHTED) Mh[h] *= p1;  // M_{t-1}/d_{t-1} -> M_{t-1}/d_t
         }
         float mn[C::H];
@@ -505,7 +511,12 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB) acs_grouped_kernel(Encod
                 const float* Mp = Mteam + ((t - 1) & 1) * C::NU;
                 float* Mn = Mteam + (t & 1) * C::NU;
                 uint32_t planes[C::K];
-                acs_step<C, WEIGHTED, FIRST, LAST>(cw, ax.x, ax.y, Mp, Mn, tid, planes, bestv, bests);
+                uint32_t s0 = 0xffffffffu;
+                if constexpr (FIRST) {
+                    if (a.fixed_start) s0 = a.fixed_start[b] & (uint32_t)(C::NU - 1);
+                }
+                acs_step<C, WEIGHTED, FIRST, LAST>(cw, ax.x, ax.y, Mp, Mn, tid, planes, bestv, bests,
+                                                   s0);
                 if constexpr (!LAST) {
                     unit_t rec = 0;
 #pragma unroll

@@ -23,6 +23,7 @@ struct EncodeArgs {
     uint32_t* bits;        // block b at bits + b * out_stride * W
     float* path_cost;      // block b at path_cost[b * out_stride]
     long long x_stride, d_stride, out_stride;
+    const uint32_t* fixed_start;  // block b starts in fixed_start[b] (low L-k bits), or nullptr: free
     unsigned char* ws;     // workspace base: gridDim.x slots of slot_bytes
     size_t slot_bytes;
 };

@@ -154,6 +154,48 @@ tcq_status tcq_encode(const float* x, const float* d, const void* codebook, tcq_
     a.x_stride = T;
     a.d_stride = T;
     a.out_stride = 1;
+    a.fixed_start = nullptr;
+    return run_encode(a, cb_dtype, workspace, workspace_bytes,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+tcq_status tcq_encode_fixed_start(const float* x, const float* d, const void* codebook,
+                                  tcq_dtype cb_dtype, int L, int k, int T, int64_t n_blocks,
+                                  const uint32_t* fixed_start, uint32_t* start_state,
+                                  uint32_t* bits, float* path_cost, void* workspace,
+                                  size_t workspace_bytes, tcq_stream_t stream)
+{
+    if (n_blocks > 0 && (!fixed_start || !aligned(fixed_start, 4))) return TCQ_ERR_INVALID_ARG;
+    if (n_blocks < 0) return TCQ_ERR_INVALID_ARG;
+    if (!valid_dtype(cb_dtype)) return TCQ_ERR_INVALID_ARG;
+    const tcq_status shape = check_shape(L, k, T);
+    if (shape != TCQ_OK) return shape;
+    if (n_blocks == 0) return TCQ_OK;
+    if (!x || !codebook || !start_state || !bits || !path_cost || !workspace)
+        return TCQ_ERR_INVALID_ARG;
+    const size_t entry = cb_dtype == TCQ_F16 ? 2 : 4;
+    if (!aligned(x, 4) || (d && !aligned(d, 4)) || !aligned(codebook, entry) ||
+        !aligned(start_state, 4) || !aligned(bits, 4) || !aligned(path_cost, 4) ||
+        !aligned(workspace, 256))
+        return TCQ_ERR_INVALID_ARG;
+    if ((unsigned long long)n_blocks > (1ull << 40)) return TCQ_ERR_INVALID_ARG;
+    EncodeArgs a;
+    a.x = x;
+    a.d = d;
+    a.cb = codebook;
+    a.cb_f16 = cb_dtype == TCQ_F16 ? 1 : 0;
+    a.L = L;
+    a.K = k;
+    a.T = T;
+    a.W = tcq_words_per_block(k, T);
+    a.n_blocks = n_blocks;
+    a.start_state = start_state;
+    a.bits = bits;
+    a.path_cost = path_cost;
+    a.x_stride = T;
+    a.d_stride = T;
+    a.out_stride = 1;
+    a.fixed_start = fixed_start;
     return run_encode(a, cb_dtype, workspace, workspace_bytes,
                       reinterpret_cast<cudaStream_t>(stream));
 }
@@ -307,6 +349,7 @@ tcq_status tcq_ldlq(const float* w, const float* u, const float* d, const void* 
         a.x_stride = x_ld;
         a.d_stride = 0;
         a.out_stride = nb;
+        a.fixed_start = nullptr;
         const tcq_status es = run_encode(a, cb_dtype, ws + targets, workspace_bytes - targets, st);
         if (es != TCQ_OK) return es;
 

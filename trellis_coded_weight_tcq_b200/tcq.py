@@ -58,6 +58,9 @@ def load_library() -> ctypes.CDLL:
     lib.tcq_encode_workspace_bytes.restype = sz
     lib.tcq_encode.argtypes = [vp, vp, vp, ci, ci, ci, ci, i64, vp, vp, vp, vp, sz, vp]
     lib.tcq_encode.restype = ci
+    lib.tcq_encode_fixed_start.argtypes = [vp, vp, vp, ci, ci, ci, ci, i64, vp, vp, vp, vp, vp,
+                                           sz, vp]
+    lib.tcq_encode_fixed_start.restype = ci
     lib.tcq_decode.argtypes = [vp, vp, vp, ci, ci, ci, ci, i64, vp, vp]
     lib.tcq_decode.restype = ci
     lib.tcq_status_string.argtypes = [ci]
@@ -101,6 +104,13 @@ def tcq_encode(x, d, codebook, cb_dtype, L, k, T, n_blocks, start_state, bits, p
                workspace, workspace_bytes, stream) -> int:
     return int(load_library().tcq_encode(x, d, codebook, cb_dtype, L, k, T, n_blocks, start_state,
                                           bits, path_cost, workspace, workspace_bytes, stream))
+
+
+def tcq_encode_fixed_start(x, d, codebook, cb_dtype, L, k, T, n_blocks, fixed_start, start_state,
+                           bits, path_cost, workspace, workspace_bytes, stream) -> int:
+    return int(load_library().tcq_encode_fixed_start(x, d, codebook, cb_dtype, L, k, T, n_blocks,
+                                                     fixed_start, start_state, bits, path_cost,
+                                                     workspace, workspace_bytes, stream))
 
 
 def tcq_decode(bits, start_state, codebook, cb_dtype, L, k, T, n_blocks, y, stream) -> int:
@@ -192,8 +202,9 @@ class Workspace:
 
 
 def encode(x, d, codebook, L: int, k: int, workspace: Workspace | None = None, out=None,
-           stream=None) -> Encoded:
-    """Viterbi TCQ of every row of ``x`` (fp32 CUDA tensor [n_blocks, T])."""
+           stream=None, fixed_start=None) -> Encoded:
+    """Viterbi TCQ of every row of ``x`` (fp32 CUDA tensor [n_blocks, T]); a free
+    start state per block, or the int32 tensor ``fixed_start`` of start states."""
     torch = _torch()
     if x.dim() != 2 or x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
         raise ValueError("x must be a contiguous float32 CUDA tensor [n_blocks, T]")
@@ -210,10 +221,19 @@ def encode(x, d, codebook, L: int, k: int, workspace: Workspace | None = None, o
             torch.empty(n, dtype=torch.float32, device=x.device),
         )
     ws = workspace or Workspace(L, k, T, n, cb_dtype_of(codebook), x.device)
-    _check(tcq_encode(_ptr(x), _ptr(d), _ptr(codebook), cb_dtype_of(codebook), L, k, T, n,
-                      _ptr(out.start_state), _ptr(out.bits), _ptr(out.path_cost),
-                      ctypes.c_void_p(ws.buf.data_ptr()), ws.nbytes, _stream_handle(stream)),
-           "tcq_encode")
+    if fixed_start is None:
+        _check(tcq_encode(_ptr(x), _ptr(d), _ptr(codebook), cb_dtype_of(codebook), L, k, T, n,
+                          _ptr(out.start_state), _ptr(out.bits), _ptr(out.path_cost),
+                          ctypes.c_void_p(ws.buf.data_ptr()), ws.nbytes, _stream_handle(stream)),
+               "tcq_encode")
+    else:
+        if fixed_start.numel() < n or fixed_start.dtype != torch.int32 or not fixed_start.is_cuda:
+            raise ValueError("fixed_start must be an int32 CUDA tensor of n_blocks start states")
+        _check(tcq_encode_fixed_start(_ptr(x), _ptr(d), _ptr(codebook), cb_dtype_of(codebook), L,
+                                      k, T, n, _ptr(fixed_start), _ptr(out.start_state),
+                                      _ptr(out.bits), _ptr(out.path_cost),
+                                      ctypes.c_void_p(ws.buf.data_ptr()), ws.nbytes,
+                                      _stream_handle(stream)), "tcq_encode_fixed_start")
     return out
 
 
