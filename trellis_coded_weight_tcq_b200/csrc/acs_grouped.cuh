@@ -426,7 +426,9 @@ __device__ __forceinline__ float team_max(float v, float* redv, int m)
     }
 }
 
-template <class C, bool WEIGHTED>
+// FIXED: every block starts in a.fixed_start[b] (a separate instantiation, so the
+// free-start kernel carries none of it).
+template <class C, bool WEIGHTED, bool FIXED = false>
 __global__ void __launch_bounds__(C::NTHREADS, C::MINB) acs_grouped_kernel(EncodeArgs a)
 {
     using unit_t = typename C::unit_t;
@@ -512,9 +514,7 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB) acs_grouped_kernel(Encod
                 float* Mn = Mteam + (t & 1) * C::NU;
                 uint32_t planes[C::K];
                 uint32_t s0 = 0xffffffffu;
-                if constexpr (FIRST) {
-                    if (a.fixed_start) s0 = a.fixed_start[b] & (uint32_t)(C::NU - 1);
-                }
+                if constexpr (FIRST && FIXED) s0 = a.fixed_start[b] & (uint32_t)(C::NU - 1);
                 acs_step<C, WEIGHTED, FIRST, LAST>(cw, ax.x, ax.y, Mp, Mn, tid, planes, bestv, bests,
                                                    s0);
                 if constexpr (!LAST) {
@@ -602,14 +602,14 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB) acs_grouped_kernel(Encod
     }
 }
 
-template <class C, bool WEIGHTED>
+template <class C, bool WEIGHTED, bool FIXED = false>
 cudaError_t launch_grouped_w(const EncodeArgs& a, int grid, cudaStream_t stream)
 {
     const size_t smem = C::smem_bytes(a.L, a.K, a.T);
-    cudaError_t e = cudaFuncSetAttribute(acs_grouped_kernel<C, WEIGHTED>,
+    cudaError_t e = cudaFuncSetAttribute(acs_grouped_kernel<C, WEIGHTED, FIXED>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    acs_grouped_kernel<C, WEIGHTED><<<grid, C::NTHREADS, smem, stream>>>(a);
+    acs_grouped_kernel<C, WEIGHTED, FIXED><<<grid, C::NTHREADS, smem, stream>>>(a);
     return cudaGetLastError();
 }
 
@@ -619,6 +619,8 @@ cudaError_t launch_grouped(const EncodeArgs& a, int grid, cudaStream_t stream)
     // The fp16-pair kernels always run the weighted form (an absent d reads as 1,
     // every ratio d_{t-1}/d_t is then 1): measured faster than a separate
     // unweighted instantiation, whose schedule came out worse.
+    if (a.fixed_start)  // weighted form: an absent d reads as 1
+        return launch_grouped_w<C, true, true>(a, grid, stream);
     if constexpr (C::CB16)
         return launch_grouped_w<C, true>(a, grid, stream);
     else
