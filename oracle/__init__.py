@@ -13,6 +13,7 @@ from .tcq_oracle import (  # noqa: F401
     oracle_gemv,
     oracle_greedy,
     oracle_ldlq,
+    oracle_mad_codebook,
     oracle_path_cost,
     oracle_words_per_block,
 )

@@ -463,3 +463,29 @@ int oracle_bcjr(const double* x, const double* d, const double* cb, int L, int k
     free(lb);
     return ORACLE_OK;
 }
+
+/*
+ * A computed ("lookup-free") code: the codeword of a state is computed from the
+ * state's bits instead of read from a table.  "QTIP: Quantization with
+ * Trellises and Incoherence Processing" (abstract) introduces codes from
+ * lookup-only to computed lookup-free for the bitshift trellis and gives no
+ * formula; the code here is this library's reading: a multiplicative hash of
+ * the state (its high half is a well-mixed function of every state bit) and
+ * the sum of that half's two bytes (a triangular, roughly bell-shaped value),
+ * centred and scaled by a power of two so that every codeword is exact in
+ * binary16:
+ *     v    = (A s) mod 2^32,   A = 0x9E3779B1
+ *     c[s] = (v_2 + v_3 - 255) / 128,   v_2, v_3 bits 16..23 and 24..31 of v.
+ * Writes the 2^L codewords to cb.
+ */
+int oracle_mad_codebook(int L, double* cb)
+{
+    if (L < 1 || L > 20 || !cb) return ORACLE_EINVAL;
+    const uint32_t A = 0x9E3779B1u;
+    for (uint32_t s = 0; s < (1u << L); ++s) {
+        const uint32_t v = A * s; /* unsigned arithmetic wraps mod 2^32 */
+        const int sum = (int)((v >> 16) & 0xFFu) + (int)(v >> 24);
+        cb[s] = (double)(sum - 255) / 128.0;
+    }
+    return ORACLE_OK;
+}

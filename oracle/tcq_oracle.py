@@ -56,6 +56,8 @@ def _load():
         lib.oracle_feedback.restype = ci
         lib.oracle_bcjr.argtypes = [dp, dp, dp, ci, ci, ci, i64, ctypes.c_double, dp, dp]
         lib.oracle_bcjr.restype = ci
+        lib.oracle_mad_codebook.argtypes = [ci, dp]
+        lib.oracle_mad_codebook.restype = ci
         _lib = lib
     return _lib
 
@@ -255,3 +257,12 @@ def oracle_bcjr(x, d, codebook, L: int, k: int, tau: float):
     if rc != 0:
         raise ValueError(f"oracle_bcjr failed with code {rc}")
     return y, F
+
+
+def oracle_mad_codebook(L: int):
+    """The 2^L codewords of the computed multiply-add code (fp64)."""
+    cb = np.zeros(1 << L)
+    rc = _load().oracle_mad_codebook(L, _ptr(cb, ctypes.c_double))
+    if rc != 0:
+        raise ValueError(f"oracle_mad_codebook failed with code {rc}")
+    return cb
