@@ -69,8 +69,23 @@ typedef enum {
 
 typedef enum {
     TCQ_F32 = 0, /* codebook entries are IEEE binary32 */
-    TCQ_F16 = 1  /* codebook entries are IEEE binary16 */
+    TCQ_F16 = 1, /* codebook entries are IEEE binary16 */
+    TCQ_MAD = 2  /* no table: the computed code below; the codebook pointer is
+                    ignored and may be NULL */
 } tcq_dtype;
+
+/*
+ * The computed (lookup-free) code selected by TCQ_MAD.  QTIP (abstract)
+ * introduces codes for the bitshift trellis from lookup-only tables to
+ * codewords computed from the state, without a formula; this library's code is
+ *     v = 0x9E3779B1 * s mod 2^32,   c[s] = (v_2 + v_3 - 255) / 128
+ * with v_2, v_3 bits 16..23 and 24..31 of v: a multiplicative hash of the state
+ * and the sum of its high two bytes, every codeword exact in binary16.  Decode
+ * and the matrix-vector product compute it per weight; the encoders and the
+ * soft quantizer write it as a binary16 table to the front of their workspace
+ * (the workspace queries include it) and then run as for TCQ_F16.
+ */
+#define TCQ_MAD_MULTIPLIER 0x9E3779B1u
 
 /* Supported ranges: 1 <= k <= TCQ_MAX_K, k <= L <= TCQ_MAX_L, 1 <= T <= TCQ_MAX_T. */
 #define TCQ_MAX_L 16

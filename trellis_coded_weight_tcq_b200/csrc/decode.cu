@@ -12,13 +12,13 @@
 // fits in 64 KiB, else as binary16 when the input is binary16); a binary32
 // codebook too large for that is gathered through L1.  The kernel reads k/8
 // bytes and writes 4 bytes per weight: HBM bound.
-#include "common.cuh"
+#include "codes.cuh"
 
 namespace tcq {
 
 namespace {
 
-enum TableMode { kTableF32 = 0, kTableF16 = 1, kTableGlobal = 2 };
+enum TableMode { kTableF32 = 0, kTableF16 = 1, kTableGlobal = 2, kTableMad = 3 };
 
 constexpr int kDecodeThreads = 1024;
 
@@ -57,6 +57,8 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a)
             return reinterpret_cast<const float*>(dsm)[s];
         else if constexpr (MODE == kTableF16)
             return __half2float(reinterpret_cast<const __half*>(dsm)[s]);
+        else if constexpr (MODE == kTableMad)
+            return mad_codeword(s);
         else
             return load_codeword(a.cb, a.cb_f16, s);
     };
@@ -154,7 +156,10 @@ cudaError_t launch_decode(const DecodeArgs& a, int num_sms, cudaStream_t stream)
     const size_t entries = (size_t)1 << a.L;
     int mode;
     size_t smem;
-    if (entries * 4 <= 64 * 1024) {
+    if (a.cb_f16 == kMadCodebook) {
+        mode = kTableMad;
+        smem = 0;
+    } else if (entries * 4 <= 64 * 1024) {
         mode = kTableF32;
         smem = entries * 4;
     } else if (a.cb_f16) {
@@ -180,7 +185,9 @@ cudaError_t launch_decode(const DecodeArgs& a, int num_sms, cudaStream_t stream)
     case 2: return launch_mode<kTableF16, false>(a, (int)grid, smem, stream);
     case 3: return launch_mode<kTableF16, true>(a, (int)grid, smem, stream);
     case 4: return launch_mode<kTableGlobal, false>(a, (int)grid, smem, stream);
-    default: return launch_mode<kTableGlobal, true>(a, (int)grid, smem, stream);
+    case 5: return launch_mode<kTableGlobal, true>(a, (int)grid, smem, stream);
+    case 6: return launch_mode<kTableMad, false>(a, (int)grid, smem, stream);
+    default: return launch_mode<kTableMad, true>(a, (int)grid, smem, stream);
     }
 }
 

@@ -17,7 +17,7 @@
 // lookups.  Per weight: a window extract, a table lookup (random addresses, so
 // shared-memory bank conflicts bound the kernel), a widening and an FMA; the
 // bits are k/8 bytes per weight from HBM.
-#include "common.cuh"
+#include "codes.cuh"
 
 namespace tcq {
 
@@ -26,15 +26,23 @@ namespace {
 constexpr int kGemvThreads = 1024;
 constexpr int kGemvUnroll = 4;
 
-template <bool CB16, bool XSMEM>
+// CODE: kCodeF32 / kCodeF16 (the table staged in shared memory as fp32 or
+// binary16) or kCodeMad (the computed code, no table).
+enum GemvCode { kCodeF32 = 0, kCodeF16 = 1, kCodeMad = 2 };
+
+template <int CODE, bool XSMEM>
 __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(GemvArgs a)
 {
+    constexpr bool CB16 = CODE == kCodeF16;
     extern __shared__ __align__(16) unsigned char gsm[];
     const int n_entries = 1 << a.L;
-    const size_t tab_bytes = (size_t)n_entries * (CB16 ? 2 : 4);
+    const size_t tab_bytes = CODE == kCodeMad ? 0 : (size_t)n_entries * (CB16 ? 2 : 4);
     float* xs = reinterpret_cast<float*>(gsm + ((tab_bytes + 15) & ~(size_t)15));
     // stage the codebook (16-byte copies when possible) and x
-    {
+    if constexpr (CODE == kCodeMad) {
+        if constexpr (XSMEM)
+            for (long long i = threadIdx.x; i < a.cols; i += blockDim.x) xs[i] = a.x[i];
+    } else {
         const unsigned char* src = reinterpret_cast<const unsigned char*>(a.cb);
         if (CB16 || !a.cb_f16) {  // same representation in and out
             if ((reinterpret_cast<uintptr_t>(src) & 15) == 0 && tab_bytes % 16 == 0) {
@@ -121,7 +129,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(GemvArgs a)
             for (int e = 0; e < 4; ++e) {
                 const uint32_t top = e == 0 ? ahi : __funnelshift_l(alo, ahi, e * K);  // e k <= 12
                 const uint32_t s = top >> (32 - L);
-                if constexpr (CB16)
+                if constexpr (CODE == kCodeMad)
+                    c[e] = mad_codeword(s);
+                else if constexpr (CB16)
                     c[e] = __half2float(reinterpret_cast<const __half*>(gsm)[s]);
                 else
                     c[e] = reinterpret_cast<const float*>(gsm)[s];
@@ -162,17 +172,21 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(GemvArgs a)
 // state windows all lie in the high word of the 64-bit read once it is aligned
 // to the first window, (N-1)k + L <= 32, so a state is one shift and one mask.
 // Everything else as gemv_kernel; each item's sum runs as two FMA chains.
-template <int L, int K, int N, bool CB16, bool XSMEM>
+template <int L, int K, int N, int CODE, bool XSMEM>
 __global__ void __launch_bounds__(kGemvThreads, 1) gemv_fast_kernel(GemvArgs a)
 {
     static_assert((N - 1) * K + L <= 32 && N % 4 == 0, "item windows must share one word");
+    constexpr bool CB16 = CODE == kCodeF16;
     constexpr int U = 2;  // items per lane per fetch
     constexpr uint32_t MASK = (1u << L) - 1u;
     extern __shared__ __align__(16) unsigned char gsm[];
     const int n_entries = 1 << L;
-    const size_t tab_bytes = (size_t)n_entries * (CB16 ? 2 : 4);
+    const size_t tab_bytes = CODE == kCodeMad ? 0 : (size_t)n_entries * (CB16 ? 2 : 4);
     float* xs = reinterpret_cast<float*>(gsm + ((tab_bytes + 15) & ~(size_t)15));
-    {
+    if constexpr (CODE == kCodeMad) {
+        if constexpr (XSMEM)
+            for (long long i = threadIdx.x; i < a.cols; i += blockDim.x) xs[i] = a.x[i];
+    } else {
         const unsigned char* src = reinterpret_cast<const unsigned char*>(a.cb);
         if (CB16 || !a.cb_f16) {
             if ((reinterpret_cast<uintptr_t>(src) & 15) == 0 && tab_bytes % 16 == 0) {
@@ -243,7 +257,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_fast_kernel(GemvArgs a)
 #pragma unroll
             for (int e = 0; e < N; ++e) {
                 const uint32_t s = (w >> (32 - L - e * K)) & MASK;
-                if constexpr (CB16)
+                if constexpr (CODE == kCodeMad)
+                    c[e] = mad_codeword(s);
+                else if constexpr (CB16)
                     c[e] = __half2float(reinterpret_cast<const __half*>(gsm)[s]);
                 else
                     c[e] = reinterpret_cast<const float*>(gsm)[s];
@@ -297,23 +313,23 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_fast_kernel(GemvArgs a)
     }
 }
 
-template <int L, int K, int N, bool CB16, bool XSMEM>
+template <int L, int K, int N, int CODE, bool XSMEM>
 cudaError_t launch_gemv_fast_t(const GemvArgs& a, int grid, size_t smem, cudaStream_t stream)
 {
-    cudaError_t e = cudaFuncSetAttribute(gemv_fast_kernel<L, K, N, CB16, XSMEM>,
+    cudaError_t e = cudaFuncSetAttribute(gemv_fast_kernel<L, K, N, CODE, XSMEM>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    gemv_fast_kernel<L, K, N, CB16, XSMEM><<<grid, kGemvThreads, smem, stream>>>(a);
+    gemv_fast_kernel<L, K, N, CODE, XSMEM><<<grid, kGemvThreads, smem, stream>>>(a);
     return cudaGetLastError();
 }
 
-template <bool CB16, bool XSMEM>
+template <int CODE, bool XSMEM>
 cudaError_t launch_gemv_t(const GemvArgs& a, int grid, size_t smem, cudaStream_t stream)
 {
-    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<CB16, XSMEM>,
+    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<CODE, XSMEM>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    gemv_kernel<CB16, XSMEM><<<grid, kGemvThreads, smem, stream>>>(a);
+    gemv_kernel<CODE, XSMEM><<<grid, kGemvThreads, smem, stream>>>(a);
     return cudaGetLastError();
 }
 
@@ -322,10 +338,12 @@ cudaError_t launch_gemv_t(const GemvArgs& a, int grid, size_t smem, cudaStream_t
 cudaError_t launch_gemv(const GemvArgs& a, int num_sms, cudaStream_t stream)
 {
     const size_t entries = (size_t)1 << a.L;
+    const bool mad = a.cb_f16 == kMadCodebook;
     // the table as fp32 when it fits in 64 KiB, else as binary16 (binary16 input only;
-    // the host refuses a binary32 table of 2^15 or more entries)
-    const bool cb16 = entries * 4 > 64 * 1024;
-    const size_t tab = (entries * (cb16 ? 2 : 4) + 15) & ~(size_t)15;
+    // the host refuses a binary32 table of 2^15 or more entries); none for the computed code
+    const bool cb16 = !mad && entries * 4 > 64 * 1024;
+    const int code = mad ? kCodeMad : cb16 ? kCodeF16 : kCodeF32;
+    const size_t tab = mad ? 0 : (entries * (cb16 ? 2 : 4) + 15) & ~(size_t)15;
     const size_t xbytes = (size_t)a.cols * 4;
     const bool xsmem = tab + xbytes <= 200 * 1024;
     const size_t smem = tab + (xsmem ? xbytes : 0);
@@ -334,20 +352,25 @@ cudaError_t launch_gemv(const GemvArgs& a, int num_sms, cudaStream_t stream)
     if (grid > num_sms) grid = num_sms;
     if (grid < 1) grid = 1;
     // specialised (L, k): compile-time shifts and masks, 8 or 4 weights per item
-#define TCQ_GEMV_FAST(LL, KK, NN, C16)                                                        \
-    if (a.L == LL && a.K == KK && cb16 == C16 && a.T % NN == 0)                                \
-        return xsmem ? launch_gemv_fast_t<LL, KK, NN, C16, true>(a, (int)grid, smem, stream) \
-                     : launch_gemv_fast_t<LL, KK, NN, C16, false>(a, (int)grid, smem, stream);
-    TCQ_GEMV_FAST(16, 2, 8, true)
-    TCQ_GEMV_FAST(16, 3, 4, true)
-    TCQ_GEMV_FAST(12, 2, 8, false)
-    TCQ_GEMV_FAST(8, 2, 8, false)
+#define TCQ_GEMV_FAST(LL, KK, NN, CC)                                                         \
+    if (a.L == LL && a.K == KK && code == CC && a.T % NN == 0)                                 \
+        return xsmem ? launch_gemv_fast_t<LL, KK, NN, CC, true>(a, (int)grid, smem, stream) \
+                     : launch_gemv_fast_t<LL, KK, NN, CC, false>(a, (int)grid, smem, stream);
+    TCQ_GEMV_FAST(16, 2, 8, kCodeF16)
+    TCQ_GEMV_FAST(16, 3, 4, kCodeF16)
+    TCQ_GEMV_FAST(12, 2, 8, kCodeF32)
+    TCQ_GEMV_FAST(8, 2, 8, kCodeF32)
+    TCQ_GEMV_FAST(16, 2, 8, kCodeMad)
+    TCQ_GEMV_FAST(16, 3, 4, kCodeMad)
 #undef TCQ_GEMV_FAST
+    if (mad)
+        return xsmem ? launch_gemv_t<kCodeMad, true>(a, (int)grid, smem, stream)
+                     : launch_gemv_t<kCodeMad, false>(a, (int)grid, smem, stream);
     if (cb16)
-        return xsmem ? launch_gemv_t<true, true>(a, (int)grid, smem, stream)
-                     : launch_gemv_t<true, false>(a, (int)grid, smem, stream);
-    return xsmem ? launch_gemv_t<false, true>(a, (int)grid, smem, stream)
-                 : launch_gemv_t<false, false>(a, (int)grid, smem, stream);
+        return xsmem ? launch_gemv_t<kCodeF16, true>(a, (int)grid, smem, stream)
+                     : launch_gemv_t<kCodeF16, false>(a, (int)grid, smem, stream);
+    return xsmem ? launch_gemv_t<kCodeF32, true>(a, (int)grid, smem, stream)
+                 : launch_gemv_t<kCodeF32, false>(a, (int)grid, smem, stream);
 }
 
 }  // namespace tcq

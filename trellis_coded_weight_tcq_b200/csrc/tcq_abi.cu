@@ -3,7 +3,7 @@
 // point allocates, frees, synchronises or keeps state between calls.
 #include <stdint.h>
 
-#include "common.cuh"
+#include "codes.cuh"
 
 using namespace tcq;
 
@@ -18,11 +18,46 @@ tcq_status check_shape(int L, int k, int T)
     return TCQ_OK;
 }
 
-bool valid_dtype(tcq_dtype dt) { return dt == TCQ_F32 || dt == TCQ_F16; }
+bool valid_dtype(tcq_dtype dt) { return dt == TCQ_F32 || dt == TCQ_F16 || dt == TCQ_MAD; }
+
+// A table codebook must be present and aligned to its entry; the computed code has none.
+bool codebook_ok(const void* cb, tcq_dtype dt)
+{
+    return dt == TCQ_MAD || (cb && aligned(cb, dt == TCQ_F16 ? 2 : 4));
+}
+
+// The kernels' codebook mode: 0 binary32 table, 1 binary16 table, 2 computed code.
+int code_mode(tcq_dtype dt) { return dt == TCQ_F16 ? 1 : dt == TCQ_MAD ? kMadCodebook : 0; }
+
+// Workspace bytes of the binary16 table a computed code is written to for the
+// table-based kernels (encoders, soft quantizer); 0 for a table codebook.
+size_t mad_table_bytes(int L, tcq_dtype dt)
+{
+    return dt == TCQ_MAD ? ((((size_t)2) << L) + 255) & ~(size_t)255 : 0;
+}
+
+// The dtype the table-based kernels run with.
+tcq_dtype table_dtype(tcq_dtype dt) { return dt == TCQ_MAD ? TCQ_F16 : dt; }
+
+// For the table-based kernels: writes the computed code's table to the front of
+// the workspace and points (cb, dt) at it; the workspace shrinks by its size.
+tcq_status resolve_table(const void*& cb, tcq_dtype& dt, int L, unsigned char*& ws,
+                         size_t& ws_bytes, cudaStream_t stream)
+{
+    if (dt != TCQ_MAD) return TCQ_OK;
+    const size_t tb = mad_table_bytes(L, dt);
+    if (ws_bytes < tb) return TCQ_ERR_WORKSPACE;
+    if (launch_mad_table(L, ws, stream) != cudaSuccess) return TCQ_ERR_CUDA;
+    cb = ws;
+    dt = TCQ_F16;
+    ws += tb;
+    ws_bytes -= tb;
+    return TCQ_OK;
+}
 
 const EncodeKernelInfo* select_kernel(int L, int k, tcq_dtype dt)
 {
-    const EncodeKernelInfo* g = find_grouped_kernel(L, k, dt == TCQ_F16 ? 1 : 0);
+    const EncodeKernelInfo* g = find_grouped_kernel(L, k, table_dtype(dt) == TCQ_F16 ? 1 : 0);
     return g ? g : generic_kernel_info(L, k);
 }
 
@@ -68,7 +103,7 @@ long long wanted_ctas(const EncodeKernelInfo* info, int L, int k, int T, long lo
 long long bcjr_grid(int L, int k, long long n_blocks, tcq_dtype dt, int sms)
 {
     const long long resident =
-        (long long)(sms > 0 ? sms : 148) * bcjr_ctas_per_sm(L, k, dt == TCQ_F16 ? 1 : 0);
+        (long long)(sms > 0 ? sms : 148) * bcjr_ctas_per_sm(L, k, table_dtype(dt) == TCQ_F16 ? 1 : 0);
     return n_blocks < resident ? n_blocks : resident;
 }
 
@@ -95,6 +130,18 @@ tcq_status run_encode(EncodeArgs& a, tcq_dtype cb_dtype, void* workspace, size_t
     return e == cudaSuccess ? TCQ_OK : TCQ_ERR_CUDA;
 }
 
+// run_encode for a caller's codebook of any dtype (a computed code is written
+// to the front of the workspace first).
+tcq_status resolve_and_encode(EncodeArgs& a, tcq_dtype dt, void* workspace, size_t workspace_bytes,
+                              cudaStream_t stream)
+{
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    const tcq_status r = resolve_table(a.cb, dt, a.L, ws, workspace_bytes, stream);
+    if (r != TCQ_OK) return r;
+    a.cb_f16 = code_mode(dt);
+    return run_encode(a, dt, ws, workspace_bytes, stream);
+}
+
 }  // namespace
 
 extern "C" {
@@ -110,7 +157,7 @@ size_t tcq_encode_workspace_bytes(int L, int k, int T, int64_t n_blocks, tcq_dty
     if (check_shape(L, k, T) != TCQ_OK || n_blocks <= 0 || !valid_dtype(cb_dtype)) return 0;
     const EncodeKernelInfo* info = select_kernel(L, k, cb_dtype);
     const long long ctas = wanted_ctas(info, L, k, T, n_blocks, current_sms());
-    return (size_t)ctas * info->slot_bytes(L, k, T);
+    return mad_table_bytes(L, cb_dtype) + (size_t)ctas * info->slot_bytes(L, k, T);
 }
 
 const char* tcq_encode_path(int L, int k, tcq_dtype cb_dtype)
@@ -129,12 +176,11 @@ tcq_status tcq_encode(const float* x, const float* d, const void* codebook, tcq_
     const tcq_status shape = check_shape(L, k, T);
     if (shape != TCQ_OK) return shape;
     if (n_blocks == 0) return TCQ_OK;
-    if (!x || !codebook || !start_state || !bits || !path_cost || !workspace)
+    if (!x || !codebook_ok(codebook, cb_dtype) || !start_state || !bits || !path_cost ||
+        !workspace)
         return TCQ_ERR_INVALID_ARG;
-    const size_t entry = cb_dtype == TCQ_F16 ? 2 : 4;
-    if (!aligned(x, 4) || (d && !aligned(d, 4)) || !aligned(codebook, entry) ||
-        !aligned(start_state, 4) || !aligned(bits, 4) || !aligned(path_cost, 4) ||
-        !aligned(workspace, 256))
+    if (!aligned(x, 4) || (d && !aligned(d, 4)) || !aligned(start_state, 4) ||
+        !aligned(bits, 4) || !aligned(path_cost, 4) || !aligned(workspace, 256))
         return TCQ_ERR_INVALID_ARG;
     if ((unsigned long long)n_blocks > (1ull << 40)) return TCQ_ERR_INVALID_ARG;
 
@@ -155,8 +201,8 @@ tcq_status tcq_encode(const float* x, const float* d, const void* codebook, tcq_
     a.d_stride = T;
     a.out_stride = 1;
     a.fixed_start = nullptr;
-    return run_encode(a, cb_dtype, workspace, workspace_bytes,
-                      reinterpret_cast<cudaStream_t>(stream));
+    return resolve_and_encode(a, cb_dtype, workspace, workspace_bytes,
+                              reinterpret_cast<cudaStream_t>(stream));
 }
 
 tcq_status tcq_encode_fixed_start(const float* x, const float* d, const void* codebook,
@@ -171,12 +217,11 @@ tcq_status tcq_encode_fixed_start(const float* x, const float* d, const void* co
     const tcq_status shape = check_shape(L, k, T);
     if (shape != TCQ_OK) return shape;
     if (n_blocks == 0) return TCQ_OK;
-    if (!x || !codebook || !start_state || !bits || !path_cost || !workspace)
+    if (!x || !codebook_ok(codebook, cb_dtype) || !start_state || !bits || !path_cost ||
+        !workspace)
         return TCQ_ERR_INVALID_ARG;
-    const size_t entry = cb_dtype == TCQ_F16 ? 2 : 4;
-    if (!aligned(x, 4) || (d && !aligned(d, 4)) || !aligned(codebook, entry) ||
-        !aligned(start_state, 4) || !aligned(bits, 4) || !aligned(path_cost, 4) ||
-        !aligned(workspace, 256))
+    if (!aligned(x, 4) || (d && !aligned(d, 4)) || !aligned(start_state, 4) ||
+        !aligned(bits, 4) || !aligned(path_cost, 4) || !aligned(workspace, 256))
         return TCQ_ERR_INVALID_ARG;
     if ((unsigned long long)n_blocks > (1ull << 40)) return TCQ_ERR_INVALID_ARG;
     EncodeArgs a;
@@ -196,8 +241,8 @@ tcq_status tcq_encode_fixed_start(const float* x, const float* d, const void* co
     a.d_stride = T;
     a.out_stride = 1;
     a.fixed_start = fixed_start;
-    return run_encode(a, cb_dtype, workspace, workspace_bytes,
-                      reinterpret_cast<cudaStream_t>(stream));
+    return resolve_and_encode(a, cb_dtype, workspace, workspace_bytes,
+                              reinterpret_cast<cudaStream_t>(stream));
 }
 
 tcq_status tcq_decode(const uint32_t* bits, const uint32_t* start_state, const void* codebook,
@@ -209,11 +254,8 @@ tcq_status tcq_decode(const uint32_t* bits, const uint32_t* start_state, const v
     const tcq_status shape = check_shape(L, k, T);
     if (shape != TCQ_OK) return shape;
     if (n_blocks == 0) return TCQ_OK;
-    if (!bits || !start_state || !codebook || !y) return TCQ_ERR_INVALID_ARG;
-    const size_t entry = cb_dtype == TCQ_F16 ? 2 : 4;
-    if (!aligned(bits, 4) || !aligned(start_state, 4) || !aligned(codebook, entry) ||
-        !aligned(y, 4))
-        return TCQ_ERR_INVALID_ARG;
+    if (!bits || !start_state || !codebook_ok(codebook, cb_dtype) || !y) return TCQ_ERR_INVALID_ARG;
+    if (!aligned(bits, 4) || !aligned(start_state, 4) || !aligned(y, 4)) return TCQ_ERR_INVALID_ARG;
     if ((unsigned long long)n_blocks > (1ull << 40)) return TCQ_ERR_INVALID_ARG;
     const int sms = current_sms();
     if (sms <= 0) return TCQ_ERR_CUDA;
@@ -222,7 +264,7 @@ tcq_status tcq_decode(const uint32_t* bits, const uint32_t* start_state, const v
     a.bits = bits;
     a.start_state = start_state;
     a.cb = codebook;
-    a.cb_f16 = cb_dtype == TCQ_F16 ? 1 : 0;
+    a.cb_f16 = code_mode(cb_dtype);
     a.L = L;
     a.K = k;
     a.T = T;
@@ -248,10 +290,10 @@ tcq_status tcq_gemv(const uint32_t* bits, const uint32_t* start_state, const flo
     if (cols % T != 0) return TCQ_ERR_INVALID_ARG;
     if (rows == 0) return TCQ_OK;
     if (cols > ((int64_t)1 << 31)) return TCQ_ERR_INVALID_ARG;
-    if (!bits || !start_state || !codebook || !x || !y) return TCQ_ERR_INVALID_ARG;
-    const size_t entry = cb_dtype == TCQ_F16 ? 2 : 4;
+    if (!bits || !start_state || !codebook_ok(codebook, cb_dtype) || !x || !y)
+        return TCQ_ERR_INVALID_ARG;
     if (!aligned(bits, 4) || !aligned(start_state, 4) || (scale && !aligned(scale, 4)) ||
-        !aligned(codebook, entry) || !aligned(x, 16) || !aligned(y, 4))
+        !aligned(x, 16) || !aligned(y, 4))
         return TCQ_ERR_INVALID_ARG;
     if ((unsigned long long)rows * (unsigned long long)(cols / T) > (1ull << 40))
         return TCQ_ERR_INVALID_ARG;
@@ -262,7 +304,7 @@ tcq_status tcq_gemv(const uint32_t* bits, const uint32_t* start_state, const flo
     a.start_state = start_state;
     a.scale = scale;
     a.cb = codebook;
-    a.cb_f16 = cb_dtype == TCQ_F16 ? 1 : 0;
+    a.cb_f16 = code_mode(cb_dtype);
     a.L = L;
     a.K = k;
     a.T = T;
@@ -297,21 +339,23 @@ tcq_status tcq_ldlq(const float* w, const float* u, const float* d, const void* 
     if (shape != TCQ_OK) return shape;
     if (cols % T != 0) return TCQ_ERR_INVALID_ARG;
     if (rows == 0 || cols == 0) return TCQ_OK;
-    if (!w || !u || !codebook || !q || !start_state || !bits || !path_cost || !workspace)
+    if (!w || !u || !codebook_ok(codebook, cb_dtype) || !q || !start_state || !bits ||
+        !path_cost || !workspace)
         return TCQ_ERR_INVALID_ARG;
-    const size_t entry = cb_dtype == TCQ_F16 ? 2 : 4;
-    if (!aligned(w, 4) || !aligned(u, 4) || (d && !aligned(d, 4)) || !aligned(codebook, entry) ||
-        !aligned(q, 4) || (x && !aligned(x, 4)) || !aligned(start_state, 4) ||
-        !aligned(bits, 4) || !aligned(path_cost, 4) || !aligned(workspace, 256))
+    if (!aligned(w, 4) || !aligned(u, 4) || (d && !aligned(d, 4)) || !aligned(q, 4) ||
+        (x && !aligned(x, 4)) || !aligned(start_state, 4) || !aligned(bits, 4) ||
+        !aligned(path_cost, 4) || !aligned(workspace, 256))
         return TCQ_ERR_INVALID_ARG;
     // grid rows of the feedback product, and the block count of the code
     if (rows > 65535LL * 128 || cols > ((int64_t)1 << 31)) return TCQ_ERR_INVALID_ARG;
     const size_t targets = ((size_t)rows * (size_t)T * sizeof(float) + 255) & ~(size_t)255;
-    if (workspace_bytes <= targets) return TCQ_ERR_WORKSPACE;
+    if (workspace_bytes <= targets + mad_table_bytes(L, cb_dtype)) return TCQ_ERR_WORKSPACE;
     const int sms = current_sms();
     if (sms <= 0) return TCQ_ERR_CUDA;
     const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     unsigned char* ws = static_cast<unsigned char*>(workspace);
+    const tcq_status rt = resolve_table(codebook, cb_dtype, L, ws, workspace_bytes, st);
+    if (rt != TCQ_OK) return rt;
     const int64_t nb = cols / T;
     const int W = tcq_words_per_block(k, T);
     // targets of the current column block: x[:, B] when the caller keeps them,
@@ -337,7 +381,7 @@ tcq_status tcq_ldlq(const float* w, const float* u, const float* d, const void* 
         a.x = f.x;
         a.d = d ? d + c0 : nullptr;
         a.cb = codebook;
-        a.cb_f16 = cb_dtype == TCQ_F16 ? 1 : 0;
+        a.cb_f16 = code_mode(cb_dtype);
         a.L = L;
         a.K = k;
         a.T = T;
@@ -374,7 +418,8 @@ tcq_status tcq_ldlq(const float* w, const float* u, const float* d, const void* 
 size_t tcq_bcjr_workspace_bytes(int L, int k, int T, int64_t n_blocks, tcq_dtype cb_dtype)
 {
     if (check_shape(L, k, T) != TCQ_OK || n_blocks <= 0 || !valid_dtype(cb_dtype)) return 0;
-    return (size_t)bcjr_grid(L, k, n_blocks, cb_dtype, current_sms()) * bcjr_slot_bytes(L, k, T);
+    return mad_table_bytes(L, cb_dtype) +
+           (size_t)bcjr_grid(L, k, n_blocks, cb_dtype, current_sms()) * bcjr_slot_bytes(L, k, T);
 }
 
 tcq_status tcq_bcjr(const float* x, const float* d, const void* codebook, tcq_dtype cb_dtype,
@@ -388,15 +433,19 @@ tcq_status tcq_bcjr(const float* x, const float* d, const void* codebook, tcq_dt
     if (shape != TCQ_OK) return shape;
     if (!(tau > 0.f) || !(tau < INFINITY)) return TCQ_ERR_INVALID_ARG;
     if (n_blocks == 0) return TCQ_OK;
-    if (!x || !codebook || !y_soft || !workspace) return TCQ_ERR_INVALID_ARG;
-    const size_t entry = cb_dtype == TCQ_F16 ? 2 : 4;
-    if (!aligned(x, 4) || (d && !aligned(d, 4)) || !aligned(codebook, entry) ||
-        !aligned(y_soft, 4) || (free_energy && !aligned(free_energy, 4)) ||
-        !aligned(workspace, 256))
+    if (!x || !codebook_ok(codebook, cb_dtype) || !y_soft || !workspace) return TCQ_ERR_INVALID_ARG;
+    if (!aligned(x, 4) || (d && !aligned(d, 4)) || !aligned(y_soft, 4) ||
+        (free_energy && !aligned(free_energy, 4)) || !aligned(workspace, 256))
         return TCQ_ERR_INVALID_ARG;
     if ((unsigned long long)n_blocks > (1ull << 40)) return TCQ_ERR_INVALID_ARG;
+    const float w_scale = (float)(1.4426950408889634 / (double)tau);
+    if (!(w_scale < INFINITY)) return TCQ_ERR_INVALID_ARG;
     const int sms = current_sms();
     if (sms <= 0) return TCQ_ERR_CUDA;
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    const tcq_status rt = resolve_table(codebook, cb_dtype, L, ws, workspace_bytes,
+                                        reinterpret_cast<cudaStream_t>(stream));
+    if (rt != TCQ_OK) return rt;
     const size_t slot = bcjr_slot_bytes(L, k, T);
     long long grid = bcjr_grid(L, k, n_blocks, cb_dtype, sms);
     const long long fit = (long long)(workspace_bytes / slot);
@@ -412,12 +461,11 @@ tcq_status tcq_bcjr(const float* x, const float* d, const void* codebook, tcq_dt
     a.K = k;
     a.T = T;
     a.n_blocks = n_blocks;
-    a.w_scale = (float)(1.4426950408889634 / (double)tau);
-    if (!(a.w_scale < INFINITY)) return TCQ_ERR_INVALID_ARG;
+    a.w_scale = w_scale;
     a.tau_ln2 = (double)tau * 0.6931471805599453;
     a.y = y_soft;
     a.free_energy = free_energy;
-    a.ws = static_cast<unsigned char*>(workspace);
+    a.ws = ws;
     a.slot_bytes = slot;
     const cudaError_t e = launch_bcjr(a, (int)grid, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TCQ_OK : TCQ_ERR_CUDA;

@@ -27,6 +27,17 @@ TCQ_ERR_CUDA = 4
 TCQ_ERR_INTERNAL = 5
 TCQ_F32 = 0
 TCQ_F16 = 1
+TCQ_MAD = 2
+
+
+class _ComputedCode:
+    """Stands for the computed (lookup-free) code wherever a codebook tensor goes."""
+
+    def __repr__(self):
+        return "MAD"
+
+
+MAD = _ComputedCode()  # pass as ``codebook`` to select TCQ_MAD
 TCQ_MAX_L = 16
 TCQ_MAX_K = 4
 TCQ_MAX_T = 1 << 20
@@ -162,6 +173,8 @@ def _torch():
 
 
 def cb_dtype_of(codebook) -> int:
+    if codebook is MAD:
+        return TCQ_MAD
     torch = _torch()
     if codebook.dtype == torch.float16:
         return TCQ_F16
@@ -171,7 +184,7 @@ def cb_dtype_of(codebook) -> int:
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    return None if t is None or t is MAD else ctypes.c_void_p(t.data_ptr())
 
 
 def _stream_handle(stream=None):
