@@ -326,6 +326,27 @@ def run_ours(args, rank, world, local_rank):
                 "hbm_gbs": g_bytes / (g_ms / 1e3) / 1e9,
                 "hbm_frac": g_bytes / (g_ms / 1e3) / 1e9 / float(peaks_g.get("hbm_gbs", 6650.0)),
                 "bytes": g_bytes}
+        # the same bitstreams read as the computed (lookup-free) code: no table,
+        # each codeword computed in registers
+        for _ in range(3):
+            tcq.gemv(out.bits, out.start_state, scale, tcq.MAD, L, k, T, rows_m, cols_m, xv, ym)
+        m_ev = []
+        for _ in range(10):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            tcq.gemv(out.bits, out.start_state, scale, tcq.MAD, L, k, T, rows_m, cols_m, xv, ym)
+            b.record(stream)
+            m_ev.append((a, b))
+        torch.cuda.synchronize()
+        m_ms = min(a.elapsed_time(b) for a, b in m_ev)
+        # issue-bound: about 6 instructions per weight at best (state, multiply,
+        # byte sum, float, FMA) against 148 SMs x 128 lanes x the max clock
+        issue_peak = SMS * LANES_PER_SM * float(peaks_g.get("sm_max_mhz", 1965.0)) * 1e6
+        gemv["computed_code"] = {
+            "ms": m_ms, "weights_per_s": rows_m * cols_m / (m_ms / 1e3),
+            "hbm_gbs": g_bytes / (m_ms / 1e3) / 1e9,
+            "bound": "alu", "ops_per_weight": 6,
+            "frac": rows_m * cols_m * 6 / (m_ms / 1e3) / issue_peak}
 
     # ---- end to end through the C ABI from pinned host buffers
     e2e = None
@@ -502,7 +523,7 @@ def main():
                     help="skip the soft forward-backward quantization of the workload")
     ap.add_argument("--no-ldlq", action="store_true",
                     help="skip the error-feedback encode of the MLP matrix")
-    ap.add_argument("--cpu-blocks-per-core", type=int, default=8)
+    ap.add_argument("--cpu-blocks-per-core", type=int, default=16)
     ap.add_argument("--blocks", type=int, default=0,
                     help="encode only the first N blocks of the workload (a smaller profiling "
                          "case; reported in config.n_blocks)")

@@ -76,6 +76,7 @@ def test_decode_computed_code_bit_exact(L, k, T, cuda_device):
 @pytest.mark.parametrize("L,k,T,rows,nb", [
     (16, 2, 256, 300, 16),   # the MLP shape's blocks: compile-time kernel
     (16, 3, 256, 60, 16),
+    (16, 2, 256, 40, 6),     # 6 blocks per row: the per-item compile-time kernel
     (12, 2, 256, 70, 8),     # runtime kernel
     (16, 2, 24, 33, 5),      # T not a multiple of 8: runtime kernel
 ])
