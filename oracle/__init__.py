@@ -9,6 +9,8 @@ from .tcq_oracle import (  # noqa: F401
     build_oracle,
     oracle_decode,
     oracle_encode,
+    oracle_encode_vec,
+    oracle_decode_vec,
     oracle_feedback_targets,
     oracle_gemv,
     oracle_greedy,

@@ -489,3 +489,119 @@ int oracle_mad_codebook(int L, double* cb)
     }
     return ORACLE_OK;
 }
+
+/*
+ * Vector trellis: V weights per trellis step ("QTIP: Quantization with
+ * Trellises and Incoherence Processing", abstract: the bitshift trellis with a
+ * stateful decoder that separates the codebook size from the bitrate and the
+ * effective dimension).  Each step shifts kV bits into the state and the state
+ * selects a V-dimensional codeword; V = 1 is oracle_encode.
+ *
+ * One block: T weights (V | T), steps tau = 1..T/V, codebook cb[2^L][V]
+ * (row-major), with mask = 2^L - 1:
+ *     s_tau = ((s_{tau-1} << kV) | b_tau) & mask,   b_tau in [0, 2^{kV})
+ *     y_{(tau-1)V + v} = cb[s_tau][v]
+ *     J = sum_tau sum_v d_{(tau-1)V+v} (x_{(tau-1)V+v} - cb[s_tau][v])^2
+ * Same dynamic program per state as oracle_encode (smallest predecessor on
+ * ties, smallest final state), same packing with symbols of kV bits, the
+ * stored start s_1 >> kV.  Requires kV <= L and kV <= 8.
+ */
+int oracle_encode_vec(const double* x, const double* d, const double* cb, int L, int k, int V,
+                      int T, int64_t n_blocks, int64_t fixed_start, uint32_t* start_state,
+                      uint32_t* bits, double* cost)
+{
+    if (V < 1 || k < 1 || k * V > L || k * V > 8 || T < 1 || T % V != 0 || n_blocks < 0 ||
+        !valid_shape(L, k, T))
+        return ORACLE_EINVAL;
+    if (n_blocks == 0) return ORACLE_OK;
+    if (!x || !cb || !start_state || !bits || !cost) return ORACLE_EINVAL;
+    const int K = k * V;          /* bits per step */
+    const int NS = T / V;         /* steps */
+    const int64_t S = (int64_t)1 << L;
+    const uint32_t mask = (uint32_t)(S - 1);
+    const uint32_t low_mask = (uint32_t)(((uint64_t)1 << (L - K)) - 1);
+    const int H = 1 << K;
+    const int W = oracle_words_per_block(k, T);
+    double* prev = (double*)malloc(sizeof(double) * S);
+    double* cur = (double*)malloc(sizeof(double) * S);
+    uint8_t* bp = (uint8_t*)malloc((size_t)NS * (size_t)S);
+    uint32_t* path = (uint32_t*)malloc(sizeof(uint32_t) * (size_t)NS);
+    if (!prev || !cur || !bp || !path) {
+        free(prev); free(cur); free(bp); free(path);
+        return ORACLE_ENOMEM;
+    }
+    for (int64_t blk = 0; blk < n_blocks; ++blk) {
+        const double* xb = x + blk * T;
+        const double* db = d ? d + blk * T : NULL;
+        for (int tau = 1; tau <= NS; ++tau) {
+            uint8_t* bpt = bp + (size_t)(tau - 1) * (size_t)S;
+            for (int64_t s = 0; s < S; ++s) {
+                double bm = 0.0; /* the step's branch metric: V weighted squared errors */
+                for (int v = 0; v < V; ++v) {
+                    const int i = (tau - 1) * V + v;
+                    const double e = xb[i] - cb[s * V + v];
+                    bm += weight_at(db, i) * e * e;
+                }
+                double best;
+                int best_h = 0;
+                if (tau == 1) {
+                    int reachable = 1;
+                    if (fixed_start >= 0)
+                        reachable = (((uint32_t)s >> K) == ((uint32_t)fixed_start & low_mask));
+                    best = reachable ? 0.0 : INFINITY;
+                } else {
+                    best = INFINITY;
+                    for (int h = 0; h < H; ++h) {
+                        const uint32_t pred = (((uint32_t)h << (L - K)) | ((uint32_t)s >> K)) & mask;
+                        if (prev[pred] < best) {
+                            best = prev[pred];
+                            best_h = h;
+                        }
+                    }
+                }
+                cur[s] = best + bm;
+                bpt[s] = (uint8_t)best_h;
+            }
+            double* tmp = prev; prev = cur; cur = tmp;
+        }
+        int64_t s_best = 0;
+        for (int64_t s = 1; s < S; ++s)
+            if (prev[s] < prev[s_best]) s_best = s;
+        cost[blk] = prev[s_best];
+        uint32_t s = (uint32_t)s_best;
+        path[NS - 1] = s;
+        for (int tau = NS; tau >= 2; --tau) {
+            const uint32_t h = bp[(size_t)(tau - 1) * (size_t)S + s];
+            s = ((h << (L - K)) | (s >> K)) & mask;
+            path[tau - 2] = s;
+        }
+        uint32_t* wb = bits + blk * W;
+        memset(wb, 0, sizeof(uint32_t) * (size_t)W);
+        for (int tau = 1; tau <= NS; ++tau) put_symbol(wb, K, tau, path[tau - 1] & (uint32_t)(H - 1));
+        start_state[blk] = path[0] >> K;
+    }
+    free(prev); free(cur); free(bp); free(path);
+    return ORACLE_OK;
+}
+
+/* Decode of the vector trellis: y_{(tau-1)V + v} = cb[s_tau][v]. */
+int oracle_decode_vec(const uint32_t* bits, const uint32_t* start_state, const double* cb, int L,
+                      int k, int V, int T, int64_t n_blocks, double* y)
+{
+    if (V < 1 || k < 1 || k * V > L || T < 1 || T % V != 0 || n_blocks < 0 ||
+        !valid_shape(L, k, T))
+        return ORACLE_EINVAL;
+    if (n_blocks == 0) return ORACLE_OK;
+    if (!bits || !start_state || !cb || !y) return ORACLE_EINVAL;
+    const int K = k * V;
+    const uint64_t mask = ((uint64_t)1 << L) - 1;
+    const int W = oracle_words_per_block(k, T);
+    for (int64_t blk = 0; blk < n_blocks; ++blk) {
+        uint64_t s = start_state[blk];
+        for (int tau = 1; tau <= T / V; ++tau) {
+            s = ((s << K) | get_symbol(bits + blk * W, K, tau)) & mask;
+            for (int v = 0; v < V; ++v) y[blk * T + (tau - 1) * V + v] = cb[s * V + v];
+        }
+    }
+    return ORACLE_OK;
+}

@@ -58,6 +58,10 @@ def _load():
         lib.oracle_bcjr.restype = ci
         lib.oracle_mad_codebook.argtypes = [ci, dp]
         lib.oracle_mad_codebook.restype = ci
+        lib.oracle_encode_vec.argtypes = [dp, dp, dp, ci, ci, ci, ci, i64, i64, up, up, dp]
+        lib.oracle_encode_vec.restype = ci
+        lib.oracle_decode_vec.argtypes = [up, up, dp, ci, ci, ci, ci, i64, dp]
+        lib.oracle_decode_vec.restype = ci
         _lib = lib
     return _lib
 
@@ -266,3 +270,40 @@ def oracle_mad_codebook(L: int):
     if rc != 0:
         raise ValueError(f"oracle_mad_codebook failed with code {rc}")
     return cb
+
+
+def oracle_encode_vec(x, d, codebook, L: int, k: int, V: int, fixed_start: int | None = None):
+    """Viterbi TCQ over the vector trellis (V weights per step, kV bits shifted in,
+    codebook [2^L, V]).  Returns (start, bits, cost) like oracle_encode."""
+    x = _f64(x)
+    if x.ndim == 1:
+        x = x[None, :]
+    n, T = x.shape
+    dd = None if d is None else _f64(d).reshape(n, T)
+    cb = _f64(codebook).reshape(-1)
+    W = oracle_words_per_block(k, T)
+    start = np.zeros(n, dtype=np.uint32)
+    bits = np.zeros((n, W), dtype=np.uint32)
+    cost = np.zeros(n)
+    rc = _load().oracle_encode_vec(
+        _ptr(x, ctypes.c_double), None if dd is None else _ptr(dd, ctypes.c_double),
+        _ptr(cb, ctypes.c_double), L, k, V, T, n, -1 if fixed_start is None else int(fixed_start),
+        _ptr(start, ctypes.c_uint32), _ptr(bits, ctypes.c_uint32), _ptr(cost, ctypes.c_double))
+    if rc != 0:
+        raise ValueError(f"oracle_encode_vec failed with code {rc}")
+    return start, bits, cost
+
+
+def oracle_decode_vec(bits, start_state, codebook, L: int, k: int, V: int, T: int):
+    """Values [n, T] of the vector trellis from packed bits and start states."""
+    bits = np.ascontiguousarray(bits, dtype=np.uint32)
+    start = np.ascontiguousarray(start_state, dtype=np.uint32).reshape(-1)
+    n = start.shape[0]
+    cb = _f64(codebook).reshape(-1)
+    y = np.zeros((n, T))
+    rc = _load().oracle_decode_vec(_ptr(bits, ctypes.c_uint32), _ptr(start, ctypes.c_uint32),
+                                   _ptr(cb, ctypes.c_double), L, k, V, T, n,
+                                   _ptr(y, ctypes.c_double))
+    if rc != 0:
+        raise ValueError(f"oracle_decode_vec failed with code {rc}")
+    return y

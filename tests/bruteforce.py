@@ -104,3 +104,34 @@ def boltzmann_brute_force(x, d, codebook, L: int, k: int, tau: float):
     p = np.exp(a - logz)
     y = (p[:, None] * c[st]).sum(axis=0)
     return y, -tau * logz
+
+
+def brute_force_vec(x, d, codebook, L: int, k: int, V: int):
+    """Minimum over every start state and bitstream of the vector trellis (V
+    weights per step, kV bits per step, codebook [2^L, V]); (J_min, s0, n)."""
+    x = np.asarray(x, dtype=np.float64).reshape(-1)
+    T = x.size
+    d = np.ones(T) if d is None else np.asarray(d, dtype=np.float64).reshape(-1)
+    c = np.asarray(codebook, dtype=np.float64).reshape(1 << L, V)
+    steps, K = T // V, k * V
+    assert steps * K <= 16, "keep the enumeration small"
+    s0 = np.arange(1 << L, dtype=np.int64)
+    n = np.arange(1 << (steps * K), dtype=np.int64)
+    st = states_for(L, K, steps, s0[:, None], n[None, :])  # [S0, N, steps]
+    vals = c[st]                                          # [S0, N, steps, V]
+    err = (d.reshape(steps, V) * (x.reshape(steps, V) - vals) ** 2).sum(axis=(-1, -2))
+    flat = int(np.argmin(err))
+    i0, i1 = np.unravel_index(flat, err.shape)
+    return float(err[i0, i1]), int(s0[i0]), int(n[i1])
+
+
+def decode_window_vec(words, start: int, codebook, L: int, k: int, V: int, T: int) -> np.ndarray:
+    """Values of one vector-trellis block by the bit window (symbols of kV bits)."""
+    K, steps = k * V, T // V
+    sym = unpack_symbols(words, K, steps)
+    n = stream_value(sym, K)
+    s0 = int(start) & 0xFFFFFFFF
+    mask = (1 << L) - 1
+    st = [((s0 << (t * K)) | (n >> ((steps - t) * K))) & mask for t in range(1, steps + 1)]
+    c = np.asarray(codebook, dtype=np.float64).reshape(1 << L, V)
+    return c[np.array(st, dtype=np.int64)].reshape(-1)
