@@ -265,6 +265,35 @@ tcq_status tcq_bcjr(const float* x, const float* d, const void* codebook, tcq_dt
                     float* free_energy, void* workspace, size_t workspace_bytes,
                     tcq_stream_t stream);
 
+/*
+ * Vector trellis: V weights per trellis step (QTIP abstract: the bitshift
+ * trellis with a stateful decoder separates the codebook size from the bitrate
+ * and the effective dimension).  Each step shifts k V bits into the L-bit state
+ * and the state selects a V-dimensional codeword:
+ *     s_t = ((s_{t-1} << kV) | b_t) & (2^L - 1),   y_{(t-1)V + v} = c[s_t][v],
+ * and the search minimises J = sum_i d_i (x_i - y_i)^2 over every start state and
+ * bitstream.  Bits are packed as for tcq_encode with symbols of kV bits (still
+ * k bits per weight, W = ceil(T k / 32)); start_state = s_1 >> kV.
+ *
+ *   codebook  2^L rows of V entries (row-major), binary32 or binary16; the
+ *             computed code (TCQ_MAD) is scalar: TCQ_ERR_UNSUPPORTED for V > 1.
+ * Supported: 1 <= V <= 8, V | T, k V <= min(L, 8) (else TCQ_ERR_UNSUPPORTED).
+ * V == 1 is exactly tcq_encode / tcq_decode.  V > 1 runs the runtime-(L, k)
+ * kernel (not tuned).  Other arguments, outputs and errors as tcq_encode /
+ * tcq_decode.
+ */
+size_t tcq_encode_vec_workspace_bytes(int L, int k, int V, int T, int64_t n_blocks,
+                                      tcq_dtype cb_dtype);
+
+tcq_status tcq_encode_vec(const float* x, const float* d, const void* codebook, tcq_dtype cb_dtype,
+                          int L, int k, int V, int T, int64_t n_blocks, uint32_t* start_state,
+                          uint32_t* bits, float* path_cost, void* workspace,
+                          size_t workspace_bytes, tcq_stream_t stream);
+
+tcq_status tcq_decode_vec(const uint32_t* bits, const uint32_t* start_state, const void* codebook,
+                          tcq_dtype cb_dtype, int L, int k, int V, int T, int64_t n_blocks,
+                          float* y, tcq_stream_t stream);
+
 /* Static, human-readable name of a status code. */
 const char* tcq_status_string(tcq_status status);
 

@@ -1,0 +1,99 @@
+"""GPU parity of the vector trellis (tcq_encode_vec / tcq_decode_vec: V weights
+per step, kV bits shifted in, V-dimensional codewords) against the oracle."""
+import ctypes
+
+import numpy as np
+import pytest
+
+from tests.parity import ABS_TOL_PER_D, REL_TOL
+from trellis_coded_weight_tcq_b200 import tcq
+
+pytestmark = pytest.mark.gpu
+
+# L, k, V, T, blocks, codebook dtype, weighted
+CASES = [
+    (8, 1, 2, 32, 40, "f32", True),
+    (8, 2, 2, 64, 30, "f32", False),
+    (12, 2, 2, 128, 8, "f32", True),
+    (6, 1, 4, 24, 50, "f16", True),
+    (10, 2, 3, 48, 12, "f32", True),
+    (16, 1, 2, 64, 3, "f16", True),    # metrics in the workspace
+    (8, 4, 2, 16, 10, "f32", True),    # kV = L: no trellis memory
+    (5, 1, 5, 35, 20, "f32", False),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "L{}k{}V{}T{}_B{}_{}{}".format(*c[:6], "_w" if c[6] else ""))
+def test_encode_vec_parity(case, cuda_device):
+    import torch
+    from oracle import oracle_decode_vec, oracle_encode_vec
+
+    L, k, V, T, n, cbt, weighted = case
+    rng = np.random.default_rng(8000 + 31 * L + 7 * k + V + T)
+    x = rng.standard_normal((n, T)).astype(np.float32)
+    d = rng.lognormal(0.0, 1.0, (n, T)).astype(np.float32) if weighted else None
+    cb = rng.standard_normal((1 << L, V))
+    cb = cb.astype(np.float16) if cbt == "f16" else cb.astype(np.float32)
+    out = tcq.encode_vec(torch.from_numpy(x).to(cuda_device),
+                         None if d is None else torch.from_numpy(d).to(cuda_device),
+                         torch.from_numpy(cb).to(cuda_device), L, k, V)
+    torch.cuda.synchronize()
+    start = out.start_state.cpu().numpy().view(np.uint32)
+    bits = out.bits.cpu().numpy().view(np.uint32)
+    cost = out.path_cost.cpu().numpy().astype(np.float64)
+    assert np.all(start < (1 << (L - k * V)))
+    _, _, J_o = oracle_encode_vec(x, d, cb, L, k, V)
+    y = oracle_decode_vec(bits, start, cb, L, k, V, T)
+    dd = np.ones((n, T)) if d is None else d.astype(np.float64)
+    J_g = (dd * (x.astype(np.float64) - y) ** 2).sum(axis=1)
+    tol = REL_TOL * J_o + ABS_TOL_PER_D * dd.sum(axis=1)
+    assert np.all(np.abs(J_g - J_o) <= tol), float(np.max(np.abs(J_g - J_o) / J_o))
+    assert np.all(np.abs(cost - J_g) <= tol)
+    # the GPU's own decode of its bits
+    yg = tcq.decode_vec(out.bits, out.start_state, torch.from_numpy(cb).to(cuda_device), L, k, V, T)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(yg.cpu().numpy(), y.astype(np.float32))
+
+
+@pytest.mark.parametrize("L,k,V,T", [(8, 1, 2, 32), (12, 2, 2, 256), (16, 1, 4, 64), (9, 3, 2, 30)])
+def test_decode_vec_bit_exact(L, k, V, T, cuda_device):
+    import torch
+    from oracle import oracle_decode_vec
+
+    rng = np.random.default_rng(8100 + L + V)
+    n = 33
+    W = tcq.tcq_words_per_block(k, T)
+    bits = rng.integers(0, 2**32, size=(n, W), dtype=np.uint64).astype(np.uint32)
+    start = rng.integers(0, 2**32, size=n, dtype=np.uint64).astype(np.uint32)
+    cb = rng.standard_normal((1 << L, V)).astype(np.float32)
+    y = tcq.decode_vec(torch.from_numpy(bits.view(np.int32)).to(cuda_device),
+                       torch.from_numpy(start.view(np.int32)).to(cuda_device),
+                       torch.from_numpy(cb).to(cuda_device), L, k, V, T)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(y.cpu().numpy(), oracle_decode_vec(bits, start, cb, L, k, V, T).astype(np.float32))
+
+
+def test_v1_is_tcq_encode(cuda_device):
+    import torch
+
+    rng = np.random.default_rng(8200)
+    x = torch.from_numpy(rng.standard_normal((20, 256)).astype(np.float32)).to(cuda_device)
+    cb = torch.from_numpy(rng.standard_normal(1 << 12).astype(np.float32)).to(cuda_device)
+    a = tcq.encode(x, None, cb, 12, 2)
+    b = tcq.encode_vec(x, None, cb, 12, 2, 1)
+    torch.cuda.synchronize()
+    assert torch.equal(a.bits, b.bits) and torch.equal(a.start_state, b.start_state)
+    assert torch.equal(a.path_cost, b.path_cost)
+
+
+def test_vec_rejections(cuda_device):
+    fake = ctypes.c_void_p(0x10000)
+    enc = lambda **o: tcq.tcq_encode_vec(fake, None, o.get("cb", fake), o.get("dt", tcq.TCQ_F32),  # noqa: E731
+                                         o.get("L", 8), o.get("k", 2), o.get("V", 2), o.get("T", 32),
+                                         4, fake, fake, fake, fake, 1 << 30, None)
+    assert enc(T=33) == tcq.TCQ_ERR_UNSUPPORTED            # V does not divide T
+    assert enc(k=3, V=3, L=12) == tcq.TCQ_ERR_UNSUPPORTED  # kV = 9 > 8
+    assert enc(k=2, V=3, L=5) == tcq.TCQ_ERR_UNSUPPORTED   # kV > L
+    assert enc(V=9) == tcq.TCQ_ERR_UNSUPPORTED
+    assert enc(dt=tcq.TCQ_MAD, cb=None) == tcq.TCQ_ERR_UNSUPPORTED
+    assert enc(cb=None) == tcq.TCQ_ERR_INVALID_ARG

@@ -6,8 +6,10 @@
 // without their compile-time layout: one thread per u per step, codewords read
 // through the L1 cache, one byte of backpointer per (step, u) in the workspace,
 // and the traceback done by thread 0 after each block's forward pass.  It
-// covers shapes the grouped kernels do not (L < 2k, odd sizes) and serves as a
-// second, independent GPU path in the tests; it is not tuned.
+// covers shapes the grouped kernels do not (L < 2k, odd sizes) and the vector
+// trellis (V weights per step: kV bits shifted in, a V-dimensional codeword per
+// state, the branch metric summed over the V weights), and serves as a second,
+// independent GPU path in the tests; it is not tuned.
 #include "common.cuh"
 
 namespace tcq {
@@ -15,6 +17,7 @@ namespace tcq {
 namespace {
 
 constexpr int kGenericThreads = 256;
+constexpr int kMaxV = 8;  // weights per step
 // path metrics stay in shared memory up to this many bytes of ping-pong, else
 // they go to the workspace slot (global memory, L2 resident)
 constexpr size_t kGenericSmemMetricBytes = 96 * 1024;
@@ -43,7 +46,8 @@ __global__ void __launch_bounds__(kGenericThreads) acs_generic_kernel(EncodeArgs
     __shared__ uint32_t reds[kGenericThreads / 32];
     __shared__ uint32_t fin;
 
-    const int L = a.L, K = a.K, T = a.T;
+    // a step shifts in K = k V bits and covers V weights; NS steps per block
+    const int L = a.L, V = a.V, K = a.K * a.V, NS = a.T / a.V;
     const int LK = L - K;
     const uint32_t NU = 1u << LK;
     const int H = 1 << K;
@@ -51,7 +55,7 @@ __global__ void __launch_bounds__(kGenericThreads) acs_generic_kernel(EncodeArgs
     uint8_t* bp = slot;
     float* Mbase = generic_metrics_in_smem(L, K)
                        ? gsm
-                       : reinterpret_cast<float*>(slot + generic_bp_bytes(L, K, T));
+                       : reinterpret_cast<float*>(slot + generic_bp_bytes(L, K, NS));
 
     for (long long b = blockIdx.x; b < a.n_blocks; b += gridDim.x) {
         const float* xb = a.x + b * a.x_stride;
@@ -60,9 +64,17 @@ __global__ void __launch_bounds__(kGenericThreads) acs_generic_kernel(EncodeArgs
         uint32_t bests = 0xffffffffu;
         // a fixed start s_0 leaves only its successors reachable at step 1
         const uint32_t s0 = a.fixed_start ? (a.fixed_start[b] & (NU - 1u)) : 0xffffffffu;
-        for (int t = 1; t <= T; ++t) {
-            const float sd = db ? sqrtf(db[t - 1]) : 1.f;
-            const float ca = -sd, cx = sd * xb[t - 1];
+        for (int t = 1; t <= NS; ++t) {
+            float ca[kMaxV], cx[kMaxV];
+#pragma unroll
+            for (int v = 0; v < kMaxV; ++v) {
+                if (v < V) {
+                    const int i = (t - 1) * V + v;
+                    const float sd = db ? sqrtf(db[i]) : 1.f;
+                    ca[v] = -sd;
+                    cx[v] = sd * xb[i];
+                }
+            }
             const float* Mp = Mbase + ((t - 1) & 1) * NU;
             float* Mn = Mbase + (t & 1) * NU;
             for (uint32_t u = threadIdx.x; u < NU; u += blockDim.x) {
@@ -70,15 +82,21 @@ __global__ void __launch_bounds__(kGenericThreads) acs_generic_kernel(EncodeArgs
                 uint32_t bh = 0;
                 for (int h = 0; h < H; ++h) {
                     const uint32_t s = ((uint32_t)h << LK) | u;
-                    const float e = fmaf(ca, load_codeword(a.cb, a.cb_f16, s), cx);
                     const float m0 = (s0 == 0xffffffffu || (s >> K) == s0) ? 0.f : __int_as_float(0x7f800000);
-                    const float v = fmaf(e, e, t == 1 ? m0 : Mp[s >> K]);
+                    float v = t == 1 ? m0 : Mp[s >> K];
+#pragma unroll
+                    for (int w = 0; w < kMaxV; ++w) {
+                        if (w < V) {
+                            const float e = fmaf(ca[w], load_codeword(a.cb, a.cb_f16, s * V + w), cx[w]);
+                            v = fmaf(e, e, v);
+                        }
+                    }
                     if (v < best) {
                         best = v;
                         bh = (uint32_t)h;
                     }
                 }
-                if (t < T) {
+                if (t < NS) {
                     Mn[u] = best;
                     bp[(size_t)(t - 1) * NU + u] = (uint8_t)bh;
                 } else {
@@ -107,10 +125,13 @@ __global__ void __launch_bounds__(kGenericThreads) acs_generic_kernel(EncodeArgs
             BackwardBitWriter bw(a.bits + b * a.out_stride * a.W, a.W);
             uint32_t s = fin;
             double cost = 0.0;
-            for (int t = T; t >= 1; --t) {
-                const float dv = db ? db[t - 1] : 1.f;
-                const double e = (double)xb[t - 1] - (double)load_codeword(a.cb, a.cb_f16, s);
-                cost += (double)dv * e * e;
+            for (int t = NS; t >= 1; --t) {
+                for (int w = 0; w < V; ++w) {
+                    const int i = (t - 1) * V + w;
+                    const float dv = db ? db[i] : 1.f;
+                    const double e = (double)xb[i] - (double)load_codeword(a.cb, a.cb_f16, s * V + w);
+                    cost += (double)dv * e * e;
+                }
                 bw.put(t, K, s & (uint32_t)(H - 1));
                 if (t > 1) {
                     const uint32_t u = s >> K;
@@ -140,7 +161,7 @@ size_t generic_smem_bytes(int L, int K, int)
 
 cudaError_t launch_generic(const EncodeArgs& a, int grid, cudaStream_t stream)
 {
-    const size_t smem = generic_smem_bytes(a.L, a.K, a.T);
+    const size_t smem = generic_smem_bytes(a.L, a.K * a.V, a.T / a.V);  // per step: kV bits
     cudaError_t e = cudaFuncSetAttribute(acs_generic_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -157,9 +178,12 @@ const EncodeKernelInfo kGenericInfo = {"generic", 1, kGenericThreads, 2, &generi
 
 }  // namespace
 
+// K: bits shifted in per step (k V for the vector trellis), at most 8 since a
+// backpointer is one byte.  The info's size callbacks take (L, bits per step,
+// steps per block).
 const EncodeKernelInfo* generic_kernel_info(int L, int K)
 {
-    if (L < 1 || L > TCQ_MAX_L || K < 1 || K > TCQ_MAX_K || K > L) return nullptr;
+    if (L < 1 || L > TCQ_MAX_L || K < 1 || K > 8 || K > L) return nullptr;
     return &kGenericInfo;
 }
 

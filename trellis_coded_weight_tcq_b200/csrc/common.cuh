@@ -26,6 +26,7 @@ struct EncodeArgs {
     const uint32_t* fixed_start;  // block b starts in fixed_start[b] (low L-k bits), or nullptr: free
     unsigned char* ws;     // workspace base: gridDim.x slots of slot_bytes
     size_t slot_bytes;
+    int V = 1;             // weights per trellis step (kV bits shifted in; codebook [2^L][V])
 };
 
 // A value the compiler must treat as unknown at each use: a volatile move keeps
@@ -171,6 +172,8 @@ size_t bcjr_slot_bytes(int L, int K, int T);
 int bcjr_ctas_per_sm(int L, int K, int cb_f16);
 cudaError_t launch_bcjr(const BcjrArgs& a, int grid, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, int num_sms, cudaStream_t stream);
+// vector trellis: a.K = k V bits per step, a.T weights per block (V | T)
+cudaError_t launch_decode_vec(const DecodeArgs& a, int V, int num_sms, cudaStream_t stream);
 cudaError_t launch_gemv(const GemvArgs& a, int num_sms, cudaStream_t stream);
 
 }  // namespace tcq

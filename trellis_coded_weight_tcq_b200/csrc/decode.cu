@@ -151,6 +151,40 @@ cudaError_t launch_mode(const DecodeArgs& a, int grid, size_t smem, cudaStream_t
 
 }  // namespace
 
+// Vector trellis: one thread per (block, step); the step's state is the L-bit
+// window ending at stream bit t K (K = k V bits per step, stream word -1 the
+// start state), and the step writes the V values of its codeword.
+__global__ void decode_vec_kernel(DecodeArgs a, int V)
+{
+    const int K = a.K, L = a.L, W = a.W, NS = a.T / V;
+    const uint32_t mask = (1u << L) - 1u;
+    const long long total = a.n_blocks * NS;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const long long b = i / NS;
+        const int t = (int)(i - b * NS) + 1;
+        const int p0 = t * K - L;  // window start, > -32
+        const int wi = p0 >> 5;
+        const uint32_t* wb = a.bits + b * W;
+        const unsigned long long hi = wi < 0 ? a.start_state[b] : wb[wi];
+        const unsigned long long lo = wi + 1 < W ? wb[wi + 1] : 0ull;
+        const uint32_t s = (uint32_t)((((hi << 32) | lo) >> (64 - (p0 & 31) - L)) & mask);
+        float* y = a.y + b * a.T + (long long)(t - 1) * V;
+        for (int v = 0; v < V; ++v) y[v] = load_codeword(a.cb, a.cb_f16, s * V + v);
+    }
+}
+
+cudaError_t launch_decode_vec(const DecodeArgs& a, int V, int num_sms, cudaStream_t stream)
+{
+    const long long total = a.n_blocks * (a.T / V);
+    long long grid = (total + 255) / 256;
+    const long long cap = (long long)num_sms * 8;
+    if (grid > cap) grid = cap;
+    if (grid < 1) grid = 1;
+    decode_vec_kernel<<<(int)grid, 256, 0, stream>>>(a, V);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_decode(const DecodeArgs& a, int num_sms, cudaStream_t stream)
 {
     const size_t entries = (size_t)1 << a.L;

@@ -130,6 +130,16 @@ tcq_status run_encode(EncodeArgs& a, tcq_dtype cb_dtype, void* workspace, size_t
     return e == cudaSuccess ? TCQ_OK : TCQ_ERR_CUDA;
 }
 
+// Vector trellis shapes: V weights per step, k V bits per step (at most 8,
+// one backpointer byte), V | T.
+tcq_status check_vec_shape(int L, int k, int V, int T)
+{
+    if (V < 1 || V > 8 || k < 1 || k > TCQ_MAX_K || k * V > 8 || k * V > L || L > TCQ_MAX_L)
+        return TCQ_ERR_UNSUPPORTED;
+    if (T < 1 || T > TCQ_MAX_T || T % V != 0) return TCQ_ERR_UNSUPPORTED;
+    return TCQ_OK;
+}
+
 // run_encode for a caller's codebook of any dtype (a computed code is written
 // to the front of the workspace first).
 tcq_status resolve_and_encode(EncodeArgs& a, tcq_dtype dt, void* workspace, size_t workspace_bytes,
@@ -347,7 +357,7 @@ tcq_status tcq_ldlq(const float* w, const float* u, const float* d, const void* 
         !aligned(path_cost, 4) || !aligned(workspace, 256))
         return TCQ_ERR_INVALID_ARG;
     // grid rows of the feedback product, and the block count of the code
-    if (rows > 65535LL * 128 || cols > ((int64_t)1 << 31)) return TCQ_ERR_INVALID_ARG;
+    if (rows > 65535LL * 128 || cols >= ((int64_t)1 << 31)) return TCQ_ERR_INVALID_ARG;
     const size_t targets = ((size_t)rows * (size_t)T * sizeof(float) + 255) & ~(size_t)255;
     if (workspace_bytes <= targets + mad_table_bytes(L, cb_dtype)) return TCQ_ERR_WORKSPACE;
     const int sms = current_sms();
@@ -468,6 +478,106 @@ tcq_status tcq_bcjr(const float* x, const float* d, const void* codebook, tcq_dt
     a.ws = ws;
     a.slot_bytes = slot;
     const cudaError_t e = launch_bcjr(a, (int)grid, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TCQ_OK : TCQ_ERR_CUDA;
+}
+
+size_t tcq_encode_vec_workspace_bytes(int L, int k, int V, int T, int64_t n_blocks,
+                                      tcq_dtype cb_dtype)
+{
+    if (V == 1) return tcq_encode_workspace_bytes(L, k, T, n_blocks, cb_dtype);
+    if (check_vec_shape(L, k, V, T) != TCQ_OK || n_blocks <= 0 ||
+        (cb_dtype != TCQ_F32 && cb_dtype != TCQ_F16))
+        return 0;
+    const EncodeKernelInfo* info = generic_kernel_info(L, k * V);
+    const long long ctas = wanted_ctas(info, L, k * V, T / V, n_blocks, current_sms());
+    return (size_t)ctas * info->slot_bytes(L, k * V, T / V);
+}
+
+tcq_status tcq_encode_vec(const float* x, const float* d, const void* codebook, tcq_dtype cb_dtype,
+                          int L, int k, int V, int T, int64_t n_blocks, uint32_t* start_state,
+                          uint32_t* bits, float* path_cost, void* workspace,
+                          size_t workspace_bytes, tcq_stream_t stream)
+{
+    if (V == 1)
+        return tcq_encode(x, d, codebook, cb_dtype, L, k, T, n_blocks, start_state, bits,
+                          path_cost, workspace, workspace_bytes, stream);
+    if (n_blocks < 0) return TCQ_ERR_INVALID_ARG;
+    if (cb_dtype == TCQ_MAD) return TCQ_ERR_UNSUPPORTED;  // the computed code is scalar
+    if (!valid_dtype(cb_dtype)) return TCQ_ERR_INVALID_ARG;
+    const tcq_status shape = check_vec_shape(L, k, V, T);
+    if (shape != TCQ_OK) return shape;
+    if (n_blocks == 0) return TCQ_OK;
+    if (!x || !codebook_ok(codebook, cb_dtype) || !start_state || !bits || !path_cost ||
+        !workspace)
+        return TCQ_ERR_INVALID_ARG;
+    if (!aligned(x, 4) || (d && !aligned(d, 4)) || !aligned(start_state, 4) ||
+        !aligned(bits, 4) || !aligned(path_cost, 4) || !aligned(workspace, 256))
+        return TCQ_ERR_INVALID_ARG;
+    if ((unsigned long long)n_blocks > (1ull << 40)) return TCQ_ERR_INVALID_ARG;
+    const EncodeKernelInfo* info = generic_kernel_info(L, k * V);
+    if (!info) return TCQ_ERR_INTERNAL;
+    const int sms = current_sms();
+    if (sms <= 0) return TCQ_ERR_CUDA;
+    const size_t slot = info->slot_bytes(L, k * V, T / V);
+    long long grid = wanted_ctas(info, L, k * V, T / V, n_blocks, sms);
+    const long long fit = (long long)(workspace_bytes / slot);
+    if (fit < 1) return TCQ_ERR_WORKSPACE;
+    if (grid > fit) grid = fit;
+    if (grid < 1) grid = 1;
+    EncodeArgs a;
+    a.x = x;
+    a.d = d;
+    a.cb = codebook;
+    a.cb_f16 = cb_dtype == TCQ_F16 ? 1 : 0;
+    a.L = L;
+    a.K = k;
+    a.T = T;
+    a.W = tcq_words_per_block(k, T);
+    a.n_blocks = n_blocks;
+    a.start_state = start_state;
+    a.bits = bits;
+    a.path_cost = path_cost;
+    a.x_stride = T;
+    a.d_stride = T;
+    a.out_stride = 1;
+    a.fixed_start = nullptr;
+    a.V = V;
+    a.ws = static_cast<unsigned char*>(workspace);
+    a.slot_bytes = slot;
+    const cudaError_t e = info->launch(a, (int)grid, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TCQ_OK : TCQ_ERR_CUDA;
+}
+
+tcq_status tcq_decode_vec(const uint32_t* bits, const uint32_t* start_state, const void* codebook,
+                          tcq_dtype cb_dtype, int L, int k, int V, int T, int64_t n_blocks,
+                          float* y, tcq_stream_t stream)
+{
+    if (V == 1) return tcq_decode(bits, start_state, codebook, cb_dtype, L, k, T, n_blocks, y, stream);
+    if (n_blocks < 0) return TCQ_ERR_INVALID_ARG;
+    if (cb_dtype == TCQ_MAD) return TCQ_ERR_UNSUPPORTED;
+    if (!valid_dtype(cb_dtype)) return TCQ_ERR_INVALID_ARG;
+    const tcq_status shape = check_vec_shape(L, k, V, T);
+    if (shape != TCQ_OK) return shape;
+    if (n_blocks == 0) return TCQ_OK;
+    if (!bits || !start_state || !codebook_ok(codebook, cb_dtype) || !y) return TCQ_ERR_INVALID_ARG;
+    if (!aligned(bits, 4) || !aligned(start_state, 4) || !aligned(y, 4)) return TCQ_ERR_INVALID_ARG;
+    if ((unsigned long long)n_blocks > (1ull << 40)) return TCQ_ERR_INVALID_ARG;
+    const int sms = current_sms();
+    if (sms <= 0) return TCQ_ERR_CUDA;
+    DecodeArgs a;
+    a.bits = bits;
+    a.start_state = start_state;
+    a.cb = codebook;
+    a.cb_f16 = cb_dtype == TCQ_F16 ? 1 : 0;
+    a.L = L;
+    a.K = k * V;
+    a.T = T;
+    a.W = tcq_words_per_block(k, T);
+    a.n_blocks = n_blocks;
+    a.y = y;
+    a.in_stride = 1;
+    a.y_stride = T;
+    const cudaError_t e = launch_decode_vec(a, V, sms, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TCQ_OK : TCQ_ERR_CUDA;
 }
 

@@ -72,6 +72,12 @@ def load_library() -> ctypes.CDLL:
     lib.tcq_encode_fixed_start.argtypes = [vp, vp, vp, ci, ci, ci, ci, i64, vp, vp, vp, vp, vp,
                                            sz, vp]
     lib.tcq_encode_fixed_start.restype = ci
+    lib.tcq_encode_vec_workspace_bytes.argtypes = [ci, ci, ci, ci, i64, ci]
+    lib.tcq_encode_vec_workspace_bytes.restype = sz
+    lib.tcq_encode_vec.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, i64, vp, vp, vp, vp, sz, vp]
+    lib.tcq_encode_vec.restype = ci
+    lib.tcq_decode_vec.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, i64, vp, vp]
+    lib.tcq_decode_vec.restype = ci
     lib.tcq_decode.argtypes = [vp, vp, vp, ci, ci, ci, ci, i64, vp, vp]
     lib.tcq_decode.restype = ci
     lib.tcq_status_string.argtypes = [ci]
@@ -122,6 +128,22 @@ def tcq_encode_fixed_start(x, d, codebook, cb_dtype, L, k, T, n_blocks, fixed_st
     return int(load_library().tcq_encode_fixed_start(x, d, codebook, cb_dtype, L, k, T, n_blocks,
                                                      fixed_start, start_state, bits, path_cost,
                                                      workspace, workspace_bytes, stream))
+
+
+def tcq_encode_vec_workspace_bytes(L, k, V, T, n_blocks, cb_dtype) -> int:
+    return int(load_library().tcq_encode_vec_workspace_bytes(L, k, V, T, n_blocks, cb_dtype))
+
+
+def tcq_encode_vec(x, d, codebook, cb_dtype, L, k, V, T, n_blocks, start_state, bits, path_cost,
+                   workspace, workspace_bytes, stream) -> int:
+    return int(load_library().tcq_encode_vec(x, d, codebook, cb_dtype, L, k, V, T, n_blocks,
+                                             start_state, bits, path_cost, workspace,
+                                             workspace_bytes, stream))
+
+
+def tcq_decode_vec(bits, start_state, codebook, cb_dtype, L, k, V, T, n_blocks, y, stream) -> int:
+    return int(load_library().tcq_decode_vec(bits, start_state, codebook, cb_dtype, L, k, V, T,
+                                             n_blocks, y, stream))
 
 
 def tcq_decode(bits, start_state, codebook, cb_dtype, L, k, T, n_blocks, y, stream) -> int:
@@ -349,6 +371,42 @@ def bcjr(x, d, codebook, L: int, k: int, tau: float, workspace=None, out=None, s
                     float(tau), _ptr(y), _ptr(F), ctypes.c_void_p(workspace.data_ptr()),
                     workspace.numel(), _stream_handle(stream)), "tcq_bcjr")
     return y, F
+
+
+def encode_vec(x, d, codebook, L: int, k: int, V: int, stream=None) -> Encoded:
+    """Viterbi TCQ over the vector trellis: V weights per step, codebook [2^L, V]."""
+    torch = _torch()
+    if x.dim() != 2 or x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous float32 CUDA tensor [n_blocks, T]")
+    n, T = x.shape
+    if d is not None and (d.shape != x.shape or d.dtype != torch.float32 or not d.is_contiguous()):
+        raise ValueError("d must be None or a contiguous float32 tensor shaped like x")
+    if codebook is not MAD and codebook.numel() != (1 << L) * V:
+        raise ValueError("codebook must hold 2^L rows of V entries")
+    W = max(tcq_words_per_block(k, T), 1)
+    out = Encoded(torch.empty(n, dtype=torch.int32, device=x.device),
+                  torch.empty((n, W), dtype=torch.int32, device=x.device),
+                  torch.empty(n, dtype=torch.float32, device=x.device))
+    nbytes = max(tcq_encode_vec_workspace_bytes(L, k, V, T, n, cb_dtype_of(codebook)), 256)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
+    _check(tcq_encode_vec(_ptr(x), _ptr(d), _ptr(codebook), cb_dtype_of(codebook), L, k, V, T, n,
+                          _ptr(out.start_state), _ptr(out.bits), _ptr(out.path_cost),
+                          ctypes.c_void_p(ws.data_ptr()), ws.numel(), _stream_handle(stream)),
+           "tcq_encode_vec")
+    return out
+
+
+def decode_vec(bits, start_state, codebook, L: int, k: int, V: int, T: int, stream=None):
+    """Values [n_blocks, T] of the vector trellis."""
+    torch = _torch()
+    n = start_state.shape[0]
+    W = tcq_words_per_block(k, T)
+    if bits.numel() < n * max(W, 0):
+        raise ValueError("decode_vec: bits holds fewer than n_blocks * W words")
+    out = torch.empty((n, T), dtype=torch.float32, device=bits.device)
+    _check(tcq_decode_vec(_ptr(bits), _ptr(start_state), _ptr(codebook), cb_dtype_of(codebook), L,
+                          k, V, T, n, _ptr(out), _stream_handle(stream)), "tcq_decode_vec")
+    return out
 
 
 class HostPipeline:
