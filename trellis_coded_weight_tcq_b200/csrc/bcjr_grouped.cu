@@ -16,9 +16,10 @@
 // The forward values of every step go to the workspace (coalesced 16-byte
 // stores); the backward pass brings each thread's own values for the next step
 // into private shared-memory slots with cp.async while it works on the current
-// step.  Per state and pass: one ex2 (the special-function unit bounds the
-// kernel), one lg2 per 2^k states, three FP32 operations for the branch
-// metric and two for the log-sum-exp.
+// step.  Per state: one ex2 per pass (three per four states in the forward
+// pass, where the maximum's term is exactly 1), one lg2 per 2^k states, three
+// FP32 operations for the branch metric and two for the log-sum-exp; the
+// special-function unit bounds the kernel.
 #include "acs_grouped.cuh"
 
 namespace tcq {
@@ -150,10 +151,20 @@ __global__ void __launch_bounds__(C::NT, 1) bcjr_grouped_kernel(BcjrArgs a)
                         const float e = diff(i, h, j, st.x);
                         c[h] = fmaf(-st.y * e, e, p[h]);
                     }
-                    const float m = hmax<H>(c);
-                    float s = 0.f;
+                    float m, s;
+                    if constexpr (H == 4) {
+                        // the maximum's term is exactly 1: the other three by a
+                        // min/max network, so three exponentials instead of four
+                        const float lo01 = fminf(c[0], c[1]), hi01 = fmaxf(c[0], c[1]);
+                        const float lo23 = fminf(c[2], c[3]), hi23 = fmaxf(c[2], c[3]);
+                        m = fmaxf(hi01, hi23);
+                        s = 1.f + ex2g(lo01 - m) + ex2g(lo23 - m) + ex2g(fminf(hi01, hi23) - m);
+                    } else {
+                        m = hmax<H>(c);
+                        s = 0.f;
 #pragma unroll
-                    for (int h = 0; h < H; ++h) s += ex2g(c[h] - m);
+                        for (int h = 0; h < H; ++h) s += ex2g(c[h] - m);
+                    }
                     out[j] = m + lg2g(s);
                     lmax = fmaxf(lmax, out[j]);
                 }
