@@ -5,13 +5,22 @@ The compute lives in the CUDA library ``libtcq.so`` (C ABI: ``include/tcq.h``);
 inputs.
 """
 from .tcq import (  # noqa: F401
+    MAD,
+    TCQ_F16,
+    TCQ_F32,
+    TCQ_MAD,
     Encoded,
     HostPipeline,
+    LdlqResult,
     TCQError,
     Workspace,
+    bcjr,
     decode,
+    decode_vec,
     encode,
+    encode_vec,
     gemv,
+    ldlq,
     load_library,
     tcq_decode,
     tcq_encode,
