@@ -139,6 +139,90 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a)
     }
 }
 
+// Compile-time (L, k, T) with T / 4 a multiple of 32: a warp decodes whole
+// blocks, and lane l always holds quads l, l + 32, ... of a block, so its
+// window offsets are constants; the four windows of a quad lie in one 32-bit
+// word once it is aligned ((4 - 1) k + L <= 32), so a state is one shift and one
+// mask.  The next block's words are loaded before the current block is written.
+template <int L, int K, int T, int MODE>
+__global__ void __launch_bounds__(kDecodeThreads) decode_fast_kernel(DecodeArgs a)
+{
+    constexpr int Q = T / 4;    // quads per block
+    constexpr int QPL = Q / 32; // quads per lane per block
+    constexpr int W = (T * K + 31) / 32;
+    constexpr uint32_t MASK = (1u << L) - 1u;
+    static_assert(Q % 32 == 0 && 3 * K + L <= 32, "shape");
+    extern __shared__ __align__(16) unsigned char dsm[];
+    const int n_entries = 1 << L;
+    if constexpr (MODE == kTableF32) {
+        float* tab = reinterpret_cast<float*>(dsm);
+        for (int i = threadIdx.x; i < n_entries; i += blockDim.x) tab[i] = load_codeword(a.cb, a.cb_f16, i);
+    } else if constexpr (MODE == kTableF16) {
+        const uint4* s4 = reinterpret_cast<const uint4*>(a.cb);
+        uint4* d4 = reinterpret_cast<uint4*>(dsm);
+        for (int i = threadIdx.x; i < n_entries / 8; i += blockDim.x) d4[i] = s4[i];
+    }
+    __syncthreads();
+    auto lookup = [&](uint32_t s) -> float {
+        if constexpr (MODE == kTableF32)
+            return reinterpret_cast<const float*>(dsm)[s];
+        else if constexpr (MODE == kTableF16)
+            return __half2float(reinterpret_cast<const __half*>(dsm)[s]);
+        else
+            return mad_codeword(s);
+    };
+    const int lane = threadIdx.x & 31;
+    int wi[QPL], off[QPL];
+#pragma unroll
+    for (int r = 0; r < QPL; ++r) {
+        const int p0 = (4 * (lane + 32 * r) + 1) * K - L;  // first window of the quad
+        wi[r] = p0 >> 5;                                    // -1: the start state
+        off[r] = p0 & 31;
+    }
+    const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+    long long b = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    uint32_t hi[QPL], lo[QPL];
+    auto fetch = [&](long long blk, uint32_t (&h)[QPL], uint32_t (&l)[QPL]) {
+        const uint32_t* wb = a.bits + blk * a.in_stride * W;
+#pragma unroll
+        for (int r = 0; r < QPL; ++r) {
+            h[r] = wi[r] < 0 ? a.start_state[blk * a.in_stride] : wb[wi[r]];
+            l[r] = wi[r] + 1 < W ? wb[wi[r] + 1] : 0u;
+        }
+    };
+    if (b < a.n_blocks) fetch(b, hi, lo);
+    while (b < a.n_blocks) {
+        const long long bn = b + nwarps;
+        uint32_t nhi[QPL], nlo[QPL];
+        if (bn < a.n_blocks) fetch(bn, nhi, nlo);
+        float* yb = a.y + b * a.y_stride;
+#pragma unroll
+        for (int r = 0; r < QPL; ++r) {
+            const uint32_t w = __funnelshift_l(lo[r], hi[r], off[r]);
+            float v[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) v[e] = lookup((w >> (32 - L - e * K)) & MASK);
+            __stcs(reinterpret_cast<float4*>(yb + 4 * (lane + 32 * r)), make_float4(v[0], v[1], v[2], v[3]));
+        }
+#pragma unroll
+        for (int r = 0; r < QPL; ++r) {
+            hi[r] = nhi[r];
+            lo[r] = nlo[r];
+        }
+        b = bn;
+    }
+}
+
+template <int L, int K, int T, int MODE>
+cudaError_t launch_fast(const DecodeArgs& a, int grid, size_t smem, cudaStream_t stream)
+{
+    cudaError_t e = cudaFuncSetAttribute(decode_fast_kernel<L, K, T, MODE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    decode_fast_kernel<L, K, T, MODE><<<grid, kDecodeThreads, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
 template <int MODE, bool VEC>
 cudaError_t launch_mode(const DecodeArgs& a, int grid, size_t smem, cudaStream_t stream)
 {
@@ -213,6 +297,22 @@ cudaError_t launch_decode(const DecodeArgs& a, int num_sms, cudaStream_t stream)
     if (grid < 1) grid = 1;
     const bool vec = (a.T % 4 == 0) && (a.y_stride % 4 == 0) &&
                      ((reinterpret_cast<uintptr_t>(a.y) & 15) == 0);
+    // compile-time shapes: whole blocks per warp, constant per-lane offsets
+    if (vec && mode != kTableGlobal && a.T == 256) {
+        long long fg = (long long)num_sms * ctas_per_sm;
+        const long long need = (a.n_blocks + kDecodeThreads / 32 - 1) / (kDecodeThreads / 32);
+        if (fg > need) fg = need;
+        if (fg < 1) fg = 1;
+#define TCQ_DECODE_FAST(LL, KK, MM) \
+        if (a.L == LL && a.K == KK && mode == MM) return launch_fast<LL, KK, 256, MM>(a, (int)fg, smem, stream);
+        TCQ_DECODE_FAST(16, 2, kTableF16)
+        TCQ_DECODE_FAST(16, 2, kTableMad)
+        TCQ_DECODE_FAST(16, 3, kTableF16)
+        TCQ_DECODE_FAST(16, 3, kTableMad)
+        TCQ_DECODE_FAST(12, 2, kTableF32)
+        TCQ_DECODE_FAST(12, 2, kTableMad)
+#undef TCQ_DECODE_FAST
+    }
     switch (mode * 2 + (vec ? 1 : 0)) {
     case 0: return launch_mode<kTableF32, false>(a, (int)grid, smem, stream);
     case 1: return launch_mode<kTableF32, true>(a, (int)grid, smem, stream);
