@@ -313,23 +313,24 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_fast_kernel(GemvArgs a)
     }
 }
 
-// Computed code, compile-time T as well: a warp takes whole rows, and within a
+// Compile-time (L, k, N) and T: a warp takes whole rows, and within a
 // row lane l always holds the same positions of every block (items l, l + 32,
 // ... of N weights), so each lane's window offsets are constants and a block's
 // words sit at fixed offsets from its base.  A warp walks its rows CH blocks at
 // a time and loads the next CH blocks' words (row boundaries included) while
 // it sums the current ones, so every lane keeps 2 CH loads in flight.  Per
-// weight: the state (a shift and a mask), one multiply, one byte dot product,
-// n - 255 as a float by its bits, and one FMA; the 2^-7 and the block scale
-// apply once per block.
+// weight: the state (a shift and a mask), the codeword, one FMA.  The computed
+// code's codeword is one multiply, one byte dot product and n - 255 as a float
+// by its bits (the 2^-7 applies once per block with the block scale); a table
+// code's is a shared-memory lookup.
 // 16 warps of up to 128 registers: eight blocks' words in flight per lane
 // (measured 27.1 us on the 14336 x 4096 matrix, against 29.0 us with four
 // blocks and 30.0 us with 32 warps of 64 registers)
-constexpr int kMadRowsChunk = 8;  // blocks per fetch of gemv_mad_rows_kernel
+constexpr int kMadRowsChunk = 8;  // blocks per fetch of gemv_rows_kernel
 constexpr int kMadRowsThreads = 512;
 
-template <int L, int K, int N, int T>
-__global__ void __launch_bounds__(kMadRowsThreads, 1) gemv_mad_rows_kernel(GemvArgs a)
+template <int L, int K, int N, int T, int CODE>
+__global__ void __launch_bounds__(kMadRowsThreads, 1) gemv_rows_kernel(GemvArgs a)
 {
     constexpr int IPB = T / N;  // items per block
     static_assert(IPB % 32 == 0 && (N - 1) * K + L <= 32 && N % 4 == 0, "shape");
@@ -338,7 +339,16 @@ __global__ void __launch_bounds__(kMadRowsThreads, 1) gemv_mad_rows_kernel(GemvA
     constexpr int CH = kMadRowsChunk;
     constexpr uint32_t MASK = (1u << L) - 1u;
     extern __shared__ __align__(16) unsigned char gsm[];
-    float* xs = reinterpret_cast<float*>(gsm);
+    constexpr size_t TAB = CODE == kCodeMad ? 0 : ((size_t(1) << L) * (CODE == kCodeF16 ? 2 : 4) + 15) & ~size_t(15);
+    float* xs = reinterpret_cast<float*>(gsm + TAB);
+    if constexpr (CODE == kCodeF16) {  // binary16 input, binary16 table
+        const uint4* s4 = reinterpret_cast<const uint4*>(a.cb);
+        uint4* d4 = reinterpret_cast<uint4*>(gsm);
+        for (int i = threadIdx.x; i < (1 << L) / 8; i += blockDim.x) d4[i] = s4[i];
+    } else if constexpr (CODE == kCodeF32) {
+        float* tab = reinterpret_cast<float*>(gsm);
+        for (int i = threadIdx.x; i < (1 << L); i += blockDim.x) tab[i] = load_codeword(a.cb, a.cb_f16, (uint32_t)i);
+    }
     for (long long i = threadIdx.x; i < a.cols; i += blockDim.x) xs[i] = a.x[i];
     __syncthreads();
 
@@ -392,9 +402,16 @@ __global__ void __launch_bounds__(kMadRowsThreads, 1) gemv_mad_rows_kernel(GemvA
 #pragma unroll
                     for (int g = 0; g < 4; ++g) {
                         const uint32_t st = (w >> (32 - L - (e + g) * K)) & MASK;
-                        // the byte sum lands on the bits of 2^23: 2^23 + n exactly
-                        const uint32_t nb23 = __dp4a(st * kMadA, 0x01010000u, 0x4B000000u);
-                        const float cv = __uint_as_float(nb23) - 8388863.0f;  // n - 255
+                        float cv;
+                        if constexpr (CODE == kCodeMad) {
+                            // the byte sum lands on the bits of 2^23: 2^23 + n exactly
+                            const uint32_t nb23 = __dp4a(st * kMadA, 0x01010000u, 0x4B000000u);
+                            cv = __uint_as_float(nb23) - 8388863.0f;  // n - 255
+                        } else if constexpr (CODE == kCodeF16) {
+                            cv = __half2float(reinterpret_cast<const __half*>(gsm)[st]);
+                        } else {
+                            cv = reinterpret_cast<const float*>(gsm)[st];
+                        }
                         if (g & 1)
                             p1 = fmaf(cv, xe[g], p1);
                         else
@@ -403,7 +420,8 @@ __global__ void __launch_bounds__(kMadRowsThreads, 1) gemv_mad_rows_kernel(GemvA
                 }
                 part += p0 + p1;
             }
-            acc = fmaf(f.sc[b] * 0.0078125f, part, acc);  // (n - 255) / 128
+            // (n - 255) / 128 for the computed code
+            acc = fmaf(CODE == kCodeMad ? f.sc[b] * 0.0078125f : f.sc[b], part, acc);
         }
         return acc;
     };
@@ -443,14 +461,15 @@ __global__ void __launch_bounds__(kMadRowsThreads, 1) gemv_mad_rows_kernel(GemvA
     }
 }
 
-template <int L, int K, int N, int T>
-cudaError_t launch_gemv_mad_rows(const GemvArgs& a, int grid, cudaStream_t stream)
+template <int L, int K, int N, int T, int CODE>
+cudaError_t launch_gemv_rows(const GemvArgs& a, int grid, cudaStream_t stream)
 {
-    const size_t smem = (size_t)a.cols * 4;
-    cudaError_t e = cudaFuncSetAttribute(gemv_mad_rows_kernel<L, K, N, T>,
+    const size_t tab = CODE == kCodeMad ? 0 : (((size_t)1 << L) * (CODE == kCodeF16 ? 2 : 4) + 15) & ~(size_t)15;
+    const size_t smem = tab + (size_t)a.cols * 4;
+    cudaError_t e = cudaFuncSetAttribute(gemv_rows_kernel<L, K, N, T, CODE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    gemv_mad_rows_kernel<L, K, N, T><<<grid, kMadRowsThreads, smem, stream>>>(a);
+    gemv_rows_kernel<L, K, N, T, CODE><<<grid, kMadRowsThreads, smem, stream>>>(a);
     return cudaGetLastError();
 }
 
@@ -493,11 +512,16 @@ cudaError_t launch_gemv(const GemvArgs& a, int num_sms, cudaStream_t stream)
     if (grid > num_sms) grid = num_sms;
     if (grid < 1) grid = 1;
     // computed code at T = 256: whole rows per warp, constant per-lane offsets
-    const bool rows_ok = mad && xsmem && a.T == 256 && (a.cols / 256) % kMadRowsChunk == 0;
-    if (rows_ok && a.L == 16 && a.K == 2)
-        return launch_gemv_mad_rows<16, 2, 8, 256>(a, (int)grid, stream);
-    if (rows_ok && a.L == 16 && a.K == 3)
-        return launch_gemv_mad_rows<16, 3, 4, 256>(a, (int)grid, stream);
+    // T = 256: whole rows per warp, constant per-lane offsets
+    const bool rows_ok = xsmem && a.T == 256 && (a.cols / 256) % kMadRowsChunk == 0;
+#define TCQ_GEMV_ROWS(LL, KK, NN, CC) \
+    if (rows_ok && a.L == LL && a.K == KK && code == CC) return launch_gemv_rows<LL, KK, NN, 256, CC>(a, (int)grid, stream);
+    TCQ_GEMV_ROWS(16, 2, 8, kCodeMad)
+    TCQ_GEMV_ROWS(16, 3, 4, kCodeMad)
+    TCQ_GEMV_ROWS(16, 2, 8, kCodeF16)
+    TCQ_GEMV_ROWS(16, 3, 4, kCodeF16)
+    TCQ_GEMV_ROWS(12, 2, 8, kCodeF32)
+#undef TCQ_GEMV_ROWS
     // specialised (L, k): compile-time shifts and masks, 8 or 4 weights per item
 #define TCQ_GEMV_FAST(LL, KK, NN, CC)                                                         \
     if (a.L == LL && a.K == KK && code == CC && a.T % NN == 0)                                 \
