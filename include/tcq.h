@@ -34,7 +34,9 @@
  *
  * Conventions for every entry point:
  *   - All array pointers are DEVICE pointers owned by the caller.  The library
- *     never allocates, never frees and keeps no global state (thread-safe).
+ *     never allocates, never frees and keeps no global state (thread-safe),
+ *     with one documented exception: tcq_encode_static_scratch's fixed device
+ *     array (see there).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
  *     default stream) and never synchronise.  Device-side failures surface on
  *     the stream like any kernel failure.
@@ -99,7 +101,7 @@ int tcq_words_per_block(int k, int T);
  * Workspace bytes tcq_encode wants for this problem on the CURRENT device
  * (enough for every persistent CTA the encoder would keep resident; it holds
  * the Viterbi backpointers, k bits per group of 2^k states per step, double
- * buffered per CTA).  Returns 0 for arguments tcq_encode would reject and for
+ * buffered per CTA, and for TCQ_MAD the code's binary16 table in front).  Returns 0 for arguments tcq_encode would reject and for
  * n_blocks == 0.  A smaller workspace is accepted down to one CTA's share: the
  * encoder then runs fewer CTAs, and slower.
  */
