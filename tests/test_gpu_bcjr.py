@@ -149,3 +149,20 @@ def test_bcjr_register_kernel_loops_over_blocks(cuda_device):
     y_tol, F_tol = _tolerances(T, cb.astype(np.float64), F_o, 0.2)
     assert np.abs(y1[[0, 4]] - y_o).max() <= y_tol
     assert np.all(np.abs(F1[[0, 4]] - F_o) <= F_tol)
+
+
+@pytest.mark.parametrize("L,k,T,cbt", [(16, 2, 64, "f16"), (10, 2, 40, "f32"), (8, 3, 30, "f32")])
+def test_bcjr_zero_weights_uniform(L, k, T, cbt, cuda_device):
+    """d = 0: uniform over paths, y_t = mean c, F = -tau (L + k (T - 1)) ln 2."""
+    rng = np.random.default_rng(9000 + L)
+    n, tau = 3, 0.4
+    x = rng.standard_normal((n, T)).astype(np.float32)
+    d = np.zeros((n, T), dtype=np.float32)
+    cb = rng.standard_normal(1 << L)
+    cb = cb.astype(np.float16) if cbt == "f16" else cb.astype(np.float32)
+    y, F = _run(x, d, cb, L, k, tau, cuda_device)
+    c64 = cb.astype(np.float64)
+    y_tol, _ = _tolerances(T, c64, np.zeros(n), tau)
+    assert np.abs(y - c64.mean()).max() <= y_tol
+    F_exact = -tau * (L + k * (T - 1)) * np.log(2.0)
+    np.testing.assert_allclose(F.astype(np.float64), F_exact, rtol=1e-6)

@@ -132,3 +132,15 @@ def test_soft_code_within_codebook_range_and_rejections():
     for bad_tau in (0.0, -1.0, float("inf"), float("nan")):
         with pytest.raises(ValueError):
             oracle_bcjr(np.zeros(4), None, cb, 8, 2, bad_tau)
+
+
+def test_zero_weights_are_uniform_over_paths():
+    """d = 0: every path has J = 0, so P is uniform over the 2^(L + k(T-1))
+    paths, every state equally likely at every step (y_t = mean c) and
+    F = -tau (L + k (T - 1)) ln 2."""
+    rng = np.random.default_rng(17)
+    L, k, T, tau = 6, 2, 9, 0.7
+    cb = rng.standard_normal(1 << L)
+    y, F = oracle_bcjr(rng.standard_normal(T), np.zeros(T), cb, L, k, tau)
+    np.testing.assert_allclose(y[0], np.full(T, cb.mean()), rtol=1e-12, atol=1e-14)
+    assert F[0] == pytest.approx(-tau * (L + k * (T - 1)) * np.log(2.0), rel=1e-12)
