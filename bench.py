@@ -498,7 +498,7 @@ def run_ours(args, rank, world, local_rank):
         "bound": "hbm", "kernel": "decode_kernel", "ms_per_launch": dec_ms,
         "achieved": dec_bytes / (dec_ms / 1e3) / 1e9, "peak": float(peaks.get("hbm_gbs", 6650.0)),
         "unit": "GB/s", "frac": dec_bytes / (dec_ms / 1e3) / 1e9 / float(peaks.get("hbm_gbs", 6650.0)),
-        "bytes_per_launch": dec_bytes,
+        "bytes_per_launch": dec_bytes, "weights_per_s": wl.weights / (dec_ms / 1e3),
     }
     cpu_baseline = None
     if pool is not None:
