@@ -389,6 +389,14 @@ struct Tracer {
     }
 };
 
+// CTA warp index of the w-th warp of team m (see the team mapping in the kernel)
+template <class C>
+__device__ __forceinline__ int team_warp(int m, int w)
+{
+    constexpr bool STRIDED = C::NTEAM > 1 && C::NT % 32 == 0 && C::NTEAM % 4 == 0;
+    return STRIDED ? m + C::NTEAM * w : ((m * C::NT) >> 5) + w;
+}
+
 // Sum of v over a team; the team's thread 0 gets the total.  Called by all
 // threads of the CTA (it contains __syncthreads for multi-warp teams).
 template <class C>
@@ -401,8 +409,7 @@ __device__ __forceinline__ double team_sum(double v, double* redd, int m, int ti
         __syncthreads();
         double r = 0.0;
         if (tid == 0) {
-            const int w0 = (m * C::NT) >> 5;
-            for (int w = 0; w < C::NT / 32; ++w) r += redd[w0 + w];
+            for (int w = 0; w < C::NT / 32; ++w) r += redd[team_warp<C>(m, w)];
         }
         __syncthreads();
         return r;
@@ -460,9 +467,8 @@ __device__ __forceinline__ float team_max(float v, float* redv, int m)
         for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
         if ((threadIdx.x & 31) == 0) redv[threadIdx.x >> 5] = v;
         __syncthreads();
-        const int w0 = (m * C::NT) >> 5;
-        float r = redv[w0];
-        for (int w = 1; w < C::NT / 32; ++w) r = fmaxf(r, redv[w0 + w]);
+        float r = redv[team_warp<C>(m, 0)];
+        for (int w = 1; w < C::NT / 32; ++w) r = fmaxf(r, redv[team_warp<C>(m, w)]);
         __syncthreads();
         return r;
     } else {
@@ -493,8 +499,13 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB) acs_grouped_kernel(Group
     unsigned char* slot = a.ws + (size_t)blockIdx.x * a.slot_bytes;
     const size_t team_bytes = C::team_bytes(T);
 
-    const int m = threadIdx.x / C::NT;    // team
-    const int tid = threadIdx.x % C::NT;  // thread within the team
+    // teams of whole warps take warps m, m + NTEAM, ...: a team's warps then share
+    // a scheduler (warp w issues from scheduler w mod 4) and wait for each other
+    // less at the team barrier
+    constexpr bool STRIDED = C::NTEAM > 1 && C::NT % 32 == 0 && C::NTEAM % 4 == 0;
+    const int m = STRIDED ? (int)((threadIdx.x >> 5) % C::NTEAM) : threadIdx.x / C::NT;  // team
+    const int tid = STRIDED ? (int)(((threadIdx.x >> 5) / C::NTEAM) * 32 + (threadIdx.x & 31))
+                            : threadIdx.x % C::NT;  // thread within the team
     // the team's first warp (or whole sub-warp team) runs the traceback in
     // lockstep: no divergent branch, the loads of all lanes hit one address
     const bool tracer = tid < 32;
@@ -526,6 +537,17 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB) acs_grouped_kernel(Group
         uint32_t bests = 0xffffffffu;
 
         unit_t* bpw = bp + tid;  // next backpointer record of this thread
+        // a team's steps depend only on its own metrics and staged inputs: with
+        // several warp-wide teams per CTA each syncs alone on a named barrier
+        auto team_sync = [&]() {
+            if constexpr (C::NTEAM == 1) {
+                __syncthreads();
+            } else if constexpr (C::NT % 32 == 0) {
+                named_barrier(1 + m, C::NT);
+            } else {  // teams narrower than a warp: measured faster with the CTA barrier
+                __syncthreads();
+            }
+        };
         // one trellis step; FIRST and LAST select the variant
         auto step = [&](auto first_tag, auto last_tag, int t) {
             constexpr bool FIRST = decltype(first_tag)::value;
@@ -550,7 +572,7 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB) acs_grouped_kernel(Group
                         }
                     }
                 }
-                __syncthreads();
+                team_sync();
             }
             const bool tracing = tracer && tr.b >= 0;
             if (tracing) tr.issue();
@@ -582,7 +604,7 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB) acs_grouped_kernel(Group
                 }
             }
             if (tracing && tr.retire(tid == 0)) tr.b = -1;
-            if (!LAST) __syncthreads();
+            if (!LAST) team_sync();
         };
         using T0 = std::false_type;
         using T1 = std::true_type;
@@ -609,10 +631,10 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB) acs_grouped_kernel(Group
             }
             __syncthreads();
             if (tid == 0) {
-                const int w0 = (m * C::NT) >> 5;
-                float bv = redv[w0];
-                uint32_t bs = reds[w0];
-                for (int w = 1; w < C::NT / 32; ++w) keep_best(redv[w0 + w], reds[w0 + w], bv, bs);
+                float bv = redv[team_warp<C>(m, 0)];
+                uint32_t bs = reds[team_warp<C>(m, 0)];
+                for (int w = 1; w < C::NT / 32; ++w)
+                    keep_best(redv[team_warp<C>(m, w)], reds[team_warp<C>(m, w)], bv, bs);
                 bests = bs;
             }
         } else {
