@@ -412,13 +412,15 @@ def decode_vec(bits, start_state, codebook, L: int, k: int, V: int, T: int, stre
 class HostPipeline:
     """End-to-end encode of host arrays: pinned host -> device -> encode -> host.
 
-    Buffers are allocated once; ``run`` copies one step's inputs in, encodes and
-    decodes on the device, and copies start states, bits, costs (and optionally
-    the decoded values) back, all on one stream.
+    Buffers are allocated once.  ``run`` splits the blocks into ``chunks`` parts:
+    a copy stream brings part i + 1's inputs in while the compute stream encodes
+    and decodes part i, and takes part i's start states, bits and costs back
+    while part i + 1 is encoded, so only the first part's input copy and the last
+    part's output copy are not hidden behind the encoder.
     """
 
     def __init__(self, n_blocks: int, T: int, L: int, k: int, weighted: bool, codebook_host,
-                 device=None, with_decode: bool = True):
+                 device=None, with_decode: bool = True, chunks: int = 8):
         torch = _torch()
         dev = torch.device(device or "cuda")
         self.L, self.k, self.T, self.n = L, k, T, n_blocks
@@ -426,7 +428,9 @@ class HostPipeline:
         self.x_dev = torch.empty((n_blocks, T), dtype=torch.float32, device=dev)
         self.d_dev = torch.empty((n_blocks, T), dtype=torch.float32, device=dev) if weighted else None
         self.cb_dev = codebook_host.to(dev)
-        self.ws = Workspace(L, k, T, n_blocks, cb_dtype_of(self.cb_dev), dev)
+        per = -(-n_blocks // max(1, chunks))
+        self.parts = [(lo, min(n_blocks, lo + per)) for lo in range(0, n_blocks, per)]
+        self.ws = Workspace(L, k, T, per, cb_dtype_of(self.cb_dev), dev)
         self.enc = Encoded(torch.empty(n_blocks, dtype=torch.int32, device=dev),
                            torch.empty((n_blocks, W), dtype=torch.int32, device=dev),
                            torch.empty(n_blocks, dtype=torch.float32, device=dev))
@@ -434,6 +438,9 @@ class HostPipeline:
         self.start_h = torch.empty(n_blocks, dtype=torch.int32, pin_memory=True)
         self.bits_h = torch.empty((n_blocks, W), dtype=torch.int32, pin_memory=True)
         self.cost_h = torch.empty(n_blocks, dtype=torch.float32, pin_memory=True)
+        self.copy_stream = torch.cuda.Stream(device=dev)
+        self.ev_in = [torch.cuda.Event() for _ in self.parts]
+        self.ev_done = [torch.cuda.Event() for _ in self.parts]
 
     def h2d_bytes(self) -> int:
         return self.x_dev.numel() * 4 + (self.d_dev.numel() * 4 if self.d_dev is not None else 0)
@@ -442,16 +449,37 @@ class HostPipeline:
         return (self.start_h.numel() + self.bits_h.numel() + self.cost_h.numel()) * 4
 
     def run(self, x_pinned, d_pinned=None, stream=None):
-        self.x_dev.copy_(x_pinned, non_blocking=True)
-        if self.d_dev is not None:
-            self.d_dev.copy_(d_pinned, non_blocking=True)
-        encode(self.x_dev, self.d_dev, self.cb_dev, self.L, self.k, self.ws, self.enc, stream)
-        if self.y_dev is not None:
-            decode(self.enc.bits, self.enc.start_state, self.cb_dev, self.L, self.k, self.T,
-                   self.y_dev, stream)
-        self.start_h.copy_(self.enc.start_state, non_blocking=True)
-        self.bits_h.copy_(self.enc.bits, non_blocking=True)
-        self.cost_h.copy_(self.enc.path_cost, non_blocking=True)
+        torch = _torch()
+        cs = self.copy_stream
+        ms = stream or torch.cuda.current_stream()
+        cs.wait_stream(ms)  # the previous run's readers of these buffers are done
+
+        def copy_in(i):
+            lo, hi = self.parts[i]
+            with torch.cuda.stream(cs):
+                self.x_dev[lo:hi].copy_(x_pinned[lo:hi], non_blocking=True)
+                if self.d_dev is not None:
+                    self.d_dev[lo:hi].copy_(d_pinned[lo:hi], non_blocking=True)
+                self.ev_in[i].record(cs)
+
+        copy_in(0)
+        for i, (lo, hi) in enumerate(self.parts):
+            if i + 1 < len(self.parts):
+                copy_in(i + 1)
+            ms.wait_event(self.ev_in[i])
+            part = Encoded(self.enc.start_state[lo:hi], self.enc.bits[lo:hi], self.enc.path_cost[lo:hi])
+            encode(self.x_dev[lo:hi], None if self.d_dev is None else self.d_dev[lo:hi], self.cb_dev,
+                   self.L, self.k, self.ws, part, ms)
+            if self.y_dev is not None:
+                decode(part.bits, part.start_state, self.cb_dev, self.L, self.k, self.T,
+                       self.y_dev[lo:hi], ms)
+            self.ev_done[i].record(ms)
+            with torch.cuda.stream(cs):
+                cs.wait_event(self.ev_done[i])
+                self.start_h[lo:hi].copy_(part.start_state, non_blocking=True)
+                self.bits_h[lo:hi].copy_(part.bits, non_blocking=True)
+                self.cost_h[lo:hi].copy_(part.path_cost, non_blocking=True)
+        ms.wait_stream(cs)
         return self.start_h, self.bits_h, self.cost_h
 
 
