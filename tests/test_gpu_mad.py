@@ -149,3 +149,24 @@ def test_workspace_holds_the_table_and_null_codebook(cuda_device):
     # a workspace too small for the table is refused before anything is launched
     assert tcq.tcq_encode(fake, None, None, tcq.TCQ_MAD, 16, 2, 256, 1, fake, fake, fake, fake,
                           100, None) == tcq.TCQ_ERR_WORKSPACE
+
+
+def test_fixed_start_with_computed_code(cuda_device):
+    import torch
+    from oracle import oracle_decode, oracle_encode, oracle_path_cost
+
+    L, k, T, n = 16, 2, 64, 6
+    rng = np.random.default_rng(7500)
+    x = rng.standard_normal((n, T)).astype(np.float32)
+    starts = rng.integers(0, 1 << (L - k), size=n).astype(np.uint32)
+    out = tcq.encode(torch.from_numpy(x).to(cuda_device), None, tcq.MAD, L, k,
+                     fixed_start=torch.from_numpy(starts.view(np.int32)).to(cuda_device))
+    torch.cuda.synchronize()
+    cb = _cb(L)
+    start = out.start_state.cpu().numpy().view(np.uint32)
+    bits = out.bits.cpu().numpy().view(np.uint32)
+    np.testing.assert_array_equal(start, starts)
+    for b in range(n):
+        _, _, J_o = oracle_encode(x[b:b + 1], None, cb, L, k, fixed_start=int(starts[b]))
+        J_g = oracle_path_cost(x[b:b + 1], None, oracle_decode(bits[b:b + 1], start[b:b + 1], cb, L, k, T))
+        assert abs(J_g[0] - J_o[0]) <= REL_TOL * J_o[0] + ABS_TOL_PER_D * T
