@@ -166,3 +166,20 @@ def test_bcjr_zero_weights_uniform(L, k, T, cbt, cuda_device):
     assert np.abs(y - c64.mean()).max() <= y_tol
     F_exact = -tau * (L + k * (T - 1)) * np.log(2.0)
     np.testing.assert_allclose(F.astype(np.float64), F_exact, rtol=1e-6)
+
+
+def test_bcjr_long_block_takes_the_runtime_kernel(cuda_device):
+    """T beyond the register-resident kernel's staged steps (1024) at L=16, k=2:
+    the runtime kernel, still against the oracle."""
+    from oracle import oracle_bcjr
+
+    L, k, T, n, tau = 16, 2, 1100, 1, 0.5
+    rng = np.random.default_rng(9100)
+    x = rng.standard_normal((n, T)).astype(np.float32)
+    d = rng.lognormal(0.0, 1.0, (n, T)).astype(np.float32)
+    cb = rng.standard_normal(1 << L).astype(np.float16)
+    y_g, F_g = _run(x, d, cb, L, k, tau, cuda_device)
+    y_o, F_o = oracle_bcjr(x, d, cb, L, k, tau)
+    y_tol, F_tol = _tolerances(T, cb.astype(np.float64), F_o, tau)
+    assert np.abs(y_g - y_o).max() <= y_tol
+    assert np.all(np.abs(F_g.astype(np.float64) - F_o) <= F_tol)

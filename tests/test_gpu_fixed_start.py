@@ -49,6 +49,8 @@ CASES = [
     (10, 3, 33, 20, "f32", True),     # runtime-(L,k) encoder
     (16, 2, 1, 9, "f16", True),       # T = 1: only the successors of s_0
     (6, 1, 7, 16, "f32", True),
+    (16, 2, 2048, 2, "f16", True),    # long blocks: the renormalising instantiation
+    (12, 2, 3000, 2, "f32", False),
 ]
 
 

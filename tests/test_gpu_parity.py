@@ -268,3 +268,27 @@ def test_empty_and_invalid_calls():
     torch.cuda.synchronize()
     # nothing launched by a rejected call, the stream is healthy
     assert torch.cuda.current_stream().query() in (True, False)
+
+
+def test_maximum_block_length():
+    """T = TCQ_MAX_T (2^20 weights in one block): staging chunks, backpointer
+    records and the traceback over a million steps, with path metrics that
+    would reach about 1e5 unless the kernel shifted them back towards 0."""
+    wl = workloads.small_random(8, 2, tcq.TCQ_MAX_T, 2, True, "f32", seed=4242)
+    start, bits, cost = gpu_encode(wl)
+    check_encode(wl, start, bits, cost)
+
+
+@pytest.mark.parametrize("L,k,T,cb", [
+    (16, 2, 4096, "f16"),   # register-resident encoder, its long-block instantiation
+    (16, 3, 2048, "f16"),
+    (12, 2, 8192, "f32"),
+    (16, 2, 1500, "f32"),   # runtime-(L,k) encoder
+    (16, 2, 1025, "f16"),   # one step past the threshold
+])
+def test_long_blocks(L, k, T, cb):
+    """Blocks longer than the renormalisation threshold (1024 steps) take the
+    renormalising code; the cost stays within the short blocks' tolerance."""
+    wl = workloads.small_random(L, k, T, 3, True, cb, seed=4300 + L + T)
+    start, bits, cost = gpu_encode(wl)
+    check_encode(wl, start, bits, cost)

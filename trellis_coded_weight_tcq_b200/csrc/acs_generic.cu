@@ -104,6 +104,14 @@ __global__ void __launch_bounds__(kGenericThreads) acs_generic_kernel(EncodeArgs
                 }
             }
             __syncthreads();
+            // long blocks: shift the metrics by state 0's every 64 steps
+            if (NS > kRenormAfter && (t & 63) == 0 && t < NS) {
+                const float o = Mn[0];
+                const float off = (o < __int_as_float(0x7f800000)) ? o : 0.f;
+                __syncthreads();
+                for (uint32_t u = threadIdx.x; u < NU; u += blockDim.x) Mn[u] -= off;
+                __syncthreads();
+            }
         }
         // final state: lexicographic (cost, state) minimum over the CTA
         for (int o = 16; o >= 1; o >>= 1) {

@@ -479,8 +479,10 @@ __device__ __forceinline__ float team_max(float v, float* redv, int m)
 }
 
 // FIXED: every block starts in a.fixed_start[b] (a separate instantiation, so the
-// free-start kernel carries none of it).
-template <class C, bool WEIGHTED, bool FIXED = false>
+// free-start kernel carries none of it).  LONG: blocks of more than kRenormAfter
+// steps, whose metrics are shifted every 64 steps; it reads a fixed start, if
+// any, at run time.
+template <class C, bool WEIGHTED, bool FIXED = false, bool LONG = false>
 __global__ void __launch_bounds__(C::NTHREADS, C::MINB) acs_grouped_kernel(GroupedArgs a)
 {
     using unit_t = typename C::unit_t;
@@ -583,6 +585,8 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB) acs_grouped_kernel(Group
                 uint32_t planes[C::K];
                 uint32_t s0 = 0xffffffffu;
                 if constexpr (FIRST && FIXED) s0 = a.fixed_start[b] & (uint32_t)(C::NU - 1);
+                if constexpr (FIRST && LONG)
+                    if (a.fixed_start) s0 = a.fixed_start[b] & (uint32_t)(C::NU - 1);
                 acs_step<C, WEIGHTED, FIRST, LAST>(cw, ax.x, ax.y, Mp, Mn, tid, planes, bestv, bests,
                                                    s0);
                 if constexpr (!LAST) {
@@ -605,6 +609,22 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB) acs_grouped_kernel(Group
             }
             if (tracing && tr.retire(tid == 0)) tr.b = -1;
             if (!LAST) team_sync();
+            if constexpr (LONG && !LAST) {
+                // long blocks: shift the team's metrics by state 0's every 64 steps
+                if ((t & 63) == 0) {
+                    float* Mn = Mteam + (t & 1) * C::NU;
+                    const float o = Mn[0];
+                    const float off = (o < __int_as_float(0x7f800000)) ? o : 0.f;
+                    team_sync();
+#pragma unroll
+                    for (int i = 0; i < C::GPT; ++i) {
+                        float* row = Mn + ((size_t)(tid + i * C::NT) << C::K);
+#pragma unroll
+                        for (int j = 0; j < C::H; ++j) row[j] -= off;
+                    }
+                    team_sync();
+                }
+            }
         };
         using T0 = std::false_type;
         using T1 = std::true_type;
@@ -670,14 +690,14 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB) acs_grouped_kernel(Group
     }
 }
 
-template <class C, bool WEIGHTED, bool FIXED = false>
+template <class C, bool WEIGHTED, bool FIXED = false, bool LONG = false>
 cudaError_t launch_grouped_w(const EncodeArgs& a, int grid, cudaStream_t stream)
 {
     const size_t smem = C::smem_bytes(a.L, a.K, a.T);
-    cudaError_t e = cudaFuncSetAttribute(acs_grouped_kernel<C, WEIGHTED, FIXED>,
+    cudaError_t e = cudaFuncSetAttribute(acs_grouped_kernel<C, WEIGHTED, FIXED, LONG>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    acs_grouped_kernel<C, WEIGHTED, FIXED><<<grid, C::NTHREADS, smem, stream>>>(grouped_args(a));
+    acs_grouped_kernel<C, WEIGHTED, FIXED, LONG><<<grid, C::NTHREADS, smem, stream>>>(grouped_args(a));
     return cudaGetLastError();
 }
 
@@ -687,6 +707,10 @@ cudaError_t launch_grouped(const EncodeArgs& a, int grid, cudaStream_t stream)
     // The fp16-pair kernels always run the weighted form (an absent d reads as 1,
     // every ratio d_{t-1}/d_t is then 1): measured faster than a separate
     // unweighted instantiation, whose schedule came out worse.
+    // blocks of more than kRenormAfter steps: the renormalising instantiation
+    // (weighted form, free or fixed start read at run time), kept apart so that
+    // the code of short blocks does not change
+    if (a.T > kRenormAfter) return launch_grouped_w<C, true, false, true>(a, grid, stream);
     if (a.fixed_start)  // weighted form: an absent d reads as 1
         return launch_grouped_w<C, true, true>(a, grid, stream);
     if constexpr (C::CB16)

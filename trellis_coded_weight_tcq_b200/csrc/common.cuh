@@ -40,6 +40,14 @@ __device__ __forceinline__ long long opaque(long long v)
     return r;
 }
 
+// Blocks longer than this many trellis steps have their path metrics shifted
+// by a common constant every 64 steps (state 0's metric), so that they stay
+// near 0, where fp32 still resolves the differences that decide each argmin;
+// without it a block of 2^20 steps grows metrics near 1e5 and loses about
+// 7e-5 of the optimal cost to mis-decided near-ties.  Costs are recomputed
+// along the traced path, so the shift does not reach them.
+constexpr int kRenormAfter = 1024;
+
 struct DecodeArgs {
     const uint32_t* bits;         // block b at bits + b * in_stride * W
     const uint32_t* start_state;  // block b at start_state[b * in_stride]
