@@ -20,6 +20,12 @@ CASES = [
     (16, 1, 2, 64, 3, "f16", True),    # metrics in the workspace
     (8, 4, 2, 16, 10, "f32", True),    # kV = L: no trellis memory
     (5, 1, 5, 35, 20, "f32", False),
+    # the compile-time kernel (L=16, k=2, V=2, binary16 pairs)
+    (16, 2, 2, 256, 3, "f16", True),
+    (16, 2, 2, 2, 5, "f16", True),      # one step
+    (16, 2, 2, 30, 4, "f16", False),    # 15 steps: a partial last word
+    (16, 2, 2, 514, 2, "f16", True),    # 257 steps: three staging chunks
+    (16, 2, 2, 2200, 1, "f16", True),   # 1100 steps: the renormalising instantiation
 ]
 
 
@@ -97,3 +103,51 @@ def test_vec_rejections(cuda_device):
     assert enc(V=9) == tcq.TCQ_ERR_UNSUPPORTED
     assert enc(dt=tcq.TCQ_MAD, cb=None) == tcq.TCQ_ERR_UNSUPPORTED
     assert enc(cb=None) == tcq.TCQ_ERR_INVALID_ARG
+
+
+def _vec_case(L, k, V, T, n, seed, device, cb_offset=0):
+    import torch
+
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((n, T)).astype(np.float32)
+    d = rng.lognormal(0.0, 1.0, (n, T)).astype(np.float32)
+    cb = rng.standard_normal((1 << L, V)).astype(np.float16)
+    cbt = torch.empty(cb.size + cb_offset, dtype=torch.float16, device=device)[cb_offset:]
+    cbt.copy_(torch.from_numpy(cb.reshape(-1)))
+    out = tcq.encode_vec(torch.from_numpy(x).to(device), torch.from_numpy(d).to(device), cbt, L, k, V)
+    torch.cuda.synchronize()
+    return x, d, cb, out
+
+
+def _check_vec_rows(x, d, cb, L, k, V, out, rows):
+    from oracle import oracle_decode_vec, oracle_encode_vec
+
+    T = x.shape[1]
+    start = out.start_state.cpu().numpy().view(np.uint32)
+    bits = out.bits.cpu().numpy().view(np.uint32)
+    cost = out.path_cost.cpu().numpy().astype(np.float64)
+    # every block: the reported cost is its own path's
+    y = oracle_decode_vec(bits, start, cb, L, k, V, T)
+    J_g = (d.astype(np.float64) * (x.astype(np.float64) - y) ** 2).sum(axis=1)
+    tol_all = REL_TOL * J_g + ABS_TOL_PER_D * d.astype(np.float64).sum(axis=1)
+    assert np.all(np.abs(cost - J_g) <= tol_all)
+    # sampled blocks: optimal
+    _, _, J_o = oracle_encode_vec(x[rows], d[rows], cb, L, k, V)
+    tol = REL_TOL * J_o + ABS_TOL_PER_D * d[rows].astype(np.float64).sum(axis=1)
+    assert np.all(np.abs(J_g[rows] - J_o) <= tol), float(np.max(np.abs(J_g[rows] - J_o) / J_o))
+
+
+def test_vec2_kernel_many_rounds(cuda_device):
+    """More blocks than CTAs: each CTA encodes several blocks in turn, tracing
+    one back while it searches the next (double-buffered backpointers)."""
+    L, k, V, T, n = 16, 2, 2, 64, 400
+    x, d, cb, out = _vec_case(L, k, V, T, n, 8300, cuda_device)
+    _check_vec_rows(x, d, cb, L, k, V, out, [0, 1, 147, 148, 149, 296, 398, 399])
+
+
+def test_vec2_unaligned_codebook_takes_the_runtime_kernel(cuda_device):
+    """A binary16 codebook that is not 4-byte aligned cannot be read as pairs:
+    the runtime kernel serves it, with the same optimum."""
+    L, k, V, T, n = 16, 2, 2, 48, 3
+    x, d, cb, out = _vec_case(L, k, V, T, n, 8400, cuda_device, cb_offset=1)
+    _check_vec_rows(x, d, cb, L, k, V, out, [0, 1, 2])

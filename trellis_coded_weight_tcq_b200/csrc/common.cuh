@@ -174,6 +174,9 @@ struct EncodeKernelInfo {
 // nullptr if no specialised grouped kernel exists for (L, k, codebook dtype).
 const EncodeKernelInfo* find_grouped_kernel(int L, int K, int cb_f16);
 const EncodeKernelInfo* generic_kernel_info(int L, int K);
+// nullptr if no compile-time vector-trellis kernel exists for (L, k, V, dtype);
+// its size callbacks take (L, k V, steps per block) like the runtime kernel's.
+const EncodeKernelInfo* find_vec_kernel(int L, int k, int V, int cb_f16);
 
 cudaError_t launch_feedback(const FeedbackArgs& a, cudaStream_t stream);
 size_t bcjr_slot_bytes(int L, int K, int T);

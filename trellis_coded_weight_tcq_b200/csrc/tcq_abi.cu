@@ -488,9 +488,17 @@ size_t tcq_encode_vec_workspace_bytes(int L, int k, int V, int T, int64_t n_bloc
     if (check_vec_shape(L, k, V, T) != TCQ_OK || n_blocks <= 0 ||
         (cb_dtype != TCQ_F32 && cb_dtype != TCQ_F16))
         return 0;
-    const EncodeKernelInfo* info = generic_kernel_info(L, k * V);
-    const long long ctas = wanted_ctas(info, L, k * V, T / V, n_blocks, current_sms());
-    return (size_t)ctas * info->slot_bytes(L, k * V, T / V);
+    // enough for whichever kernel the encode picks (the compile-time one needs a
+    // 4-byte aligned codebook, which the query cannot see)
+    size_t need = 0;
+    for (const EncodeKernelInfo* info : {find_vec_kernel(L, k, V, cb_dtype == TCQ_F16 ? 1 : 0),
+                                         generic_kernel_info(L, k * V)}) {
+        if (!info) continue;
+        const long long ctas = wanted_ctas(info, L, k * V, T / V, n_blocks, current_sms());
+        const size_t b = (size_t)ctas * info->slot_bytes(L, k * V, T / V);
+        if (b > need) need = b;
+    }
+    return need;
 }
 
 tcq_status tcq_encode_vec(const float* x, const float* d, const void* codebook, tcq_dtype cb_dtype,
@@ -514,7 +522,9 @@ tcq_status tcq_encode_vec(const float* x, const float* d, const void* codebook, 
         !aligned(bits, 4) || !aligned(path_cost, 4) || !aligned(workspace, 256))
         return TCQ_ERR_INVALID_ARG;
     if ((unsigned long long)n_blocks > (1ull << 40)) return TCQ_ERR_INVALID_ARG;
-    const EncodeKernelInfo* info = generic_kernel_info(L, k * V);
+    const EncodeKernelInfo* info =
+        find_vec_kernel(L, k, V, cb_dtype == TCQ_F16 && aligned(codebook, 4) ? 1 : 0);
+    if (!info) info = generic_kernel_info(L, k * V);
     if (!info) return TCQ_ERR_INTERNAL;
     const int sms = current_sms();
     if (sms <= 0) return TCQ_ERR_CUDA;
