@@ -28,6 +28,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "Viterbi trellis nodes/sec (blocks·T·2^L) and weights encoded/sec at L=16,k=2"
 ALGO_OPS_PER_NODE = 3  # error, square-accumulate, compare-select
+VEC_OPS_PER_NODE = 5   # V = 2: two errors, two square-accumulates, one compare-select
 SMS, LANES_PER_SM = 148, 128
 SFU_PER_SM = 16  # ex2 / lg2 results per SM per clock (4 per sub-partition)
 BCJR_TAU = 0.1
@@ -470,6 +471,40 @@ def run_ours(args, rank, world, local_rank):
                 "free_energy_mean": float(fe.astype(np.float64).mean())}
         del xb_t, db_t, bws, yb, fb
 
+    # ---- the vector trellis (V = 2 weights per step, 4 bits shifted in per step)
+    # over the same blocks, with a binary16 codebook of 2^16 pairs
+    vec = None
+    if rank == 0 and world == 1 and not args.no_vec and L == 16 and k == 2:
+        torch.cuda.empty_cache()
+        V = 2
+        xv_t = torch.from_numpy(wl.x).to(dev)
+        dv_t = None if wl.d is None else torch.from_numpy(wl.d).to(dev)
+        cbv = torch.from_numpy(workloads.gaussian_sample_codebook_f16((1 << L) * V)).to(dev)
+        vws = torch.empty(tcq.tcq_encode_vec_workspace_bytes(L, k, V, T, n, tcq.TCQ_F16),
+                          dtype=torch.uint8, device=dev)
+        vout = tcq.Encoded(torch.empty(n, dtype=torch.int32, device=dev),
+                           torch.empty((n, tcq.tcq_words_per_block(k, T)), dtype=torch.int32, device=dev),
+                           torch.empty(n, dtype=torch.float32, device=dev))
+        tcq.encode_vec(xv_t, dv_t, cbv, L, k, V, workspace=vws, out=vout)
+        v_ev = []
+        for _ in range(2):
+            a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            tcq.encode_vec(xv_t, dv_t, cbv, L, k, V, workspace=vws, out=vout)
+            b2.record(stream)
+            v_ev.append((a, b2))
+        torch.cuda.synchronize()
+        v_ms = sum(a.elapsed_time(b2) for a, b2 in v_ev) / len(v_ev)
+        vcost = vout.path_cost.cpu().numpy()
+        assert np.all(np.isfinite(vcost)) and np.all(vcost >= 0)
+        v_nodes = n * (T // V) * (1 << L)
+        vec = {"workload": wl.name + "_V2", "V": V, "ms": v_ms, "nodes_per_s": v_nodes / (v_ms / 1e3),
+               "weights_per_s": n * T / (v_ms / 1e3), "ops_per_node": VEC_OPS_PER_NODE,
+               "alu_frac": v_nodes * VEC_OPS_PER_NODE / (v_ms / 1e3) / peaks_ops(),
+               "kernel": "vec2<16,2,f16x2,512>",
+               "cost_per_weight": float(vcost.astype(np.float64).sum()) / (n * T)}
+        del xv_t, dv_t, vws, vout
+
     # sanity: the last step's result is a valid encode of the workload (cheap host check)
     cost_h = cost_last
     assert np.all(np.isfinite(cost_h)) and np.all(cost_h >= 0)
@@ -522,7 +557,7 @@ def run_ours(args, rank, world, local_rank):
         "weights_per_s": world * wl.weights / (ms / 1e3),
         "encode_ms_per_step": acs_ms, "decode_ms_per_step": dec_ms,
         "roofline": roofline, "decode_roofline": decode_roofline, "cpu_baseline": cpu_baseline, "e2e": e2e,
-        "per_workload": per_workload, "gemv": gemv, "ldlq": ldlq, "bcjr": bcjr,
+        "per_workload": per_workload, "gemv": gemv, "ldlq": ldlq, "bcjr": bcjr, "vec": vec,
         "clocks": clock_record, "remeasured": remeasured, "gpu_launches": gpu_launches,
     }
     print(json.dumps(line), flush=True)
@@ -541,6 +576,8 @@ def main():
                     help="skip the short encode/decode timing of the other named workloads")
     ap.add_argument("--no-bcjr", action="store_true",
                     help="skip the soft forward-backward quantization of the workload")
+    ap.add_argument("--no-vec", action="store_true",
+                    help="skip the vector-trellis (V = 2) encode of the workload")
     ap.add_argument("--no-ldlq", action="store_true",
                     help="skip the error-feedback encode of the MLP matrix")
     ap.add_argument("--cpu-blocks-per-core", type=int, default=16)

@@ -17,9 +17,10 @@
 // word (two binary16 halves); of a thread's 128 words, those of the first
 // kV2HR predecessors stay in registers for the whole kernel and the rest sit in
 // shared memory, thread-interleaved so that a warp's 16-byte loads are
-// contiguous.  Path metrics ping-pong in shared memory (2 x 16 KiB), read as 16
-// scalars per thread and step (conflict free: consecutive threads read
-// consecutive g) and written as two float4 per thread.
+// contiguous.  Path metrics ping-pong in shared memory (2 x 16 KiB), read as
+// 16 scalars per thread and step (conflict free: consecutive threads read
+// consecutive g) and written as two float4 per thread.  The kernel takes the
+// scalar encoders' 128-byte argument block.
 //
 // Per node: two mixed-precision subtractions (binary16 codeword minus fp32 x),
 // one product and two FMAs, with the metrics carried divided by the step's
@@ -38,7 +39,10 @@ namespace {
 
 constexpr int kV2Threads = 512;
 constexpr int kV2NU = 4096;                    // u values: 2^(L - kV)
-constexpr int kV2HR = 8;                       // predecessors with codewords in registers
+// predecessors whose codewords stay in registers: 4 (32 registers) measured 13 %
+// faster than 8 (11.74 vs 13.29 ms on 4736 blocks); fewer would overflow the
+// 227 KiB of shared memory
+constexpr int kV2HR = 4;
 constexpr int kV2SW = 16 - kV2HR;              // predecessors with codewords in shared memory
 constexpr int kV2ChunksPerJ = kV2SW / 4;       // 16-byte chunks per u value
 constexpr int kV2Chunks = 8 * kV2ChunksPerJ;   // 16-byte chunks per thread
@@ -158,12 +162,12 @@ struct V2Tracer {
 };
 
 // Bits, start state and fp64 cost of a traced block, by the whole CTA.
-__device__ __forceinline__ void v2_finish(const EncodeArgs& a, long long b,
+__device__ __forceinline__ void v2_finish(const GroupedArgs& a, long long b,
                                           const uint16_t* __restrict__ path, V2Smem& S, int NS)
 {
     const int tid = threadIdx.x;
-    const float* xb = a.x + b * a.x_stride;
-    const float* db = a.d ? a.d + b * a.d_stride : nullptr;
+    const float* xb = a.x + b * opaque(a.x_stride);
+    const float* db = a.d ? a.d + b * opaque(a.d_stride) : nullptr;
     const __half* cbh = reinterpret_cast<const __half*>(a.cb);
     double acc = 0.0;
     for (int t = tid; t < NS; t += kV2Threads) {
@@ -199,7 +203,7 @@ __device__ __forceinline__ void v2_finish(const EncodeArgs& a, long long b,
 // LONG: blocks of more than kRenormAfter steps, whose metrics are shifted
 // towards 0 every 64 steps (a separate instantiation, as in the scalar kernel).
 template <bool LONG>
-__global__ void __launch_bounds__(kV2Threads, 1) acs_vec2_kernel(EncodeArgs a)
+__global__ void __launch_bounds__(kV2Threads, 1) acs_vec2_kernel(GroupedArgs a)
 {
     extern __shared__ __align__(16) unsigned char smem[];
     V2Smem& S = *reinterpret_cast<V2Smem*>(smem);
@@ -239,8 +243,8 @@ __global__ void __launch_bounds__(kV2Threads, 1) acs_vec2_kernel(EncodeArgs a)
     for (int r = 0; r < R; ++r) {
         const long long b = first + (long long)r * stride;
         uint32_t* bp = reinterpret_cast<uint32_t*>(slot + (size_t)(r & 1) * recb);
-        const float* xb = a.x + b * a.x_stride;
-        const float* db = a.d ? a.d + b * a.d_stride : nullptr;
+        const float* xb = a.x + b * opaque(a.x_stride);
+        const float* db = a.d ? a.d + b * opaque(a.d_stride) : nullptr;
         float dm = 0.f;
         for (int q = tid; q < a.T; q += kV2Threads) dm = fmaxf(dm, db ? db[q] : 1.f);
 #pragma unroll
@@ -354,7 +358,7 @@ cudaError_t v2_launch_t(const EncodeArgs& a, int grid, cudaStream_t stream)
     cudaError_t e = cudaFuncSetAttribute(acs_vec2_kernel<LONG>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    acs_vec2_kernel<LONG><<<grid, kV2Threads, smem, stream>>>(a);
+    acs_vec2_kernel<LONG><<<grid, kV2Threads, smem, stream>>>(grouped_args(a));
     return cudaGetLastError();
 }
 

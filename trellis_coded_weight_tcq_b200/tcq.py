@@ -373,8 +373,14 @@ def bcjr(x, d, codebook, L: int, k: int, tau: float, workspace=None, out=None, s
     return y, F
 
 
-def encode_vec(x, d, codebook, L: int, k: int, V: int, stream=None) -> Encoded:
-    """Viterbi TCQ over the vector trellis: V weights per step, codebook [2^L, V]."""
+def encode_vec(x, d, codebook, L: int, k: int, V: int, workspace=None, out=None,
+               stream=None) -> Encoded:
+    """Viterbi TCQ over the vector trellis: V weights per step, codebook [2^L, V].
+
+    ``workspace`` (a uint8 CUDA tensor of at least tcq_encode_vec_workspace_bytes
+    for one block; more lets more blocks run at once) and ``out`` (an Encoded of
+    int32 start [n], int32 bits [n, W] and float32 cost [n]) are allocated when
+    not given."""
     torch = _torch()
     if x.dim() != 2 or x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
         raise ValueError("x must be a contiguous float32 CUDA tensor [n_blocks, T]")
@@ -384,11 +390,17 @@ def encode_vec(x, d, codebook, L: int, k: int, V: int, stream=None) -> Encoded:
     if codebook is not MAD and codebook.numel() != (1 << L) * V:
         raise ValueError("codebook must hold 2^L rows of V entries")
     W = max(tcq_words_per_block(k, T), 1)
-    out = Encoded(torch.empty(n, dtype=torch.int32, device=x.device),
-                  torch.empty((n, W), dtype=torch.int32, device=x.device),
-                  torch.empty(n, dtype=torch.float32, device=x.device))
-    nbytes = max(tcq_encode_vec_workspace_bytes(L, k, V, T, n, cb_dtype_of(codebook)), 256)
-    ws = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
+    if out is None:
+        out = Encoded(torch.empty(n, dtype=torch.int32, device=x.device),
+                      torch.empty((n, W), dtype=torch.int32, device=x.device),
+                      torch.empty(n, dtype=torch.float32, device=x.device))
+    elif (out.start_state.numel() < n or out.bits.numel() < n * W or out.path_cost.numel() < n):
+        raise ValueError("encode_vec: out is smaller than the blocks need")
+    if workspace is None:
+        nbytes = max(tcq_encode_vec_workspace_bytes(L, k, V, T, n, cb_dtype_of(codebook)), 256)
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
+    else:
+        ws = workspace
     _check(tcq_encode_vec(_ptr(x), _ptr(d), _ptr(codebook), cb_dtype_of(codebook), L, k, V, T, n,
                           _ptr(out.start_state), _ptr(out.bits), _ptr(out.path_cost),
                           ctypes.c_void_p(ws.data_ptr()), ws.numel(), _stream_handle(stream)),
