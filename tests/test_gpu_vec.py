@@ -151,3 +151,29 @@ def test_vec2_unaligned_codebook_takes_the_runtime_kernel(cuda_device):
     L, k, V, T, n = 16, 2, 2, 48, 3
     x, d, cb, out = _vec_case(L, k, V, T, n, 8400, cuda_device, cb_offset=1)
     _check_vec_rows(x, d, cb, L, k, V, out, [0, 1, 2])
+
+
+@pytest.mark.parametrize("pattern", ["first_zero", "second_zero", "sparse", "all_zero"])
+def test_vec2_zero_weights(pattern, cuda_device):
+    """Weights of 0 in the first coordinate force the kernel's floor on the
+    divisor of its metrics; in the second they zero the ratio; all zero makes
+    every path cost 0.  The optimum is still the oracle's."""
+    import torch
+
+    L, k, V, T, n = 16, 2, 2, 40, 3
+    rng = np.random.default_rng(8500 + len(pattern))
+    x = rng.standard_normal((n, T)).astype(np.float32)
+    d = rng.lognormal(0.0, 1.0, (n, T)).astype(np.float32)
+    if pattern == "first_zero":
+        d[:, 0::2] = 0.0
+    elif pattern == "second_zero":
+        d[:, 1::2] = 0.0
+    elif pattern == "sparse":
+        d[rng.random((n, T)) < 0.4] = 0.0
+    else:
+        d[:] = 0.0
+    cb = rng.standard_normal((1 << L, V)).astype(np.float16)
+    out = tcq.encode_vec(torch.from_numpy(x).to(cuda_device), torch.from_numpy(d).to(cuda_device),
+                         torch.from_numpy(cb).to(cuda_device), L, k, V)
+    torch.cuda.synchronize()
+    _check_vec_rows(x, d, cb, L, k, V, out, list(range(n)))
