@@ -144,6 +144,11 @@ def time_oracle(pool, cores, wl, blocks_per_core: int):
     return n, wall, float(sum(per_job))
 
 
+def peaks_hbm() -> float:
+    peaks, _ = _peaks()
+    return float(peaks.get("hbm_gbs", 6650.0))
+
+
 def peaks_ops() -> float:
     peaks, _ = _peaks()
     return SMS * LANES_PER_SM * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
@@ -498,10 +503,24 @@ def run_ours(args, rank, world, local_rank):
         vcost = vout.path_cost.cpu().numpy()
         assert np.all(np.isfinite(vcost)) and np.all(vcost >= 0)
         v_nodes = n * (T // V) * (1 << L)
+        # decode of the V = 2 stream: reads k/8 B and writes 4 B per weight
+        yv = tcq.decode_vec(vout.bits, vout.start_state, cbv, L, k, V, T)
+        vd_ev = []
+        for _ in range(3):
+            a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            tcq.decode_vec(vout.bits, vout.start_state, cbv, L, k, V, T, out=yv)
+            b2.record(stream)
+            vd_ev.append((a, b2))
+        torch.cuda.synchronize()
+        vd_ms = sum(a.elapsed_time(b2) for a, b2 in vd_ev) / len(vd_ev)
+        vd_bytes = n * T * 4 + n * tcq.tcq_words_per_block(k, T) * 4 + n * 4
+        del yv
         vec = {"workload": wl.name + "_V2", "V": V, "ms": v_ms, "nodes_per_s": v_nodes / (v_ms / 1e3),
                "weights_per_s": n * T / (v_ms / 1e3), "ops_per_node": VEC_OPS_PER_NODE,
                "alu_frac": v_nodes * VEC_OPS_PER_NODE / (v_ms / 1e3) / peaks_ops(),
                "kernel": "vec2<16,2,f16x2,512>",
+               "decode_ms": vd_ms, "decode_hbm_frac": vd_bytes / (vd_ms / 1e3) / 1e9 / peaks_hbm(),
                "cost_per_weight": float(vcost.astype(np.float64).sum()) / (n * T)}
         del xv_t, dv_t, vws, vout
 

@@ -61,17 +61,22 @@ def test_encode_vec_parity(case, cuda_device):
     np.testing.assert_array_equal(yg.cpu().numpy(), y.astype(np.float32))
 
 
-@pytest.mark.parametrize("L,k,V,T", [(8, 1, 2, 32), (12, 2, 2, 256), (16, 1, 4, 64), (9, 3, 2, 30)])
-def test_decode_vec_bit_exact(L, k, V, T, cuda_device):
+@pytest.mark.parametrize("L,k,V,T,cbt", [
+    (8, 1, 2, 32, "f32"), (12, 2, 2, 256, "f32"), (16, 1, 4, 64, "f32"), (9, 3, 2, 30, "f32"),
+    # the compile-time decoder (L=16, four bits per step, binary16 pairs, T % 8 == 0)
+    (16, 2, 2, 256, "f16"), (16, 2, 2, 8, "f16"), (16, 2, 2, 264, "f16"), (16, 2, 2, 1024, "f16"),
+    (16, 2, 2, 30, "f16"),    # T % 8 != 0: the runtime decoder
+])
+def test_decode_vec_bit_exact(L, k, V, T, cbt, cuda_device):
     import torch
     from oracle import oracle_decode_vec
 
-    rng = np.random.default_rng(8100 + L + V)
+    rng = np.random.default_rng(8100 + L + V + T)
     n = 33
     W = tcq.tcq_words_per_block(k, T)
     bits = rng.integers(0, 2**32, size=(n, W), dtype=np.uint64).astype(np.uint32)
     start = rng.integers(0, 2**32, size=n, dtype=np.uint64).astype(np.uint32)
-    cb = rng.standard_normal((1 << L, V)).astype(np.float32)
+    cb = rng.standard_normal((1 << L, V)).astype(np.float16 if cbt == "f16" else np.float32)
     y = tcq.decode_vec(torch.from_numpy(bits.view(np.int32)).to(cuda_device),
                        torch.from_numpy(start.view(np.int32)).to(cuda_device),
                        torch.from_numpy(cb).to(cuda_device), L, k, V, T)

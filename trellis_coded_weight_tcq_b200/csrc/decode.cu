@@ -258,8 +258,78 @@ __global__ void decode_vec_kernel(DecodeArgs a, int V)
     }
 }
 
+// The vector trellis at L = 16, four bits per step (k = 2, V = 2), binary16
+// pairs, one 32-bit word per state.  The 256 KiB table does not fit in shared
+// memory; its first three quarters (states below 0xC000, 192 KiB) are copied
+// there once per CTA and the rest is read through the read-only cache: a warp's
+// 32 random shared-memory reads cost a few bank passes where 32 random cache
+// lines cost 32 tag lookups (that bound the all-cache version at 0.32 of HBM).
+// A warp decodes 128 steps of a block at a time, lane l steps 4l+1 .. 4l+4:
+// their 16-bit windows end at stream bits 16l+3 .. 16l+15, so they lie in the
+// 64 bits of words (l >> 1) - 1 and l >> 1 of the chunk (word -1 of a block is
+// its start state), and the lane writes its 8 values as two 16-byte streaming
+// stores.  Needs T % 8 == 0 and a 16-byte aligned output; other shapes take
+// decode_vec_kernel.
+constexpr int kVec2DecThreads = 1024;
+constexpr uint32_t kVec2DecSmemStates = 0xC000u;
+
+__global__ void __launch_bounds__(kVec2DecThreads) decode_vec2_kernel(DecodeArgs a)
+{
+    extern __shared__ __align__(16) uint32_t tab[];  // [kVec2DecSmemStates]
+    const uint32_t* cb = reinterpret_cast<const uint32_t*>(a.cb);
+    {
+        const uint4* src = reinterpret_cast<const uint4*>(cb);
+        uint4* dst = reinterpret_cast<uint4*>(tab);
+        for (int i = threadIdx.x; i < (int)(kVec2DecSmemStates / 4); i += blockDim.x) dst[i] = __ldg(src + i);
+    }
+    __syncthreads();
+    const int NS = a.T >> 1;
+    const int chunks = (NS + 127) >> 7;
+    const long long items = a.n_blocks * chunks;
+    const int lane = threadIdx.x & 31;
+    for (long long it = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; it < items;
+         it += ((long long)gridDim.x * blockDim.x) >> 5) {
+        const long long b = it / chunks;
+        const int c = (int)(it - b * chunks);
+        const int t0 = (c << 7) + 4 * lane;  // steps t0+1 .. t0+4
+        if (t0 + 4 > NS) continue;           // NS % 4 == 0: a lane's steps are all in or all out
+        const uint32_t* wb = a.bits + b * a.W;
+        const int wi = (c << 4) + (lane >> 1);  // word holding the lane's last window end
+        const unsigned long long hi = wi >= 1 ? __ldg(wb + wi - 1) : __ldg(a.start_state + b);
+        const unsigned long long v = (hi << 32) | __ldg(wb + wi);
+        float y[8];
+#pragma unroll
+        for (int q = 1; q <= 4; ++q) {
+            // window start relative to bit 0 of v: 16 (lane & 1) + 4q + 16
+            const int sh = 48 - (16 * (lane & 1) + 4 * q + 16);
+            const uint32_t s = (uint32_t)(v >> sh) & 0xffffu;
+            const uint32_t w = s < kVec2DecSmemStates ? tab[s] : __ldg(cb + s);
+            const __half2 h2 = *reinterpret_cast<const __half2*>(&w);
+            const float2 f = __half22float2(h2);
+            y[2 * q - 2] = f.x;
+            y[2 * q - 1] = f.y;
+        }
+        float4* dst = reinterpret_cast<float4*>(a.y + b * a.y_stride + 2 * (long long)t0);
+        __stcs(dst, make_float4(y[0], y[1], y[2], y[3]));
+        __stcs(dst + 1, make_float4(y[4], y[5], y[6], y[7]));
+    }
+}
+
 cudaError_t launch_decode_vec(const DecodeArgs& a, int V, int num_sms, cudaStream_t stream)
 {
+    if (a.L == 16 && a.K == 4 && V == 2 && a.cb_f16 == 1 && a.T % 8 == 0 && a.y_stride % 4 == 0 &&
+        (reinterpret_cast<uintptr_t>(a.y) & 15) == 0 && (reinterpret_cast<uintptr_t>(a.cb) & 15) == 0) {
+        const size_t smem = kVec2DecSmemStates * sizeof(uint32_t);
+        const cudaError_t e = cudaFuncSetAttribute(decode_vec2_kernel,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        const long long warps = a.n_blocks * ((a.T / 2 + 127) / 128);
+        long long grid = (warps + kVec2DecThreads / 32 - 1) / (kVec2DecThreads / 32);
+        if (grid > num_sms) grid = num_sms;  // one CTA per SM: the table copy is paid once per SM
+        if (grid < 1) grid = 1;
+        decode_vec2_kernel<<<(int)grid, kVec2DecThreads, smem, stream>>>(a);
+        return cudaGetLastError();
+    }
     const long long total = a.n_blocks * (a.T / V);
     long long grid = (total + 255) / 256;
     const long long cap = (long long)num_sms * 8;

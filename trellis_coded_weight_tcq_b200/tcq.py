@@ -408,14 +408,17 @@ def encode_vec(x, d, codebook, L: int, k: int, V: int, workspace=None, out=None,
     return out
 
 
-def decode_vec(bits, start_state, codebook, L: int, k: int, V: int, T: int, stream=None):
-    """Values [n_blocks, T] of the vector trellis."""
+def decode_vec(bits, start_state, codebook, L: int, k: int, V: int, T: int, out=None, stream=None):
+    """Values [n_blocks, T] of the vector trellis (into ``out`` when given)."""
     torch = _torch()
     n = start_state.shape[0]
     W = tcq_words_per_block(k, T)
     if bits.numel() < n * max(W, 0):
         raise ValueError("decode_vec: bits holds fewer than n_blocks * W words")
-    out = torch.empty((n, T), dtype=torch.float32, device=bits.device)
+    if out is None:
+        out = torch.empty((n, T), dtype=torch.float32, device=bits.device)
+    elif out.numel() < n * T or out.dtype != torch.float32 or not out.is_contiguous():
+        raise ValueError("decode_vec: out must be a contiguous float32 tensor of n_blocks * T")
     _check(tcq_decode_vec(_ptr(bits), _ptr(start_state), _ptr(codebook), cb_dtype_of(codebook), L,
                           k, V, T, n, _ptr(out), _stream_handle(stream)), "tcq_decode_vec")
     return out
