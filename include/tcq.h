@@ -280,9 +280,14 @@ tcq_status tcq_bcjr(const float* x, const float* d, const void* codebook, tcq_dt
  *   codebook  2^L rows of V entries (row-major), binary32 or binary16; the
  *             computed code (TCQ_MAD) is scalar: TCQ_ERR_UNSUPPORTED for V > 1.
  * Supported: 1 <= V <= 8, V | T, k V <= min(L, 8) (else TCQ_ERR_UNSUPPORTED).
- * V == 1 is exactly tcq_encode / tcq_decode.  V > 1 runs the runtime-(L, k)
- * kernel (not tuned).  Other arguments, outputs and errors as tcq_encode /
- * tcq_decode.
+ * V == 1 is exactly tcq_encode / tcq_decode.  L = 16, k = 2, V = 2 with a
+ * binary16 codebook runs compile-time kernels: the encoder when the codebook is
+ * 4-byte aligned, the decoder when it is 16-byte aligned, T % 8 == 0 and y is
+ * 16-byte aligned; every other V > 1 shape runs the runtime-(L, k) kernels.
+ * Results do not depend on which kernel runs beyond fp32 rounding of the search
+ * (costs within the tolerance of tcq_encode; decode is exact either way), and
+ * the workspace query covers either encoder.  Other arguments, outputs and
+ * errors as tcq_encode / tcq_decode.
  */
 size_t tcq_encode_vec_workspace_bytes(int L, int k, int V, int T, int64_t n_blocks,
                                       tcq_dtype cb_dtype);
