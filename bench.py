@@ -516,11 +516,40 @@ def run_ours(args, rank, world, local_rank):
         vd_ms = sum(a.elapsed_time(b2) for a, b2 in vd_ev) / len(vd_ev)
         vd_bytes = n * T * 4 + n * tcq.tcq_words_per_block(k, T) * 4 + n * 4
         del yv
+        # decode-in-matvec over the matrix those blocks tile (rows x cols), timed
+        # like the scalar product above (unit block scales, best of 10)
+        vgemv = None
+        vmat = wl.meta.get("matrix")
+        if vmat and (n * T) % int(vmat[1]) == 0:
+            g_cols = int(vmat[1])
+            g_rows = n * T // g_cols
+            xg = torch.randn(g_cols, device=dev)
+            sg = torch.ones(n, device=dev)
+            yg = torch.empty(g_rows, device=dev)
+            for _ in range(3):
+                tcq.gemv_vec(vout.bits, vout.start_state, sg, cbv, L, k, V, T, g_rows, g_cols, xg, out=yg)
+            vg_ev = []
+            for _ in range(10):
+                a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                tcq.gemv_vec(vout.bits, vout.start_state, sg, cbv, L, k, V, T, g_rows, g_cols, xg, out=yg)
+                b2.record(stream)
+                vg_ev.append((a, b2))
+            torch.cuda.synchronize()
+            vg_ms = min(a.elapsed_time(b2) for a, b2 in vg_ev)
+            vg_bytes = n * tcq.tcq_words_per_block(k, T) * 4 + n * 8 + g_cols * 4 + g_rows * 4
+            assert bool(torch.isfinite(yg).all())
+            vgemv = {"rows": g_rows, "cols": g_cols, "ms": vg_ms,
+                     "weights_per_s": g_rows * g_cols / (vg_ms / 1e3),
+                     "hbm_gbs": vg_bytes / (vg_ms / 1e3) / 1e9,
+                     "hbm_frac": vg_bytes / (vg_ms / 1e3) / 1e9 / peaks_hbm()}
+            del xg, yg, sg
         vec = {"workload": wl.name + "_V2", "V": V, "ms": v_ms, "nodes_per_s": v_nodes / (v_ms / 1e3),
                "weights_per_s": n * T / (v_ms / 1e3), "ops_per_node": VEC_OPS_PER_NODE,
                "alu_frac": v_nodes * VEC_OPS_PER_NODE / (v_ms / 1e3) / peaks_ops(),
                "kernel": "vec2<16,2,f16x2,512>",
                "decode_ms": vd_ms, "decode_hbm_frac": vd_bytes / (vd_ms / 1e3) / 1e9 / peaks_hbm(),
+               "gemv": vgemv,
                "cost_per_weight": float(vcost.astype(np.float64).sum()) / (n * T)}
         del xv_t, dv_t, vws, vout
 

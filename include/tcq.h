@@ -301,6 +301,22 @@ tcq_status tcq_decode_vec(const uint32_t* bits, const uint32_t* start_state, con
                           tcq_dtype cb_dtype, int L, int k, int V, int T, int64_t n_blocks,
                           float* y, tcq_stream_t stream);
 
+/*
+ * Decode-in-matvec for the vector trellis: tcq_gemv's product, with each
+ * block's weights those of tcq_decode_vec (step t of block (r, j) holds columns
+ * jT + (t-1)V .. jT + tV - 1):
+ *     y[r] = sum_j scale[r, j] * sum_t sum_v c[s_{r,j,t}][v] * x[jT + (t-1)V + v]
+ * accumulated in fp32.  Arguments as tcq_gemv plus V; shapes as tcq_encode_vec
+ * (TCQ_MAD is TCQ_ERR_UNSUPPORTED for V > 1); cols % T == 0 (else
+ * TCQ_ERR_INVALID_ARG); V == 1 is exactly tcq_gemv.  L = 16, k = 2, V = 2 with a
+ * 16-byte aligned binary16 codebook and T % 8 == 0 runs a compile-time kernel
+ * (seven eighths of the pair table in shared memory), every other shape a
+ * runtime kernel.  rows == 0 is a no-op.
+ */
+tcq_status tcq_gemv_vec(const uint32_t* bits, const uint32_t* start_state, const float* scale,
+                        const void* codebook, tcq_dtype cb_dtype, int L, int k, int V, int T,
+                        int64_t rows, int64_t cols, const float* x, float* y, tcq_stream_t stream);
+
 /* Static, human-readable name of a status code. */
 const char* tcq_status_string(tcq_status status);
 

@@ -182,3 +182,98 @@ def test_vec2_zero_weights(pattern, cuda_device):
                          torch.from_numpy(cb).to(cuda_device), L, k, V)
     torch.cuda.synchronize()
     _check_vec_rows(x, d, cb, L, k, V, out, list(range(n)))
+
+
+def _gemv_vec_check(bits, start, scale, cb, L, k, V, T, rows, cols, x, y):
+    """The oracle's decode of every block, scaled, times x in fp64; bound: each
+    product passes through at most 8 ceil(NS/128) + V ceil(NS/32) fp32 roundings
+    in its lane's block sum, one per block in the row sum and 5 in the warp
+    reduction (NS = T / V steps per block)."""
+    from oracle import oracle_decode_vec
+
+    nb = cols // T
+    vals = oracle_decode_vec(bits, start, cb, L, k, V, T).reshape(rows, cols)
+    sc = np.ones(rows * nb) if scale is None else scale.astype(np.float64)
+    m = vals * np.repeat(sc.reshape(rows, nb), T, axis=1)
+    y_o = m @ x.astype(np.float64)
+    NS = T // V
+    n_round = 8 * -(-NS // 128) + V * -(-NS // 32) + nb + 8
+    bound = n_round * 2.0**-24 * np.abs(m * x.astype(np.float64)).sum(axis=1)
+    err = np.abs(y.astype(np.float64) - y_o)
+    assert np.all(err <= bound + 1e-30), float(np.max(err / np.maximum(bound, 1e-30)))
+
+
+@pytest.mark.parametrize("L,k,V,T,rows,nb,cbt,cb_offset", [
+    (16, 2, 2, 256, 300, 16, "f16", 0),   # compile-time kernel, the MLP shape's blocks
+    (16, 2, 2, 264, 37, 5, "f16", 0),     # 132 steps: a partial second chunk
+    (16, 2, 2, 256, 40, 4, "f16", 1),     # unaligned table: runtime kernel
+    (16, 2, 2, 30, 20, 3, "f16", 0),      # T % 8 != 0: runtime kernel
+    (12, 2, 2, 64, 50, 6, "f32", 0),
+    (8, 1, 4, 32, 33, 7, "f16", 0),
+])
+@pytest.mark.parametrize("scaled", [False, True])
+def test_gemv_vec(L, k, V, T, rows, nb, cbt, cb_offset, scaled, cuda_device):
+    import torch
+    from tests.test_gpu_gemv import _rand_stream
+
+    rng = np.random.default_rng(8600 + L + T + rows + V)
+    cols = nb * T
+    bits, start = _rand_stream(rng, rows * nb, k * V, T // V)
+    cb = rng.standard_normal((1 << L, V)).astype(np.float16 if cbt == "f16" else np.float32)
+    scale = rng.lognormal(0.0, 0.5, rows * nb).astype(np.float32) if scaled else None
+    x = rng.standard_normal(cols).astype(np.float32)
+    cbt_dev = torch.empty(cb.size + cb_offset, dtype=torch.from_numpy(cb).dtype,
+                          device=cuda_device)[cb_offset:]
+    cbt_dev.copy_(torch.from_numpy(cb.reshape(-1)))
+    y = tcq.gemv_vec(torch.from_numpy(bits.view(np.int32)).to(cuda_device),
+                     torch.from_numpy(start.view(np.int32)).to(cuda_device),
+                     None if scale is None else torch.from_numpy(scale).to(cuda_device),
+                     cbt_dev, L, k, V, T, rows, cols, torch.from_numpy(x).to(cuda_device))
+    torch.cuda.synchronize()
+    _gemv_vec_check(bits, start, scale, cb, L, k, V, T, rows, cols, x, y.cpu().numpy())
+
+
+def test_gemv_vec_of_encoded_matrix(cuda_device):
+    """Encode a matrix with the vector encoder and multiply through its bits: the
+    product equals the decoded matrix times x within the bound."""
+    import torch
+
+    L, k, V, T, rows, nb = 16, 2, 2, 256, 24, 4
+    cols = nb * T
+    rng = np.random.default_rng(8700)
+    w = rng.standard_normal((rows, cols)).astype(np.float32)
+    cb = rng.standard_normal((1 << L, V)).astype(np.float16)
+    cbd = torch.from_numpy(cb).to(cuda_device)
+    enc = tcq.encode_vec(torch.from_numpy(w.reshape(rows * nb, T)).to(cuda_device), None, cbd, L, k, V)
+    x = rng.standard_normal(cols).astype(np.float32)
+    y = tcq.gemv_vec(enc.bits, enc.start_state, None, cbd, L, k, V, T, rows, cols,
+                     torch.from_numpy(x).to(cuda_device))
+    torch.cuda.synchronize()
+    _gemv_vec_check(enc.bits.cpu().numpy().view(np.uint32), enc.start_state.cpu().numpy().view(np.uint32),
+                    None, cb, L, k, V, T, rows, cols, x, y.cpu().numpy())
+
+
+def test_gemv_vec_v1_and_rejections(cuda_device):
+    import torch
+    from tests.test_gpu_gemv import _rand_stream
+
+    rng = np.random.default_rng(8800)
+    L, k, T, rows, nb = 12, 2, 64, 10, 3
+    bits, start = _rand_stream(rng, rows * nb, k, T)
+    cb = torch.from_numpy(rng.standard_normal(1 << L).astype(np.float32)).to(cuda_device)
+    x = torch.from_numpy(rng.standard_normal(nb * T).astype(np.float32)).to(cuda_device)
+    b = torch.from_numpy(bits.view(np.int32)).to(cuda_device)
+    s = torch.from_numpy(start.view(np.int32)).to(cuda_device)
+    y1 = tcq.gemv(b, s, None, cb, L, k, T, rows, nb * T, x)
+    yv = tcq.gemv_vec(b, s, None, cb, L, k, 1, T, rows, nb * T, x)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, yv)
+    fake = ctypes.c_void_p(0x10000)
+    call = lambda **o: tcq.tcq_gemv_vec(fake, fake, None, o.get("cb", fake), o.get("dt", tcq.TCQ_F32),  # noqa: E731
+                                        o.get("L", 8), o.get("k", 2), o.get("V", 2), o.get("T", 32),
+                                        o.get("rows", 4), o.get("cols", 64), fake, fake, None)
+    assert call(dt=tcq.TCQ_MAD, cb=None) == tcq.TCQ_ERR_UNSUPPORTED
+    assert call(cols=48) == tcq.TCQ_ERR_INVALID_ARG        # cols % T != 0
+    assert call(T=33) == tcq.TCQ_ERR_UNSUPPORTED           # V does not divide T
+    assert call(V=9) == tcq.TCQ_ERR_UNSUPPORTED
+    assert call(rows=0) == tcq.TCQ_OK

@@ -20,6 +20,7 @@ from .tcq import (  # noqa: F401
     encode,
     encode_vec,
     gemv,
+    gemv_vec,
     ldlq,
     load_library,
     tcq_decode,
@@ -27,6 +28,7 @@ from .tcq import (  # noqa: F401
     tcq_encode_path,
     tcq_encode_workspace_bytes,
     tcq_gemv,
+    tcq_gemv_vec,
     tcq_status_string,
     tcq_words_per_block,
 )

@@ -185,6 +185,7 @@ cudaError_t launch_bcjr(const BcjrArgs& a, int grid, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, int num_sms, cudaStream_t stream);
 // vector trellis: a.K = k V bits per step, a.T weights per block (V | T)
 cudaError_t launch_decode_vec(const DecodeArgs& a, int V, int num_sms, cudaStream_t stream);
+cudaError_t launch_gemv_vec(const GemvArgs& a, int V, int num_sms, cudaStream_t stream);
 cudaError_t launch_gemv(const GemvArgs& a, int num_sms, cudaStream_t stream);
 
 }  // namespace tcq

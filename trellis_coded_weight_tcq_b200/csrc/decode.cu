@@ -260,10 +260,11 @@ __global__ void decode_vec_kernel(DecodeArgs a, int V)
 
 // The vector trellis at L = 16, four bits per step (k = 2, V = 2), binary16
 // pairs, one 32-bit word per state.  The 256 KiB table does not fit in shared
-// memory; its first three quarters (states below 0xC000, 192 KiB) are copied
+// memory; its first seven eighths (states below 0xE000, 224 KiB) are copied
 // there once per CTA and the rest is read through the read-only cache: a warp's
 // 32 random shared-memory reads cost a few bank passes where 32 random cache
-// lines cost 32 tag lookups (that bound the all-cache version at 0.32 of HBM).
+// lines cost 32 tag lookups (the all-cache version reached 0.32 of HBM, three
+// quarters in shared memory 0.46, seven eighths 0.53).
 // A warp decodes 128 steps of a block at a time, lane l steps 4l+1 .. 4l+4:
 // their 16-bit windows end at stream bits 16l+3 .. 16l+15, so they lie in the
 // 64 bits of words (l >> 1) - 1 and l >> 1 of the chunk (word -1 of a block is
@@ -271,7 +272,7 @@ __global__ void decode_vec_kernel(DecodeArgs a, int V)
 // stores.  Needs T % 8 == 0 and a 16-byte aligned output; other shapes take
 // decode_vec_kernel.
 constexpr int kVec2DecThreads = 1024;
-constexpr uint32_t kVec2DecSmemStates = 0xC000u;
+constexpr uint32_t kVec2DecSmemStates = 0xE000u;
 
 __global__ void __launch_bounds__(kVec2DecThreads) decode_vec2_kernel(DecodeArgs a)
 {

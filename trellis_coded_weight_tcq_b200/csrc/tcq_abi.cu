@@ -591,6 +591,48 @@ tcq_status tcq_decode_vec(const uint32_t* bits, const uint32_t* start_state, con
     return e == cudaSuccess ? TCQ_OK : TCQ_ERR_CUDA;
 }
 
+tcq_status tcq_gemv_vec(const uint32_t* bits, const uint32_t* start_state, const float* scale,
+                        const void* codebook, tcq_dtype cb_dtype, int L, int k, int V, int T,
+                        int64_t rows, int64_t cols, const float* x, float* y, tcq_stream_t stream)
+{
+    if (V == 1)
+        return tcq_gemv(bits, start_state, scale, codebook, cb_dtype, L, k, T, rows, cols, x, y,
+                        stream);
+    if (rows < 0 || cols < 0) return TCQ_ERR_INVALID_ARG;
+    if (cb_dtype == TCQ_MAD) return TCQ_ERR_UNSUPPORTED;  // the computed code is scalar
+    if (!valid_dtype(cb_dtype)) return TCQ_ERR_INVALID_ARG;
+    const tcq_status shape = check_vec_shape(L, k, V, T);
+    if (shape != TCQ_OK) return shape;
+    if (cols % T != 0) return TCQ_ERR_INVALID_ARG;
+    if (rows == 0) return TCQ_OK;
+    if (cols > ((int64_t)1 << 31)) return TCQ_ERR_INVALID_ARG;
+    if (!bits || !start_state || !codebook_ok(codebook, cb_dtype) || !x || !y)
+        return TCQ_ERR_INVALID_ARG;
+    if (!aligned(bits, 4) || !aligned(start_state, 4) || (scale && !aligned(scale, 4)) ||
+        !aligned(x, 16) || !aligned(y, 4))
+        return TCQ_ERR_INVALID_ARG;
+    if ((unsigned long long)rows * (unsigned long long)(cols / T) > (1ull << 40))
+        return TCQ_ERR_INVALID_ARG;
+    const int sms = current_sms();
+    if (sms <= 0) return TCQ_ERR_CUDA;
+    GemvArgs a;
+    a.bits = bits;
+    a.start_state = start_state;
+    a.scale = scale;
+    a.cb = codebook;
+    a.cb_f16 = cb_dtype == TCQ_F16 ? 1 : 0;
+    a.L = L;
+    a.K = k * V;
+    a.T = T;
+    a.W = tcq_words_per_block(k, T);
+    a.rows = rows;
+    a.cols = cols;
+    a.x = x;
+    a.y = y;
+    const cudaError_t e = launch_gemv_vec(a, V, sms, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TCQ_OK : TCQ_ERR_CUDA;
+}
+
 const char* tcq_status_string(tcq_status status)
 {
     switch (status) {

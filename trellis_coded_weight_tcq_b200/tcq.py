@@ -86,6 +86,8 @@ def load_library() -> ctypes.CDLL:
     lib.tcq_encode_path.restype = ctypes.c_char_p
     lib.tcq_gemv.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, i64, i64, vp, vp, vp]
     lib.tcq_gemv.restype = ci
+    lib.tcq_gemv_vec.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, i64, i64, vp, vp, vp]
+    lib.tcq_gemv_vec.restype = ci
     lib.tcq_ldlq_workspace_bytes.argtypes = [ci, ci, ci, i64, i64, ci]
     lib.tcq_ldlq_workspace_bytes.restype = sz
     lib.tcq_ldlq.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, i64, i64, vp, vp, vp, vp, vp, vp,
@@ -154,6 +156,12 @@ def tcq_decode(bits, start_state, codebook, cb_dtype, L, k, T, n_blocks, y, stre
 def tcq_gemv(bits, start_state, scale, codebook, cb_dtype, L, k, T, rows, cols, x, y, stream) -> int:
     return int(load_library().tcq_gemv(bits, start_state, scale, codebook, cb_dtype, L, k, T, rows,
                                         cols, x, y, stream))
+
+
+def tcq_gemv_vec(bits, start_state, scale, codebook, cb_dtype, L, k, V, T, rows, cols, x, y,
+                 stream) -> int:
+    return int(load_library().tcq_gemv_vec(bits, start_state, scale, codebook, cb_dtype, L, k, V, T,
+                                            rows, cols, x, y, stream))
 
 
 def tcq_ldlq_workspace_bytes(L: int, k: int, T: int, rows: int, cols: int, cb_dtype: int) -> int:
@@ -304,6 +312,25 @@ def gemv(bits, start_state, scale, codebook, L: int, k: int, T: int, rows: int, 
     _check(tcq_gemv(_ptr(bits), _ptr(start_state), _ptr(scale), _ptr(codebook),
                     cb_dtype_of(codebook), L, k, T, rows, cols, _ptr(x), _ptr(out),
                     _stream_handle(stream)), "tcq_gemv")
+    return out
+
+
+def gemv_vec(bits, start_state, scale, codebook, L: int, k: int, V: int, T: int, rows: int,
+             cols: int, x, out=None, stream=None):
+    """gemv for the vector trellis (V weights per step, codebook [2^L, V])."""
+    torch = _torch()
+    nb = rows * (cols // T) if T > 0 else 0
+    W = tcq_words_per_block(k, T)
+    if bits.numel() < nb * max(W, 0) or start_state.numel() < nb or x.numel() < cols or (
+            scale is not None and scale.numel() < nb):
+        raise ValueError(f"gemv_vec: tensors too small for a {rows} x {cols} matrix of T={T} blocks")
+    if out is None:
+        out = torch.empty(rows, dtype=torch.float32, device=x.device)
+    if out.numel() < rows:
+        raise ValueError("gemv_vec: out holds fewer than rows values")
+    _check(tcq_gemv_vec(_ptr(bits), _ptr(start_state), _ptr(scale), _ptr(codebook),
+                        cb_dtype_of(codebook), L, k, V, T, rows, cols, _ptr(x), _ptr(out),
+                        _stream_handle(stream)), "tcq_gemv_vec")
     return out
 
 
