@@ -132,11 +132,235 @@ __global__ void __launch_bounds__(kThreads) feedback_kernel(FeedbackArgs a)
     }
 }
 
+// ---------------------------------------------------------------------------
+// The same product on the fifth-generation tensor cores (tcgen05), for column
+// blocks of 256: one CTA computes a 128 x 256 tile of X, accumulating in tensor
+// memory (256 of its columns), with the operands split in two TF32 halves so
+// that the three products hi*hi + hi*lo + lo*hi keep the fp32 accuracy the
+// targets need (a plain TF32 product would leave a relative error near 1e-3;
+// the dropped lo*lo term and the truncation of the low halves leave about
+// 2^-20 of each term).
+//
+// Shared memory holds both halves of the error tile (128 x 32) and of the U
+// tile (256 x 32) per stage, two stages, in the tensor core's K-major layout
+// without swizzle: 8-row by 16-byte core matrices, the 8 along K adjacent
+// (leading byte offset 128) and the row groups 1024 bytes apart (stride byte
+// offset).  Each K step of 8 is one 128 x 256 x 8 MMA per product, issued by
+// one thread; tcgen05.commit on the stage's mbarrier tells the loaders when
+// the stage may be overwritten, so the next tile's loads overlap the MMAs.
+// Every wait is bounded: after kTcSpinLimit polls the CTA gives up, writes NaN
+// targets (which the encoder then reports as non-finite costs) and frees its
+// tensor memory.
+// ---------------------------------------------------------------------------
+constexpr int TC_M = 128, TC_N = 256, TC_K = 32;
+constexpr int kTcThreads = 256;
+constexpr long long kTcSpinLimit = 1ll << 26;
+
+struct __align__(1024) TcSmem {
+    float a[2][2][TC_M * TC_K];  // [stage][hi, lo]
+    float b[2][2][TC_N * TC_K];
+    unsigned long long mbar[2];
+    uint32_t tmem_base;
+    int failed;
+};
+
+// element offset of (row, k) in a K-major core-matrix tile of TC_K columns
+__device__ __forceinline__ int tc_off(int row, int k)
+{
+    return (row >> 3) * (8 * TC_K) + (k >> 2) * 32 + (row & 7) * 4 + (k & 3);
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+// shared-memory matrix descriptor: K-major, no swizzle, LBO 128 B, SBO 1024 B
+__device__ __forceinline__ unsigned long long tc_desc(uint32_t addr)
+{
+    return (unsigned long long)((addr >> 4) & 0x3fffu) | ((unsigned long long)(128 >> 4) << 16) |
+           ((unsigned long long)(1024 >> 4) << 32) | (1ull << 46);
+}
+
+// instruction descriptor: D fp32, A and B TF32, both K-major, N = 256, M = 128
+constexpr uint32_t kTcIdesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(TC_N >> 3) << 17) |
+                              ((uint32_t)(TC_M >> 4) << 24);
+
+__device__ __forceinline__ float tf32_hi(float v)
+{
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(v));
+    return __uint_as_float(r);
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
+{
+    for (long long i = 0; i < kTcSpinLimit; ++i) {
+        uint32_t done;
+        asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                     "selp.b32 %0, 1, 0, p;\n\t}"
+                     : "=r"(done) : "r"(bar), "r"(parity) : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1) feedback_tc_kernel(FeedbackArgs a)
+{
+    extern __shared__ __align__(1024) unsigned char tc_raw[];
+    TcSmem& S = *reinterpret_cast<TcSmem*>(tc_raw);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const long long m0 = (long long)blockIdx.x * TC_M;
+    const long long K = a.c0;
+    const int iters = (int)(K / TC_K);
+
+    if (tid == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&S.mbar[0])) : "memory");
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&S.mbar[1])) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        S.failed = 0;
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(&S.tmem_base)), "r"(TC_N) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = S.tmem_base;
+
+    for (int it = 0; it < iters; ++it) {
+        const int st = it & 1;
+        const long long k0 = (long long)it * TC_K;
+        // the MMAs that last read this stage (iteration it - 2) must be done
+        if (it >= 2 && !mbar_wait(smem_u32(&S.mbar[st]), (uint32_t)(((it >> 1) - 1) & 1))) S.failed = 1;
+        // error tile: lanes take 8 rows x 4 column quads (conflict-free 16-byte stores)
+#pragma unroll
+        for (int i = 0; i < (TC_M * TC_K / 4) / kTcThreads; ++i) {
+            const int idx = tid + i * kTcThreads;
+            const int r = (idx & 7) | ((idx >> 6) << 3), kq = (idx >> 3) & 7;
+            float4 e = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (m0 + r < a.rows) {
+                const long long o = (m0 + r) * a.cols + k0 + 4 * kq;
+                const float4 w = __ldg(reinterpret_cast<const float4*>(a.w + o));
+                const float4 q = __ldg(reinterpret_cast<const float4*>(a.q + o));
+                e = make_float4(w.x - q.x, w.y - q.y, w.z - q.z, w.w - q.w);
+            }
+            const float4 h = make_float4(tf32_hi(e.x), tf32_hi(e.y), tf32_hi(e.z), tf32_hi(e.w));
+            const int off = tc_off(r, 4 * kq);
+            *reinterpret_cast<float4*>(&S.a[st][0][off]) = h;
+            *reinterpret_cast<float4*>(&S.a[st][1][off]) = make_float4(e.x - h.x, e.y - h.y, e.z - h.z, e.w - h.w);
+        }
+        // U tile: lanes take 8 consecutive columns x 4 consecutive k (conflict-free stores)
+#pragma unroll 8
+        for (int i = 0; i < (TC_N * TC_K) / kTcThreads; ++i) {
+            const int e = tid + i * kTcThreads;
+            const int n = (e & 7) | (((e >> 5) & 31) << 3), kk = ((e >> 3) & 3) | ((e >> 10) << 2);
+            const float v = __ldg(a.u + (k0 + kk) * a.cols + a.c0 + n);
+            const float h = tf32_hi(v);
+            const int off = tc_off(n, kk);
+            S.b[st][0][off] = h;
+            S.b[st][1][off] = v - h;
+        }
+        // make the generic-proxy stores visible to the tensor core, then one thread issues
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+        __syncthreads();
+        if (tid == 0) {
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const uint32_t ah = smem_u32(S.a[st][0]), al = smem_u32(S.a[st][1]);
+            const uint32_t bh = smem_u32(S.b[st][0]), bl = smem_u32(S.b[st][1]);
+#pragma unroll
+            for (int ks = 0; ks < TC_K / 8; ++ks) {
+                const uint32_t step = (uint32_t)ks * 256u;  // two core matrices of 128 B
+                const unsigned long long da_h = tc_desc(ah + step), da_l = tc_desc(al + step);
+                const unsigned long long db_h = tc_desc(bh + step), db_l = tc_desc(bl + step);
+                const uint32_t acc0 = (it > 0 || ks > 0) ? 1u : 0u;
+                asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                             "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}"
+                             ::"r"(tmem), "l"(da_h), "l"(db_h), "r"(kTcIdesc), "r"(acc0) : "memory");
+                asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                             "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}"
+                             ::"r"(tmem), "l"(da_h), "l"(db_l), "r"(kTcIdesc), "r"(1u) : "memory");
+                asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                             "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}"
+                             ::"r"(tmem), "l"(da_l), "l"(db_h), "r"(kTcIdesc), "r"(1u) : "memory");
+            }
+            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                         ::"r"(smem_u32(&S.mbar[st])) : "memory");
+        }
+    }
+    // all MMAs done: the last commit covers every earlier one
+    if (iters > 0) {
+        const int last = iters - 1;
+        if (!mbar_wait(smem_u32(&S.mbar[last & 1]), (uint32_t)((last >> 1) & 1))) S.failed = 1;
+    }
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    __syncthreads();
+    const bool failed = S.failed != 0;
+
+    // epilogue: warp w reads TMEM lanes 32 (w & 3) .. + 31 (its rows), columns
+    // 128 (w >> 2) .. + 127, and writes X = W + feedback
+    const int row = 32 * (warp & 3) + lane;
+    const long long r = m0 + row;
+#pragma unroll 1
+    for (int j = 0; j < 4; ++j) {
+        const int c = 128 * (warp >> 2) + 32 * j;
+        uint32_t v[32];
+        const uint32_t taddr = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)c;
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+                     "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+                     "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+                     : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+                       "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
+                       "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]),
+                       "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+                       "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]),
+                       "=r"(v[30]), "=r"(v[31])
+                     : "r"(taddr));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        if (r < a.rows) {
+            const float* wr = a.w + r * a.cols + a.c0 + c;
+            float* xr = a.x + r * a.x_ld + c;
+#pragma unroll
+            for (int q = 0; q < 32; q += 4) {
+                const float4 w4 = __ldg(reinterpret_cast<const float4*>(wr + q));
+                float4 o;
+                o.x = failed ? __int_as_float(0x7fc00000) : w4.x + __uint_as_float(v[q + 0]);
+                o.y = failed ? __int_as_float(0x7fc00000) : w4.y + __uint_as_float(v[q + 1]);
+                o.z = failed ? __int_as_float(0x7fc00000) : w4.z + __uint_as_float(v[q + 2]);
+                o.w = failed ? __int_as_float(0x7fc00000) : w4.w + __uint_as_float(v[q + 3]);
+                *reinterpret_cast<float4*>(xr + q) = o;
+            }
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 0) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TC_N) : "memory");
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_feedback(const FeedbackArgs& a, cudaStream_t stream)
 {
     if (a.rows <= 0 || a.n <= 0) return cudaSuccess;
+    // tensor cores: column blocks of 256 with at least one block fed back, and
+    // rows of 16-byte aligned columns (the operand tiles are read as float4)
+    if (a.n == TC_N && a.c0 > 0 && a.c0 % TC_K == 0 && a.cols % 4 == 0 && a.x_ld % 4 == 0 &&
+        (reinterpret_cast<uintptr_t>(a.w) & 15) == 0 && (reinterpret_cast<uintptr_t>(a.q) & 15) == 0 &&
+        (reinterpret_cast<uintptr_t>(a.x) & 15) == 0) {
+        const size_t smem = sizeof(TcSmem);
+        const cudaError_t e = cudaFuncSetAttribute(feedback_tc_kernel,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        const unsigned grid = (unsigned)((a.rows + TC_M - 1) / TC_M);
+        feedback_tc_kernel<<<grid, kTcThreads, smem, stream>>>(a);
+        return cudaGetLastError();
+    }
     const dim3 grid((unsigned)((a.n + BN - 1) / BN), (unsigned)((a.rows + BM - 1) / BM));
     feedback_kernel<<<grid, kThreads, 0, stream>>>(a);
     return cudaGetLastError();
