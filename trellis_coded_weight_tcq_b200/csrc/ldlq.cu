@@ -230,38 +230,58 @@ __global__ void __launch_bounds__(kTcThreads, 1) feedback_tc_kernel(FeedbackArgs
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = S.tmem_base;
 
+    // the next iteration's operands are loaded into registers while the
+    // current MMAs run (software pipelining), then split and stored
+    constexpr int AQ = (TC_M * TC_K / 4) / kTcThreads;  // error quads per thread
+    constexpr int BE = (TC_N * TC_K) / kTcThreads;      // U elements per thread
+    float4 rw[AQ], rq[AQ];
+    float ru[BE];
+    auto prefetch = [&](long long k0) {
+#pragma unroll
+        for (int i = 0; i < AQ; ++i) {
+            const int idx = tid + i * kTcThreads;
+            const int r = (idx & 7) | ((idx >> 6) << 3), kq = (idx >> 3) & 7;
+            rw[i] = rq[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (m0 + r < a.rows) {
+                const long long o = (m0 + r) * a.cols + k0 + 4 * kq;
+                rw[i] = __ldg(reinterpret_cast<const float4*>(a.w + o));
+                rq[i] = __ldg(reinterpret_cast<const float4*>(a.q + o));
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < BE; ++i) {
+            const int e = tid + i * kTcThreads;
+            const int n = (e & 7) | (((e >> 5) & 31) << 3), kk = ((e >> 3) & 3) | ((e >> 10) << 2);
+            ru[i] = __ldg(a.u + (k0 + kk) * a.cols + a.c0 + n);
+        }
+    };
+    if (iters > 0) prefetch(0);
+
     for (int it = 0; it < iters; ++it) {
         const int st = it & 1;
-        const long long k0 = (long long)it * TC_K;
         // the MMAs that last read this stage (iteration it - 2) must be done
         if (it >= 2 && !mbar_wait(smem_u32(&S.mbar[st]), (uint32_t)(((it >> 1) - 1) & 1))) S.failed = 1;
         // error tile: lanes take 8 rows x 4 column quads (conflict-free 16-byte stores)
 #pragma unroll
-        for (int i = 0; i < (TC_M * TC_K / 4) / kTcThreads; ++i) {
+        for (int i = 0; i < AQ; ++i) {
             const int idx = tid + i * kTcThreads;
             const int r = (idx & 7) | ((idx >> 6) << 3), kq = (idx >> 3) & 7;
-            float4 e = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (m0 + r < a.rows) {
-                const long long o = (m0 + r) * a.cols + k0 + 4 * kq;
-                const float4 w = __ldg(reinterpret_cast<const float4*>(a.w + o));
-                const float4 q = __ldg(reinterpret_cast<const float4*>(a.q + o));
-                e = make_float4(w.x - q.x, w.y - q.y, w.z - q.z, w.w - q.w);
-            }
+            const float4 e = make_float4(rw[i].x - rq[i].x, rw[i].y - rq[i].y, rw[i].z - rq[i].z,
+                                         rw[i].w - rq[i].w);
             const float4 h = make_float4(tf32_hi(e.x), tf32_hi(e.y), tf32_hi(e.z), tf32_hi(e.w));
             const int off = tc_off(r, 4 * kq);
             *reinterpret_cast<float4*>(&S.a[st][0][off]) = h;
             *reinterpret_cast<float4*>(&S.a[st][1][off]) = make_float4(e.x - h.x, e.y - h.y, e.z - h.z, e.w - h.w);
         }
         // U tile: lanes take 8 consecutive columns x 4 consecutive k (conflict-free stores)
-#pragma unroll 8
-        for (int i = 0; i < (TC_N * TC_K) / kTcThreads; ++i) {
+#pragma unroll
+        for (int i = 0; i < BE; ++i) {
             const int e = tid + i * kTcThreads;
             const int n = (e & 7) | (((e >> 5) & 31) << 3), kk = ((e >> 3) & 3) | ((e >> 10) << 2);
-            const float v = __ldg(a.u + (k0 + kk) * a.cols + a.c0 + n);
-            const float h = tf32_hi(v);
+            const float h = tf32_hi(ru[i]);
             const int off = tc_off(n, kk);
             S.b[st][0][off] = h;
-            S.b[st][1][off] = v - h;
+            S.b[st][1][off] = ru[i] - h;
         }
         // make the generic-proxy stores visible to the tensor core, then one thread issues
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -290,6 +310,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) feedback_tc_kernel(FeedbackArgs
             asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                          ::"r"(smem_u32(&S.mbar[st])) : "memory");
         }
+        if (it + 1 < iters) prefetch((long long)(it + 1) * TC_K);
     }
     // all MMAs done: the last commit covers every earlier one
     if (iters > 0) {
