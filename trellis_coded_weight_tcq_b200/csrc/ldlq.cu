@@ -11,9 +11,10 @@
 // a rows x n x c0 product whose left operand, the error W - Q of the blocks
 // already coded, is formed while its tile is staged.  Summed over the column
 // blocks this is rows * cols^2 / 2 multiply-adds, a small fraction of the
-// Viterbi work of the same matrix, so it runs on the fp32 FMA pipe: the targets
-// decide the trellis path, and a TF32 tensor-core product would put a relative
-// error near 1e-3 into them.
+// Viterbi work of the same matrix.  The targets decide the trellis path, so
+// the product keeps fp32 accuracy: on the tensor cores (blocks of 256 columns)
+// as three TF32 products of split operands, else on the fp32 FMA pipe; a plain
+// TF32 product would put a relative error near 1e-3 into them.
 #include "common.cuh"
 
 namespace tcq {
