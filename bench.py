@@ -315,7 +315,8 @@ def run_ours(args, rank, world, local_rank):
     dec_ms = sum(a.elapsed_time(b) for a, b in dec_ev) / len(dec_ev)
     ms, acs_ms, dec_ms = max_over_ranks([ms, acs_ms, dec_ms], dev)
     cost_last = out.path_cost.cpu().numpy()
-    gpu_launches = 2 * args.steps  # one encoder kernel + one decoder kernel per step
+    # per step: the encoder, the L2 discard of its dead backpointers, the decoder
+    gpu_launches = 3 * args.steps
 
     # ---- decode-in-matvec on the encoded matrix (one row of the matrix per
     # block row: rows = blocks * T / cols)

@@ -186,6 +186,8 @@ cudaError_t launch_decode(const DecodeArgs& a, int num_sms, cudaStream_t stream)
 // vector trellis: a.K = k V bits per step, a.T weights per block (V | T)
 cudaError_t launch_decode_vec(const DecodeArgs& a, int V, int num_sms, cudaStream_t stream);
 cudaError_t launch_gemv_vec(const GemvArgs& a, int V, int num_sms, cudaStream_t stream);
+// Drops [base, base + bytes) from L2 without write-back (base 128-byte aligned).
+cudaError_t launch_discard_l2(void* base, size_t bytes, int num_sms, cudaStream_t stream);
 cudaError_t launch_gemv(const GemvArgs& a, int num_sms, cudaStream_t stream);
 
 }  // namespace tcq

@@ -126,7 +126,9 @@ tcq_status run_encode(EncodeArgs& a, tcq_dtype cb_dtype, void* workspace, size_t
     if (grid < 1) grid = 1;
     a.ws = static_cast<unsigned char*>(workspace);
     a.slot_bytes = slot;
-    const cudaError_t e = info->launch(a, (int)grid, stream);
+    cudaError_t e = info->launch(a, (int)grid, stream);
+    // the backpointers are dead once traced: drop them from L2 unwritten
+    if (e == cudaSuccess) e = launch_discard_l2(workspace, (size_t)grid * slot, sms, stream);
     return e == cudaSuccess ? TCQ_OK : TCQ_ERR_CUDA;
 }
 
