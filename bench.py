@@ -405,6 +405,28 @@ def run_ours(args, rank, world, local_rank):
                              "alu_frac": wl.nodes * ALGO_OPS_PER_NODE / (acs_ms / 1e3) / peaks_ops(),
                              "kernel": tcq.tcq_encode_path(L, k, tcq.cb_dtype_of(cb))})
 
+    # ---- the same encode from fixed start states (one per block, seeded), the
+    # separate fixed-start instantiation of the encoder
+    fixed = None
+    if rank == 0 and world == 1 and not args.no_fixed:
+        starts = torch.randint(0, 1 << (L - k), (n,), dtype=torch.int32, device=dev,
+                               generator=torch.Generator(device=dev).manual_seed(11))
+        tcq.encode(x, d, cb, L, k, ws, out, fixed_start=starts)
+        f_ev = []
+        for _ in range(2):
+            a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            tcq.encode(x, d, cb, L, k, ws, out, fixed_start=starts)
+            b2.record(stream)
+            f_ev.append((a, b2))
+        torch.cuda.synchronize()
+        f_ms = sum(a.elapsed_time(b2) for a, b2 in f_ev) / len(f_ev)
+        assert bool(torch.equal(out.start_state, starts))
+        fixed = {"workload": wl.name + "_fixed_start", "ms": f_ms, "nodes_per_s": wl.nodes / (f_ms / 1e3),
+                 "alu_frac": wl.nodes * ALGO_OPS_PER_NODE / (f_ms / 1e3) / peaks_ops(),
+                 "cost_per_weight": float(out.path_cost.double().sum()) / wl.weights}
+        del starts
+
     # ---- error-feedback (LDLQ) encode of the MLP matrix: 16 column blocks, each
     # a feedback product, an encode of 14336 blocks and a decode
     ldlq = None
@@ -606,7 +628,7 @@ def run_ours(args, rank, world, local_rank):
         "weights_per_s": world * wl.weights / (ms / 1e3),
         "encode_ms_per_step": acs_ms, "decode_ms_per_step": dec_ms,
         "roofline": roofline, "decode_roofline": decode_roofline, "cpu_baseline": cpu_baseline, "e2e": e2e,
-        "per_workload": per_workload, "gemv": gemv, "ldlq": ldlq, "bcjr": bcjr, "vec": vec,
+        "per_workload": per_workload, "gemv": gemv, "ldlq": ldlq, "bcjr": bcjr, "vec": vec, "fixed_start": fixed,
         "clocks": clock_record, "remeasured": remeasured, "gpu_launches": gpu_launches,
     }
     print(json.dumps(line), flush=True)
@@ -625,6 +647,8 @@ def main():
                     help="skip the short encode/decode timing of the other named workloads")
     ap.add_argument("--no-bcjr", action="store_true",
                     help="skip the soft forward-backward quantization of the workload")
+    ap.add_argument("--no-fixed", action="store_true",
+                    help="skip the fixed-start encode of the workload")
     ap.add_argument("--no-vec", action="store_true",
                     help="skip the vector-trellis (V = 2) encode of the workload")
     ap.add_argument("--no-ldlq", action="store_true",
