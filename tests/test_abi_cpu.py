@@ -140,3 +140,36 @@ def test_binding_rejects_undersized_tensors_before_any_launch():
         tcq.decode(bits[:5], start, cb, 16, 2, 256)
     with pytest.raises(ValueError):
         tcq.decode(bits, start, cb, 16, 2, 256, out=torch.empty((9, 256)))
+
+
+def test_vector_and_feedback_entry_points_reject_on_the_host(lib):
+    """The vector-trellis calls validate shapes, dtypes and pointers before any
+    CUDA call; their workspace query covers the compile-time kernel."""
+    fake = ctypes.c_void_p(0x10000)
+    F16, F32 = tcq.TCQ_F16, tcq.TCQ_F32
+    # the L=16, k=2, V=2 compile-time encoder: two round buffers of (T/2 - 1)
+    # steps x 512 words, plus the traced path; never less than the runtime kernel needs
+    one = tcq.tcq_encode_vec_workspace_bytes(16, 2, 2, 256, 1, F16)
+    vec2 = 2 * ((127 * 512 * 4 + 255) // 256 * 256) + 256
+    generic = tcq.tcq_encode_vec_workspace_bytes(16, 2, 2, 256, 1, F32)
+    assert one >= vec2 and one >= generic
+    assert tcq.tcq_encode_vec_workspace_bytes(16, 2, 2, 255, 1, F16) == 0  # V does not divide T
+    assert tcq.tcq_encode_vec_workspace_bytes(16, 2, 2, 256, 1, tcq.TCQ_MAD) == 0
+    gv = lambda **o: tcq.tcq_gemv_vec(o.get("bits", fake), o.get("st", fake), None,  # noqa: E731
+                                      o.get("cb", fake), o.get("dt", F16), o.get("L", 16),
+                                      o.get("k", 2), o.get("V", 2), o.get("T", 256),
+                                      o.get("rows", 4), o.get("cols", 1024), o.get("x", fake),
+                                      o.get("y", fake), None)
+    assert gv(rows=0) == tcq.TCQ_OK
+    assert gv(rows=-1) == tcq.TCQ_ERR_INVALID_ARG
+    assert gv(cols=1000) == tcq.TCQ_ERR_INVALID_ARG                  # cols % T
+    assert gv(x=ctypes.c_void_p(0x10004)) == tcq.TCQ_ERR_INVALID_ARG  # x not 16-byte aligned
+    assert gv(y=None) == tcq.TCQ_ERR_INVALID_ARG
+    assert gv(dt=tcq.TCQ_MAD, cb=None) == tcq.TCQ_ERR_UNSUPPORTED
+    assert gv(k=3, V=3) == tcq.TCQ_ERR_UNSUPPORTED                   # kV = 9 bits per step
+    dv = lambda **o: tcq.tcq_decode_vec(o.get("bits", fake), o.get("st", fake), o.get("cb", fake),  # noqa: E731
+                                        o.get("dt", F16), 16, 2, o.get("V", 2), o.get("T", 256),
+                                        o.get("n", 4), o.get("y", fake), None)
+    assert dv(n=0) == tcq.TCQ_OK
+    assert dv(T=255) == tcq.TCQ_ERR_UNSUPPORTED
+    assert dv(y=ctypes.c_void_p(0x10002)) == tcq.TCQ_ERR_INVALID_ARG
