@@ -556,7 +556,9 @@ tcq_status tcq_encode_vec(const float* x, const float* d, const void* codebook, 
     a.V = V;
     a.ws = static_cast<unsigned char*>(workspace);
     a.slot_bytes = slot;
-    const cudaError_t e = info->launch(a, (int)grid, reinterpret_cast<cudaStream_t>(stream));
+    cudaError_t e = info->launch(a, (int)grid, reinterpret_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess)  // dead backpointers: drop them from L2 unwritten
+        e = launch_discard_l2(workspace, (size_t)grid * slot, sms, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TCQ_OK : TCQ_ERR_CUDA;
 }
 
