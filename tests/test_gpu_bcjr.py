@@ -183,3 +183,27 @@ def test_bcjr_long_block_takes_the_runtime_kernel(cuda_device):
     y_tol, F_tol = _tolerances(T, cb.astype(np.float64), F_o, tau)
     assert np.abs(y_g - y_o).max() <= y_tol
     assert np.all(np.abs(F_g.astype(np.float64) - F_o) <= F_tol)
+
+
+def test_bcjr_maximum_block_length(cuda_device):
+    """T = TCQ_MAX_T (2^20 weights in one block) through the runtime kernel: the
+    per-step shifts and their fp64 sums keep a million steps finite and within
+    the per-weight bound."""
+    from oracle import oracle_bcjr
+    from trellis_coded_weight_tcq_b200 import tcq
+
+    L, k, T, n, tau = 4, 2, tcq.TCQ_MAX_T, 1, 0.5
+    rng = np.random.default_rng(9200)
+    x = rng.standard_normal((n, T)).astype(np.float32)
+    d = rng.lognormal(0.0, 1.0, (n, T)).astype(np.float32)
+    cb = rng.standard_normal(1 << L).astype(np.float32)
+    y_g, F_g = _run(x, d, cb, L, k, tau, cuda_device)
+    y_o, F_o = oracle_bcjr(x, d, cb, L, k, tau)
+    assert np.all(np.isfinite(y_g)) and np.all(np.isfinite(F_g))
+    # per weight: each step's posterior is renormalised to mass 1, so a soft
+    # codeword carries the rounding of the forward and backward values near its
+    # step rather than of all T steps: the 1024-step bound is used; the free
+    # energy sums T fp64-accumulated shifts and stays within 1e-5 relative
+    y_tol, _ = _tolerances(1024, cb.astype(np.float64), F_o, tau)
+    assert np.abs(y_g - y_o).max() <= y_tol
+    np.testing.assert_allclose(F_g.astype(np.float64), F_o, rtol=1e-5)
