@@ -83,7 +83,8 @@ struct BG {
     static constexpr size_t smem_bytes()
     {
         return sizeof(float) * 3 * NU + sizeof(float2) * kMaxT + sizeof(double) * kMaxT +
-               sizeof(float) * 2 * NW + sizeof(float2) * 2 * NW + sizeof(float) * NW;
+               sizeof(float) * 2 * NW + sizeof(float2) * 2 * NW + sizeof(float) * NW +
+               sizeof(float) * kMaxT;
     }
 };
 
@@ -100,6 +101,7 @@ __global__ void __launch_bounds__(C::NT, 1) bcjr_grouped_kernel(BcjrArgs a)
     float* wmax = reinterpret_cast<float*>(Kc + kMaxT);          // [2][NW]
     float2* red = reinterpret_cast<float2*>(wmax + 2 * NW);      // [2][NW] (moment, mass)
     float* zred = reinterpret_cast<float*>(red + 2 * NW);        // [NW]
+    float* rwv = zred + NW;                                      // [kMaxT] 1 / w_t
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int T = a.T;
@@ -117,19 +119,28 @@ __global__ void __launch_bounds__(C::NT, 1) bcjr_grouped_kernel(BcjrArgs a)
     for (long long b = blockIdx.x; b < a.n_blocks; b += gridDim.x) {
         const float* xb = a.x + b * T;
         const float* db = a.d ? a.d + b * T : nullptr;
-        for (int t = tid; t < T; t += NT) xw[t] = make_float2(xb[t], (db ? db[t] : 1.f) * a.w_scale);
+        for (int t = tid; t < T; t += NT) {
+            // w_t floored at 2^-100 (a zero weight): 1 / w_t stays finite and the
+            // scaled values below stay inside fp32; the change to any exponent is
+            // below 2^-100 e^2
+            const float w = fmaxf((db ? db[t] : 1.f) * a.w_scale, 0x1p-100f);
+            xw[t] = make_float2(xb[t], w);
+            rwv[t] = 1.f / w;
+        }
         __syncthreads();
 
         // ---- forward
         double Kcum = 0.0;
         for (int t = 1; t <= T; ++t) {
             const float2 st = xw[t - 1];
+            const float rw = rwv[t - 1];
             float cp = 0.f;
             if (t >= 2) {
                 cp = wmax[((t - 1) & 1) * NW];
 #pragma unroll
                 for (int i = 1; i < NW; ++i) cp = fmaxf(cp, wmax[((t - 1) & 1) * NW + i]);
             }
+            const float pc = -cp * rw;
             if (tid == 0) Kc[t - 1] = Kcum;
             Kcum += (double)cp;
             const float* Sp = buf + ((t - 1) & 1) * NU;
@@ -141,7 +152,7 @@ __global__ void __launch_bounds__(C::NT, 1) bcjr_grouped_kernel(BcjrArgs a)
                 const int g = tid + i * NT;
                 float p[H];
 #pragma unroll
-                for (int h = 0; h < H; ++h) p[h] = t >= 2 ? Sp[(h << SH) | g] - cp : 0.f;
+                for (int h = 0; h < H; ++h) p[h] = t >= 2 ? fmaf(Sp[(h << SH) | g], rw, pc) : 0.f;
                 float out[H];
 #pragma unroll
                 for (int j = 0; j < H; ++j) {
@@ -149,7 +160,7 @@ __global__ void __launch_bounds__(C::NT, 1) bcjr_grouped_kernel(BcjrArgs a)
 #pragma unroll
                     for (int h = 0; h < H; ++h) {
                         const float e = diff(i, h, j, st.x);
-                        c[h] = fmaf(-st.y * e, e, p[h]);
+                        c[h] = fmaf(-e, e, p[h]);  // (value - w e^2) / w
                     }
                     float m, s;
                     if constexpr (H == 4) {
@@ -157,13 +168,14 @@ __global__ void __launch_bounds__(C::NT, 1) bcjr_grouped_kernel(BcjrArgs a)
                         // min/max network, so three exponentials instead of four
                         const float lo01 = fminf(c[0], c[1]), hi01 = fmaxf(c[0], c[1]);
                         const float lo23 = fminf(c[2], c[3]), hi23 = fmaxf(c[2], c[3]);
-                        m = fmaxf(hi01, hi23);
-                        s = 1.f + ex2g(lo01 - m) + ex2g(lo23 - m) + ex2g(fminf(hi01, hi23) - m);
+                        m = fmaxf(hi01, hi23) * st.y;
+                        s = 1.f + ex2g(fmaf(lo01, st.y, -m)) + ex2g(fmaf(lo23, st.y, -m)) +
+                            ex2g(fmaf(fminf(hi01, hi23), st.y, -m));
                     } else {
-                        m = hmax<H>(c);
+                        m = hmax<H>(c) * st.y;
                         s = 0.f;
 #pragma unroll
-                        for (int h = 0; h < H; ++h) s += ex2g(c[h] - m);
+                        for (int h = 0; h < H; ++h) s += ex2g(fmaf(c[h], st.y, -m));
                     }
                     out[j] = m + lg2g(s);
                     lmax = fmaxf(lmax, out[j]);
@@ -214,12 +226,14 @@ __global__ void __launch_bounds__(C::NT, 1) bcjr_grouped_kernel(BcjrArgs a)
         double G = 0.0;
         for (int t = T; t >= 1; --t) {
             const float2 st = xw[t - 1];
+            const float rw = rwv[t - 1];
             float ep = 0.f;
             if (t < T) {
                 ep = wmax[(t & 1) * NW];
 #pragma unroll
                 for (int i = 1; i < NW; ++i) ep = fmaxf(ep, wmax[(t & 1) * NW + i]);
             }
+            const float pe = -ep * rw;
             const float shift = (float)(Kc[t - 1] + G + (double)ep - log2z);
             const float* Ri = buf + (t & 1) * NU;
             float* Ro = buf + ((t - 1) & 1) * NU;
@@ -233,13 +247,13 @@ __global__ void __launch_bounds__(C::NT, 1) bcjr_grouped_kernel(BcjrArgs a)
                 if (t < T) {
                     if constexpr (H == 4) {
                         const float4 v = *reinterpret_cast<const float4*>(Ri + (g << K));
-                        r[0] = v.x - ep;
-                        r[1] = v.y - ep;
-                        r[2] = v.z - ep;
-                        r[3] = v.w - ep;
+                        r[0] = fmaf(v.x, rw, pe);
+                        r[1] = fmaf(v.y, rw, pe);
+                        r[2] = fmaf(v.z, rw, pe);
+                        r[3] = fmaf(v.w, rw, pe);
                     } else {
 #pragma unroll
-                        for (int j = 0; j < H; ++j) r[j] = Ri[(g << K) + j] - ep;
+                        for (int j = 0; j < H; ++j) r[j] = fmaf(Ri[(g << K) + j], rw, pe);
                     }
                 } else {
 #pragma unroll
@@ -251,13 +265,14 @@ __global__ void __launch_bounds__(C::NT, 1) bcjr_grouped_kernel(BcjrArgs a)
 #pragma unroll
                     for (int j = 0; j < H; ++j) {
                         e[j] = diff(i, h, j, st.x);
-                        c[j] = fmaf(-st.y * e[j], e[j], r[j]);
+                        c[j] = fmaf(-e[j], e[j], r[j]);  // (value - w e^2) / w
                     }
-                    const float m = hmax<H>(c);
+                    const float mq = hmax<H>(c);
+                    const float m = mq * st.y;
                     float s = 0.f, se = 0.f;
 #pragma unroll
                     for (int j = 0; j < H; ++j) {
-                        const float E = ex2g(c[j] - m);
+                        const float E = ex2g(fmaf(c[j], st.y, -m));
                         s += E;
                         se = fmaf(E, e[j], se);
                     }
