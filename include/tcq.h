@@ -121,7 +121,10 @@ size_t tcq_encode_workspace_bytes(int L, int k, int T, int64_t n_blocks, tcq_dty
  *   path_cost   out: fp32 [n_blocks], J of the returned path (accumulated in
  *               fp64 along the path, rounded once to fp32).
  *   workspace   device scratch of workspace_bytes, 256-byte aligned; its
- *               contents on entry do not matter and are garbage on return.
+ *               contents on entry do not matter and are garbage on return
+ *               (the call ends by discarding the used part from L2 without
+ *               write-back, so nothing else may use it until the call's
+ *               work on `stream` has finished).
  *
  * Every returned path is optimal up to fp32 rounding of the search: J of the
  * returned path exceeds the exact minimum by at most a few fp32 rounding
