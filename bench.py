@@ -154,8 +154,13 @@ def peaks_ops() -> float:
     return SMS * LANES_PER_SM * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
 
 
-def time_workload(name, dev, tcq, workloads, peak_ops, steps=3):
-    """Encode and decode timing of one named workload (1 warm-up, best of `steps`)."""
+def _median_ms(pairs):
+    return statistics.median(a.elapsed_time(b) for a, b in pairs)
+
+
+def time_workload(name, dev, tcq, workloads, peak_ops, warmup=3, steps=10):
+    """Encode and decode timing of one named workload: `warmup` untimed
+    encode + decode passes, then the median of `steps` event-timed passes."""
     import torch
 
     wl = workloads.NAMED[name](0)
@@ -165,6 +170,9 @@ def time_workload(name, dev, tcq, workloads, peak_ops, steps=3):
     ws = tcq.Workspace(wl.L, wl.k, wl.T, wl.n_blocks, tcq.cb_dtype_of(cb), dev)
     out = tcq.encode(x, d, cb, wl.L, wl.k, ws)
     y = tcq.decode(out.bits, out.start_state, cb, wl.L, wl.k, wl.T)
+    for _ in range(warmup):
+        tcq.encode(x, d, cb, wl.L, wl.k, ws, out)
+        tcq.decode(out.bits, out.start_state, cb, wl.L, wl.k, wl.T, y)
     enc, dec = [], []
     for _ in range(steps):
         a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
@@ -176,10 +184,11 @@ def time_workload(name, dev, tcq, workloads, peak_ops, steps=3):
         enc.append((a, b))
         dec.append((b, c))
     torch.cuda.synchronize()
-    e_ms = min(a.elapsed_time(b) for a, b in enc)
-    d_ms = min(a.elapsed_time(b) for a, b in dec)
+    e_ms = _median_ms(enc)
+    d_ms = _median_ms(dec)
     return {"workload": wl.name, "nodes_per_s": wl.nodes / (e_ms / 1e3),
             "weights_per_s": wl.weights / (e_ms / 1e3), "encode_ms": e_ms, "decode_ms": d_ms,
+            "timing": f"median of {steps} after {warmup} warm-ups",
             "alu_frac": wl.nodes * ALGO_OPS_PER_NODE / (e_ms / 1e3) / peak_ops,
             "kernel": tcq.tcq_encode_path(wl.L, wl.k, tcq.cb_dtype_of(cb))}
 
@@ -339,7 +348,7 @@ def run_ours(args, rank, world, local_rank):
             b.record(stream)
             g_ev.append((a, b))
         torch.cuda.synchronize()
-        g_ms = min(a.elapsed_time(b) for a, b in g_ev)
+        g_ms = _median_ms(g_ev)
         g_bytes = n * W * 4 + n * 4 + n * 4 + cols_m * 4 + rows_m * 4
         peaks_g, _ = _peaks()
         gemv = {"rows": rows_m, "cols": cols_m, "ms": g_ms,
@@ -359,7 +368,7 @@ def run_ours(args, rank, world, local_rank):
             b.record(stream)
             m_ev.append((a, b))
         torch.cuda.synchronize()
-        m_ms = min(a.elapsed_time(b) for a, b in m_ev)
+        m_ms = _median_ms(m_ev)
         # issue-bound: about 6 instructions per weight at best (state, multiply,
         # byte sum, float, FMA) against 148 SMs x 128 lanes x the max clock
         issue_peak = SMS * LANES_PER_SM * float(peaks_g.get("sm_max_mhz", 1965.0)) * 1e6
@@ -540,7 +549,7 @@ def run_ours(args, rank, world, local_rank):
         vd_bytes = n * T * 4 + n * tcq.tcq_words_per_block(k, T) * 4 + n * 4
         del yv
         # decode-in-matvec over the matrix those blocks tile (rows x cols), timed
-        # like the scalar product above (unit block scales, best of 10)
+        # like the scalar product above (unit block scales, median of 10)
         vgemv = None
         vmat = wl.meta.get("matrix")
         if vmat and (n * T) % int(vmat[1]) == 0:
@@ -559,7 +568,7 @@ def run_ours(args, rank, world, local_rank):
                 b2.record(stream)
                 vg_ev.append((a, b2))
             torch.cuda.synchronize()
-            vg_ms = min(a.elapsed_time(b2) for a, b2 in vg_ev)
+            vg_ms = _median_ms(vg_ev)
             vg_bytes = n * tcq.tcq_words_per_block(k, T) * 4 + n * 8 + g_cols * 4 + g_rows * 4
             assert bool(torch.isfinite(yg).all())
             vgemv = {"rows": g_rows, "cols": g_cols, "ms": vg_ms,

@@ -344,15 +344,22 @@ const char* tcq_encode_path(int L, int k, tcq_dtype cb_dtype);
  * TCQ_STATIC_SCRATCH_BYTES that every GPU loading this library holds until the
  * process exits.
  *
- *   - The first call on a device looks up that array's device address (with the
- *     device current) and caches it; make that first call before any stream
- *     capture.  Calls are thread-safe on the host.
+ *   - Every call made outside stream capture looks up that array's device
+ *     address on the current device (a host query, no allocation) and caches
+ *     it; a call made while `stream` is capturing uses the cached address, so
+ *     make at least one call on the device before any stream capture.  After a
+ *     cudaDeviceReset in the caller's process the array may move: the next call
+ *     outside capture picks up the new address, but a CUDA graph captured
+ *     before the reset holds the old one and must not be replayed.  Calls are
+ *     thread-safe on the host.
  *   - The scratch limits concurrency, not problem size: blocks are processed by
  *     as many persistent CTAs as the scratch holds (at L=16, k=2, T=256 each CTA
  *     needs about 2 MiB, so about 15 CTAs run and the call is roughly 10x slower
- *     than tcq_encode with a full workspace).  A shape whose single-CTA share
- *     exceeds TCQ_STATIC_SCRATCH_BYTES (very long blocks) returns
- *     TCQ_ERR_WORKSPACE.
+ *     than tcq_encode with a full workspace).  A shape whose single-CTA share,
+ *     tcq_encode_workspace_bytes(L, k, T, 1, cb_dtype), exceeds
+ *     TCQ_STATIC_SCRATCH_BYTES returns TCQ_ERR_WORKSPACE: at L = 16 with k = 2
+ *     or 3 the longest block is T = 4096 for a binary16 table and T = 4080 for
+ *     TCQ_MAD (whose table takes 128 KiB of the array).
  *   - Every call uses the same array.  Nothing in it needs to start at zero, and
  *     a call never depends on what an earlier call left there; but calls that
  *     overlap on the GPU (two streams, or two host threads on different

@@ -202,3 +202,35 @@ def test_ldlq_mlp_sampled(cuda_device):
     rows = np.array([0, 1, 4097, 9000, 14335])
     _check_targets(wl, out, rows)
     _check_blocks(wl, out, rows[[0, 2, 4]])
+
+
+# L, k, T, rows, cols, codebook dtype, weighted
+DYADIC = [
+    (8, 2, 64, 40, 256, "f32", True),     # fp32-pipe feedback product, grouped L=8 encoder
+    (12, 2, 256, 130, 768, "f32", False),  # tensor-core feedback (two 128-row tiles), L=12 encoder
+    (16, 2, 256, 6, 768, "f16", False),    # tensor-core feedback, register-resident L=16 encoder
+]
+
+
+@pytest.mark.parametrize("case", DYADIC, ids=lambda c: "L{}k{}T{}_{}x{}_{}{}".format(
+    c[0], c[1], c[2], c[3], c[4], c[5], "_w" if c[6] else ""))
+def test_ldlq_whole_matrix_bit_exact_on_dyadic_inputs(case, cuda_device):
+    """With every fp32 operation exact (the workload's docstring says why), the
+    GPU takes exactly the oracle's decisions in every block, its tie rules
+    included: the whole reconstruction Q, the targets, the bits, the start
+    states and the costs equal the fp64 driver's."""
+    from oracle import oracle_ldlq
+    from trellis_coded_weight_tcq_b200.workloads import ldlq_dyadic_exact
+
+    L, k, T, rows, cols, cbt, weighted = case
+    wl = ldlq_dyadic_exact(L, k, T, rows, cols, weighted, cbt, seed=5000 + L + T + rows)
+    out = _run(wl, cuda_device)
+    d_o = np.ones(cols) if wl.d is None else wl.d
+    q_o, x_o, s_o, b_o, c_o = oracle_ldlq(wl.w, wl.u, d_o, wl.codebook, L, k, T)
+    np.testing.assert_array_equal(out["x"].astype(np.float64), x_o)
+    np.testing.assert_array_equal(out["q"].astype(np.float64), q_o)
+    np.testing.assert_array_equal(out["start"], s_o)
+    np.testing.assert_array_equal(out["bits"], b_o)
+    np.testing.assert_array_equal(out["cost"].astype(np.float64), c_o)
+    # the feedback did something: some targets differ from w
+    assert not np.array_equal(out["x"], wl.w)

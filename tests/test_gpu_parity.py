@@ -29,7 +29,7 @@ def _device(cuda_device):
 def test_named_workload_full(name):
     wl = workloads.NAMED[name]()
     start, bits, cost = gpu_encode(wl)
-    check_encode(wl, start, bits, cost)
+    check_encode(wl, start, bits, cost, pure=True)
     # decode of the GPU's own bits: bit-exact against the oracle's decode
     from oracle import oracle_decode
 
@@ -55,7 +55,7 @@ def test_named_workload_full_size_sampled(name):
     assert tcq.tcq_encode_path(wl.L, wl.k, dt).startswith("grouped")
     start, bits, cost = gpu_encode(wl)
     rows = _sample_rows(wl.n_blocks, 256, 7)  # first, last and 254 seeded
-    check_encode(wl, start, bits, cost, rows=rows)
+    check_encode(wl, start, bits, cost, rows=rows, pure=True)
     y = gpu_decode(bits, start, wl.codebook, wl.L, wl.k, wl.T)
     y_o = oracle_decode(bits[rows], start[rows], wl.codebook, wl.L, wl.k, wl.T).astype(np.float32)
     np.testing.assert_array_equal(y[rows], y_o)

@@ -26,16 +26,25 @@ void* g_scratch_addr[kMaxDevices] = {};
 
 // Device address of g_tcq_scratch on the current device.  In host code the
 // array's name only stands in for the symbol; the address a kernel may use is
-// looked up once per device, with that device current.
-tcq_status scratch_address(void** out)
+// looked up with that device current.  Outside stream capture it is looked up
+// on every call (a host-side query that allocates nothing), so a module reload
+// after cudaDeviceReset in the caller's process is picked up; during capture
+// the address cached by the last call outside capture is used, because a
+// lookup may have to load the module, which capture forbids.
+tcq_status scratch_address(cudaStream_t stream, void** out)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
         cudaGetLastError();
         return TCQ_ERR_CUDA;
     }
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) {
+        cudaGetLastError();  // e.g. the legacy stream while another stream captures
+        cap = cudaStreamCaptureStatusActive;
+    }
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_scratch_addr[dev]) {
+    if (cap == cudaStreamCaptureStatusNone || !g_scratch_addr[dev]) {
         void* p = nullptr;
         const cudaError_t e = cudaGetSymbolAddress(&p, g_tcq_scratch);
         if (e != cudaSuccess || !p) {
@@ -64,7 +73,7 @@ extern "C" tcq_status tcq_encode_static_scratch(const float* x, const float* d,
     const size_t one_cta = tcq_encode_workspace_bytes(L, k, T, 1, cb_dtype);
     if (one_cta > (size_t)TCQ_STATIC_SCRATCH_BYTES) return TCQ_ERR_WORKSPACE;
     void* scratch = nullptr;
-    const tcq_status st = scratch_address(&scratch);
+    const tcq_status st = scratch_address(reinterpret_cast<cudaStream_t>(stream), &scratch);
     if (st != TCQ_OK) return st;
     // Nothing in the scratch has to start at zero: every byte the encoder reads
     // was written earlier in the same call, so the previous call's leftovers

@@ -218,3 +218,30 @@ def ldlq_mlp(shard: int = 0) -> LdlqWorkload:
     u = unit_upper_factor(4096, 256, 0.5, SEED_PERM + 1 + 7919 * shard)
     return LdlqWorkload("ldlq_mlp_14336x4096_L16_k2_T256_weighted", 16, 2, 256, W.astype(np.float32),
                         u, d, gaussian_sample_codebook_f16(1 << 16), {"matrix": [14336, 4096]})
+
+
+def ldlq_dyadic_exact(L: int, k: int, T: int, rows: int, cols: int, weighted: bool,
+                      cb_dtype: str, seed: int) -> LdlqWorkload:
+    """An error-feedback case on which every fp32 operation is exact.
+
+    w and the codewords are multiples of 1/8 in [-2, 2]; U is the identity plus,
+    in each column past the first block, one entry of +1 or -1 in a random row of
+    an earlier block (only those entries feed errors forward); d is in {1/4, 1, 4}
+    or absent.  Each target is then w plus one weight error, a multiple of 1/8
+    below 8 in magnitude, every product and partial sum of the feedback is an
+    exact small dyadic (also after a split into TF32 halves), and every branch
+    metric and path metric of a block of at most 64 weighted (or 256 unweighted)
+    steps fits the fp32 significand, so the whole matrix Q, the bits and the
+    targets have a single correct value.
+    """
+    assert cols % T == 0 and T <= (64 if weighted else 256)
+    rng = np.random.default_rng(seed)
+    w = (rng.integers(-16, 17, (rows, cols)) / 8.0).astype(np.float32)
+    u = np.eye(cols, dtype=np.float32)
+    for c in range(T, cols):
+        c0 = (c // T) * T
+        u[rng.integers(0, c0), c] = np.float32(rng.choice([-1.0, 1.0]))
+    d = (4.0 ** rng.integers(-1, 2, cols)).astype(np.float32) if weighted else None
+    cb = rng.integers(-16, 17, 1 << L) / 8.0
+    cb = cb.astype(np.float16) if cb_dtype == "f16" else cb.astype(np.float32)
+    return LdlqWorkload(f"ldlq_dyadic_L{L}_k{k}_T{T}_{rows}x{cols}", L, k, T, w, u, d, cb)
