@@ -17,5 +17,7 @@ from .tcq_oracle import (  # noqa: F401
     oracle_ldlq,
     oracle_mad_codebook,
     oracle_path_cost,
+    oracle_ub8_decode,
+    oracle_ub8_encode,
     oracle_words_per_block,
 )

@@ -605,3 +605,164 @@ int oracle_decode_vec(const uint32_t* bits, const uint32_t* start_state, const d
     }
     return ORACLE_OK;
 }
+
+/*
+ * Ungerboeck's 8-state set-partitioned trellis (the 2-bit post, Pingala-8
+ * section: an 8-state set-partitioned trellis over symbols of several weights
+ * at about 2 bits per weight, its labels Ungerboeck's; the post's section on
+ * trellis-coded quantization: the state decides which subset the next group
+ * may use, the written bits pick a value inside the subset and set the next
+ * state, so the format holds twice as many values as its bits address; its
+ * background reading: Marcellin and Fischer's trellis-coded quantization).
+ * The pages give no labels and no codebook; the reading taken here is
+ * Marcellin and Fischer's TCQ on Ungerboeck's 8-state code for one-dimensional
+ * signals, generalised to V weights per symbol:
+ *
+ *   Union codebook: 4 * 2^m rows of V values; row r belongs to subset
+ *   D_{r mod 4} and is entry r >> 2 of it (for V = 1 and rows sorted
+ *   ascending this is Ungerboeck's partition of an amplitude alphabet).
+ *
+ *   Trellis: the rate-1/2 systematic feedback code with parity-check
+ *   polynomials h0 = D^3 + D + 1 and h1 = D^2 (octal 13 and 04): a label
+ *   sequence (z1_t, z0_t) is a code sequence iff
+ *       z0_t ^ z0_{t-1} ^ z0_{t-3} ^ z1_{t-2} = 0.
+ *   Realised with three memory bits, state sigma = 4p + 2q + r: a branch from
+ *   sigma with branch bit z uses subset j = 2z + p (z0 = p, z1 = z) and leads to
+ *       sigma' = 4 (p ^ q) + 2 (r ^ z) + p.
+ *   Both branches leaving a state use the two subsets of one half {D_p, D_p+2};
+ *   the two branches entering a state come from states with the same p.
+ *
+ *   A step codes V weights with 1 + m bits: symbol b_t = (z_t << m) | i_t, the
+ *   branch bit and the entry i_t of subset j_t; y_t = row 4 i_t + j_t.
+ *   Symbols are packed like every other stream here (MSB first, 1 + m bits
+ *   per step); the stored start state is sigma_0 (3 bits).
+ *
+ * The search, in the textbook order: for every step and subset the nearest
+ * entry (the branch metric of every branch carrying that subset, smallest i on
+ * ties), then the Viterbi program over the 8 states:
+ *   M_0[s] = 0 (free start; a fixed start leaves only that state at 0),
+ *   M_t[s'] = min over the branches (s, z) into s' of M_{t-1}[s] + e_t[2z + p(s)]
+ *   (predecessors taken in increasing s, strict <), final state the smallest
+ *   s minimising M_S, and the traceback.
+ */
+static int ub8_p(int s) { return (s >> 2) & 1; }
+
+static int ub8_next(int s, int z)
+{
+    const int p = (s >> 2) & 1, q = (s >> 1) & 1, r = s & 1;
+    return 4 * (p ^ q) + 2 * (r ^ z) + p;
+}
+
+int oracle_ub8_encode(const double* x, const double* d, const double* cb, int V, int m, int T,
+                      int64_t n_blocks, int64_t fixed_start, uint32_t* start_state,
+                      uint32_t* bits, double* cost)
+{
+    if (V < 1 || m < 0 || m > 16 || T < 1 || T % V != 0 || n_blocks < 0) return ORACLE_EINVAL;
+    if (n_blocks == 0) return ORACLE_OK;
+    if (!x || !cb || !start_state || !bits || !cost) return ORACLE_EINVAL;
+    const int NS = T / V;
+    const int K = 1 + m;
+    const int64_t per_subset = (int64_t)1 << m;
+    const int W = oracle_words_per_block(K, NS);
+    double* e = (double*)malloc(sizeof(double) * 4 * (size_t)NS);
+    uint32_t* idx = (uint32_t*)malloc(sizeof(uint32_t) * 4 * (size_t)NS);
+    uint8_t* bp_state = (uint8_t*)malloc(8 * (size_t)NS);
+    uint8_t* bp_z = (uint8_t*)malloc(8 * (size_t)NS);
+    if (!e || !idx || !bp_state || !bp_z) {
+        free(e); free(idx); free(bp_state); free(bp_z);
+        return ORACLE_ENOMEM;
+    }
+    for (int64_t blk = 0; blk < n_blocks; ++blk) {
+        const double* xb = x + blk * T;
+        const double* db = d ? d + blk * T : NULL;
+        /* branch metrics: nearest entry of every subset at every step */
+        for (int t = 0; t < NS; ++t) {
+            for (int j = 0; j < 4; ++j) {
+                double best = INFINITY;
+                uint32_t best_i = 0;
+                for (int64_t i = 0; i < per_subset; ++i) {
+                    const double* row = cb + (4 * i + j) * V;
+                    double dist = 0.0;
+                    for (int v = 0; v < V; ++v) {
+                        const double diff = xb[t * V + v] - row[v];
+                        dist += weight_at(db, t * V + v) * diff * diff;
+                    }
+                    if (dist < best) {
+                        best = dist;
+                        best_i = (uint32_t)i;
+                    }
+                }
+                e[4 * t + j] = best;
+                idx[4 * t + j] = best_i;
+            }
+        }
+        /* Viterbi over the 8 states */
+        double M[8], Mn[8];
+        for (int s = 0; s < 8; ++s)
+            M[s] = (fixed_start < 0 || s == (int)(fixed_start & 7)) ? 0.0 : INFINITY;
+        for (int t = 0; t < NS; ++t) {
+            for (int s2 = 0; s2 < 8; ++s2) {
+                double best = INFINITY;
+                int bs = 0, bz = 0;
+                for (int s = 0; s < 8; ++s)
+                    for (int z = 0; z < 2; ++z) {
+                        if (ub8_next(s, z) != s2) continue;
+                        const double c = M[s] + e[4 * t + 2 * z + ub8_p(s)];
+                        if (c < best) {
+                            best = c;
+                            bs = s;
+                            bz = z;
+                        }
+                    }
+                Mn[s2] = best;
+                bp_state[8 * t + s2] = (uint8_t)bs;
+                bp_z[8 * t + s2] = (uint8_t)bz;
+            }
+            for (int s = 0; s < 8; ++s) M[s] = Mn[s];
+        }
+        int s_end = 0;
+        for (int s = 1; s < 8; ++s)
+            if (M[s] < M[s_end]) s_end = s;
+        cost[blk] = M[s_end];
+        /* traceback: the state before step t and the branch bit taken */
+        uint32_t* wb = bits + blk * W;
+        memset(wb, 0, sizeof(uint32_t) * (size_t)W);
+        int s = s_end;
+        for (int t = NS - 1; t >= 0; --t) {
+            const int prev = bp_state[8 * t + s];
+            const int z = bp_z[8 * t + s];
+            const uint32_t i = idx[4 * t + 2 * z + ub8_p(prev)];
+            put_symbol(wb, K, t + 1, ((uint32_t)z << m) | i);
+            s = prev;
+        }
+        start_state[blk] = (uint32_t)s;
+    }
+    free(e); free(idx); free(bp_state); free(bp_z);
+    return ORACLE_OK;
+}
+
+/* Decode of the 8-state set-partitioned trellis: from sigma_0 = start & 7,
+ * step t reads (z, i), emits row 4 i + 2 z + p(sigma_{t-1}), moves to
+ * sigma_t = next(sigma_{t-1}, z). */
+int oracle_ub8_decode(const uint32_t* bits, const uint32_t* start_state, const double* cb, int V,
+                      int m, int T, int64_t n_blocks, double* y)
+{
+    if (V < 1 || m < 0 || m > 16 || T < 1 || T % V != 0 || n_blocks < 0) return ORACLE_EINVAL;
+    if (n_blocks == 0) return ORACLE_OK;
+    if (!bits || !start_state || !cb || !y) return ORACLE_EINVAL;
+    const int NS = T / V;
+    const int K = 1 + m;
+    const int W = oracle_words_per_block(K, NS);
+    for (int64_t blk = 0; blk < n_blocks; ++blk) {
+        int s = (int)(start_state[blk] & 7u);
+        for (int t = 1; t <= NS; ++t) {
+            const uint32_t sym = get_symbol(bits + blk * W, K, t);
+            const int z = (int)(sym >> m);
+            const int64_t i = (int64_t)(sym & (((uint32_t)1 << m) - 1));
+            const double* row = cb + (4 * i + 2 * z + ub8_p(s)) * V;
+            for (int v = 0; v < V; ++v) y[blk * T + (t - 1) * V + v] = row[v];
+            s = ub8_next(s, z);
+        }
+    }
+    return ORACLE_OK;
+}

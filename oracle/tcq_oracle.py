@@ -62,6 +62,10 @@ def _load():
         lib.oracle_encode_vec.restype = ci
         lib.oracle_decode_vec.argtypes = [up, up, dp, ci, ci, ci, ci, i64, dp]
         lib.oracle_decode_vec.restype = ci
+        lib.oracle_ub8_encode.argtypes = [dp, dp, dp, ci, ci, ci, i64, i64, up, up, dp]
+        lib.oracle_ub8_encode.restype = ci
+        lib.oracle_ub8_decode.argtypes = [up, up, dp, ci, ci, ci, i64, dp]
+        lib.oracle_ub8_decode.restype = ci
         _lib = lib
     return _lib
 
@@ -306,4 +310,58 @@ def oracle_decode_vec(bits, start_state, codebook, L: int, k: int, V: int, T: in
                                    _ptr(y, ctypes.c_double))
     if rc != 0:
         raise ValueError(f"oracle_decode_vec failed with code {rc}")
+    return y
+
+
+def oracle_ub8_encode(x, d, codebook, V: int, m: int, fixed_start: int | None = None):
+    """TCQ over Ungerboeck's 8-state set-partitioned trellis (see tcq_oracle.c).
+
+    ``x`` is [n_blocks, T] with V | T (steps of V weights); ``codebook`` holds
+    4 * 2^m rows of V values, row r in subset r mod 4.  Returns
+    ``(start_state uint32[n] in [0, 8), bits uint32[n, W], cost float64[n])``
+    with W = ceil((T / V) (1 + m) / 32).
+    """
+    x = _f64(x)
+    if x.ndim == 1:
+        x = x[None, :]
+    n, T = x.shape
+    if T % V:
+        raise ValueError("V must divide T")
+    d = _f64(d)
+    if d is not None:
+        d = np.ascontiguousarray(np.broadcast_to(d.reshape(-1, T) if d.ndim > 1 else d, (n, T)))
+    cb = _f64(codebook).reshape(-1)
+    if cb.size != 4 * (1 << m) * V:
+        raise ValueError(f"codebook must hold 4 * 2^m rows of V values, got {cb.size}")
+    W = oracle_words_per_block(1 + m, T // V)
+    start = np.zeros(n, dtype=np.uint32)
+    bits = np.zeros((n, W), dtype=np.uint32)
+    cost = np.zeros(n, dtype=np.float64)
+    rc = _load().oracle_ub8_encode(
+        _ptr(x, ctypes.c_double), _ptr(d, ctypes.c_double), _ptr(cb, ctypes.c_double),
+        V, m, T, n, -1 if fixed_start is None else int(fixed_start),
+        _ptr(start, ctypes.c_uint32), _ptr(bits, ctypes.c_uint32), _ptr(cost, ctypes.c_double),
+    )
+    if rc != 0:
+        raise ValueError(f"oracle_ub8_encode failed with code {rc}")
+    return start, bits, cost
+
+
+def oracle_ub8_decode(bits, start_state, codebook, V: int, m: int, T: int):
+    """Decode 8-state set-partitioned trellis streams ([n, W]) to fp64 values [n, T]."""
+    bits = _u32(bits)
+    if bits.ndim == 1:
+        bits = bits[None, :]
+    n = bits.shape[0]
+    start = _u32(start_state).reshape(n)
+    cb = _f64(codebook).reshape(-1)
+    if cb.size != 4 * (1 << m) * V:
+        raise ValueError("codebook must hold 4 * 2^m rows of V values")
+    if bits.shape[1] != oracle_words_per_block(1 + m, T // V):
+        raise ValueError("bits has the wrong number of words per block")
+    y = np.zeros((n, T), dtype=np.float64)
+    rc = _load().oracle_ub8_decode(_ptr(bits, ctypes.c_uint32), _ptr(start, ctypes.c_uint32),
+                                   _ptr(cb, ctypes.c_double), V, m, T, n, _ptr(y, ctypes.c_double))
+    if rc != 0:
+        raise ValueError(f"oracle_ub8_decode failed with code {rc}")
     return y

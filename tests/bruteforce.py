@@ -135,3 +135,72 @@ def decode_window_vec(words, start: int, codebook, L: int, k: int, V: int, T: in
     st = [((s0 << (t * K)) | (n >> ((steps - t) * K))) & mask for t in range(1, steps + 1)]
     c = np.asarray(codebook, dtype=np.float64).reshape(1 << L, V)
     return c[np.array(st, dtype=np.int64)].reshape(-1)
+
+
+# ---------------------------------------------------------------------------
+# Ungerboeck's 8-state set-partitioned trellis, read from its parity-check
+# equation alone (no state machine): a label sequence (z1_t, z0_t) is a path
+# of the code with h0 = D^3 + D + 1 and h1 = D^2 iff
+#     z0_t = z0_{t-1} ^ z0_{t-3} ^ z1_{t-2}      for t >= 4,
+# with z0_1, z0_2, z0_3 free (they carry the start state).  Step t emits row
+# 4 i_t + 2 z1_t + z0_t of the union codebook.
+# ---------------------------------------------------------------------------
+def ub8_first_parities(start: int, z1_first: int):
+    """z0_1, z0_2, z0_3 of a path from state start = 4p + 2q + r whose first
+    branch bit is z1_first: the register contents read off the code's
+    realisation (p, then p ^ q, then p ^ q ^ r ^ z1_1)."""
+    p, q, r = (start >> 2) & 1, (start >> 1) & 1, start & 1
+    return p, p ^ q, p ^ q ^ r ^ z1_first
+
+
+def ub8_parities(z1, head):
+    """Every z0_t of a path from its branch bits and its first three parities."""
+    S = len(z1)
+    z0 = list(head[:min(3, S)])
+    for t in range(3, S):  # 0-based t is step t + 1
+        z0.append(z0[t - 1] ^ z0[t - 3] ^ z1[t - 2])
+    return z0
+
+
+def ub8_brute_force(x, d, codebook, V: int, m: int, fixed_start: int | None = None):
+    """Minimum of J over every code sequence of the trellis (every choice of the
+    three free parities, of the branch bits and of the entries inside the
+    subsets), enumerated without the state machine.  Returns (J_min, rows)."""
+    import itertools
+
+    x = np.asarray(x, dtype=np.float64).reshape(-1)
+    T = x.size
+    S = T // V
+    d = np.ones(T) if d is None else np.asarray(d, dtype=np.float64).reshape(-1)
+    c = np.asarray(codebook, dtype=np.float64).reshape(4 << m, V)
+    assert 3 + S * (1 + m) <= 18, "keep the enumeration small"
+    xs, ds = x.reshape(S, V), d.reshape(S, V)
+    best, best_rows = np.inf, None
+    for z1 in itertools.product((0, 1), repeat=S):
+        if fixed_start is None:
+            heads = list(itertools.product((0, 1), repeat=3))
+        else:
+            heads = [ub8_first_parities(fixed_start & 7, z1[0])]
+        for head in heads:
+            z0 = ub8_parities(z1, head)
+            subs = [2 * z1[t] + z0[t] for t in range(S)]
+            # every choice of entries: [2^(mS), S] row indices
+            ii = np.array(list(itertools.product(range(1 << m), repeat=S)), dtype=np.int64)
+            rows = 4 * ii + np.array(subs, dtype=np.int64)[None, :]
+            J = (ds[None] * (xs[None] - c[rows]) ** 2).sum(axis=(1, 2))
+            a = int(np.argmin(J))
+            if J[a] < best:
+                best, best_rows = float(J[a]), rows[a]
+    return best, best_rows
+
+
+def ub8_decode_parity(words, start: int, codebook, V: int, m: int, T: int) -> np.ndarray:
+    """Values of one block from its words and start state, through the parity
+    equation instead of the state machine."""
+    S = T // V
+    sym = unpack_symbols(words, 1 + m, S)
+    z1 = [int(b) >> m for b in sym]
+    ii = [int(b) & ((1 << m) - 1) for b in sym]
+    z0 = ub8_parities(z1, ub8_first_parities(int(start) & 7, z1[0]))
+    c = np.asarray(codebook, dtype=np.float64).reshape(4 << m, V)
+    return np.concatenate([c[4 * ii[t] + 2 * z1[t] + z0[t]] for t in range(S)])
