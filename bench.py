@@ -585,6 +585,49 @@ def run_ours(args, rank, world, local_rank):
                "cost_per_weight": float(vcost.astype(np.float64).sum()) / (n * T)}
         del xv_t, dv_t, vws, vout
 
+    # ---- Ungerboeck's 8-state set-partitioned trellis over the same blocks:
+    # symbols of V = 4 weights, 1 + m = 8 bits per step (2 bits per weight),
+    # a Gaussian binary16 union codebook of 512 rows in four subsets
+    ub8 = None
+    if rank == 0 and world == 1 and not args.no_ub8:
+        torch.cuda.empty_cache()
+        V8, m8 = 4, 7
+        xu = torch.from_numpy(wl.x).to(dev)
+        du = None if wl.d is None else torch.from_numpy(wl.d).to(dev)
+        cbu = torch.from_numpy(workloads.ub8_gaussian_codebook(V8, m8, "f16")).to(dev)
+        uout = tcq.ub8_encode(xu, du, cbu, V8, m8)
+        yu = tcq.ub8_decode(uout.bits, uout.start_state, cbu, V8, m8, T)
+        for _ in range(3):
+            tcq.ub8_encode(xu, du, cbu, V8, m8, out=uout)
+            tcq.ub8_decode(uout.bits, uout.start_state, cbu, V8, m8, T, out=yu)
+        ue, ud = [], []
+        for _ in range(10):
+            a, b2, c2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            a.record(stream)
+            tcq.ub8_encode(xu, du, cbu, V8, m8, out=uout)
+            b2.record(stream)
+            tcq.ub8_decode(uout.bits, uout.start_state, cbu, V8, m8, T, out=yu)
+            c2.record(stream)
+            ue.append((a, b2))
+            ud.append((b2, c2))
+        torch.cuda.synchronize()
+        u_ms, ud_ms = _median_ms(ue), _median_ms(ud)
+        ucost = uout.path_cost.cpu().numpy()
+        assert np.all(np.isfinite(ucost)) and np.all(ucost >= 0)
+        steps = n * (T // V8)
+        cands = steps * (4 << m8)  # every row of the union scored at every step
+        u_ops = cands * (2 * V8 + 1)  # V errors, V square-accumulates, one compare-select
+        Wu = tcq.tcq_ub8_words_per_block(V8, m8, T)
+        ud_bytes = n * T * 4 + n * Wu * 4 + n * 4
+        ub8 = {"workload": wl.name + "_ub8_V4_m7", "V": V8, "m": m8, "bits_per_weight": (1 + m8) / V8,
+               "timing": "median of 10 after 3 warm-ups",
+               "ms": u_ms, "weights_per_s": n * T / (u_ms / 1e3),
+               "candidates_per_s": cands / (u_ms / 1e3), "ops_per_candidate": 2 * V8 + 1,
+               "bound": "alu", "alu_frac": u_ops / (u_ms / 1e3) / peaks_ops(),
+               "decode_ms": ud_ms, "decode_hbm_frac": ud_bytes / (ud_ms / 1e3) / 1e9 / peaks_hbm(),
+               "cost_per_weight": float(ucost.astype(np.float64).sum()) / (n * T)}
+        del xu, du, cbu, uout, yu
+
     # sanity: the last step's result is a valid encode of the workload (cheap host check)
     cost_h = cost_last
     assert np.all(np.isfinite(cost_h)) and np.all(cost_h >= 0)
@@ -638,6 +681,7 @@ def run_ours(args, rank, world, local_rank):
         "encode_ms_per_step": acs_ms, "decode_ms_per_step": dec_ms,
         "roofline": roofline, "decode_roofline": decode_roofline, "cpu_baseline": cpu_baseline, "e2e": e2e,
         "per_workload": per_workload, "gemv": gemv, "ldlq": ldlq, "bcjr": bcjr, "vec": vec, "fixed_start": fixed,
+        "ub8": ub8,
         "clocks": clock_record, "remeasured": remeasured, "gpu_launches": gpu_launches,
     }
     print(json.dumps(line), flush=True)
@@ -660,6 +704,8 @@ def main():
                     help="skip the fixed-start encode of the workload")
     ap.add_argument("--no-vec", action="store_true",
                     help="skip the vector-trellis (V = 2) encode of the workload")
+    ap.add_argument("--no-ub8", action="store_true",
+                    help="skip the 8-state set-partitioned trellis encode of the workload")
     ap.add_argument("--no-ldlq", action="store_true",
                     help="skip the error-feedback encode of the MLP matrix")
     ap.add_argument("--cpu-blocks-per-core", type=int, default=16)

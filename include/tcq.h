@@ -320,6 +320,72 @@ tcq_status tcq_gemv_vec(const uint32_t* bits, const uint32_t* start_state, const
                         const void* codebook, tcq_dtype cb_dtype, int L, int k, int V, int T,
                         int64_t rows, int64_t cols, const float* x, float* y, tcq_stream_t stream);
 
+/*
+ * Trellis-coded quantization over Ungerboeck's 8-state set-partitioned trellis
+ * (the 2-bit post, Pingala-8 section: an 8-state set-partitioned trellis with
+ * Ungerboeck's labels over symbols of several weights at about 2 bits per
+ * weight; its section on trellis-coded quantization: the state decides which
+ * subset the next symbol may use, the written bits pick a value inside the
+ * subset and set the next state, so the format holds twice as many values as
+ * its bits address; its background reading, Marcellin and Fischer's
+ * trellis-coded quantization, fixes the labels used here).  The pages give
+ * neither labels nor codebook; this library's reading:
+ *
+ *   - Union codebook: 4 * 2^m rows of V values (row-major); row r belongs to
+ *     subset D_{r mod 4} and is entry r >> 2 of it.  For V = 1 and rows sorted
+ *     ascending this is Ungerboeck's partition of an amplitude alphabet.
+ *   - Trellis: Ungerboeck's 8-state code for one-dimensional signals (the
+ *     rate-1/2 systematic feedback code with parity-check polynomials
+ *     h0 = D^3 + D + 1, h1 = D^2, octal 13 and 04).  State sigma = 4p + 2q + r;
+ *     the branch with bit z uses subset D_{2z+p} and leads to state
+ *     4 (p ^ q) + 2 (r ^ z) + p.  Both branches out of a state use the two
+ *     subsets of one half, {D_p, D_{p+2}}.
+ *   - A step codes V consecutive weights with 1 + m bits, symbol (z << m) | i,
+ *     and reconstructs them as row 4 i + 2 z + p.  Symbols are packed like
+ *     tcq_encode's (MSB first, symbol t at stream bits [t(1+m), (t+1)(1+m)));
+ *     W = tcq_ub8_words_per_block(V, m, T) words per block.  The stored start
+ *     state is sigma_0 (0..7).  Pingala-8's symbols of 4 weights at 2 bits per
+ *     weight are V = 4, m = 7 (512 rows, 8 bits per step).
+ *
+ * tcq_ub8_encode returns per block the start state, branch bits and entries
+ * that minimise J = sum_i d_i (x_i - y_i)^2 over every path of the trellis (free
+ * start, or fixed_start[b] & 7 when fixed_start is not NULL): per step the
+ * nearest entry of each subset (fp32, ties to the smaller entry), then the
+ * Viterbi recursion over the 8 states (fp32 path metrics, ties to the smaller
+ * predecessor and the smaller final state).  path_cost is J of the returned
+ * path summed in fp64 and rounded once.  Like tcq_encode, every returned path
+ * is optimal up to fp32 rounding of the search.  No workspace: the search of a
+ * block lives in shared memory.
+ *
+ *   x, d            fp32 [n_blocks, T] (d NULL: d = 1), 4-byte aligned.
+ *   codebook        4 * 2^m * V entries of cb_dtype (TCQ_F32 or TCQ_F16; the
+ *                   computed code is TCQ_ERR_UNSUPPORTED), aligned to the entry.
+ *   fixed_start     uint32 [n_blocks] or NULL.
+ *   start_state     out: uint32 [n_blocks].   bits: out uint32 [n_blocks, W].
+ *   path_cost       out: fp32 [n_blocks].
+ * tcq_ub8_decode writes y[b, (t-1)V + v] = row[v] of each step's row; it reads
+ * only the low 3 bits of start_state.  Bit-exact (the exact fp32 widening).
+ * Supported: 1 <= V <= TCQ_UB8_MAX_V, 0 <= m <= TCQ_UB8_MAX_M, V | T,
+ * T / V <= TCQ_UB8_MAX_STEPS (else TCQ_ERR_UNSUPPORTED); pointers as for
+ * tcq_encode / tcq_decode (else TCQ_ERR_INVALID_ARG).  n_blocks == 0 is a
+ * no-op.  One kernel launch each.
+ */
+#define TCQ_UB8_MAX_V 8
+#define TCQ_UB8_MAX_M 8
+#define TCQ_UB8_MAX_STEPS 512
+
+/* ceil((T / V) (1 + m) / 32); -1 for a shape tcq_ub8_encode rejects. */
+int tcq_ub8_words_per_block(int V, int m, int T);
+
+tcq_status tcq_ub8_encode(const float* x, const float* d, const void* codebook, tcq_dtype cb_dtype,
+                          int V, int m, int T, int64_t n_blocks, const uint32_t* fixed_start,
+                          uint32_t* start_state, uint32_t* bits, float* path_cost,
+                          tcq_stream_t stream);
+
+tcq_status tcq_ub8_decode(const uint32_t* bits, const uint32_t* start_state, const void* codebook,
+                          tcq_dtype cb_dtype, int V, int m, int T, int64_t n_blocks, float* y,
+                          tcq_stream_t stream);
+
 /* Static, human-readable name of a status code. */
 const char* tcq_status_string(tcq_status status);
 

@@ -173,3 +173,50 @@ def test_vector_and_feedback_entry_points_reject_on_the_host(lib):
     assert dv(n=0) == tcq.TCQ_OK
     assert dv(T=255) == tcq.TCQ_ERR_UNSUPPORTED
     assert dv(y=ctypes.c_void_p(0x10002)) == tcq.TCQ_ERR_INVALID_ARG
+
+
+def test_set_partitioned_trellis_entry_points_reject_on_the_host(lib):
+    """tcq_ub8_*: sizes as documented, shapes and pointers refused before any CUDA call."""
+    fake = ctypes.c_void_p(0x10000)
+    F16, F32 = tcq.TCQ_F16, tcq.TCQ_F32
+    assert tcq.tcq_ub8_words_per_block(4, 7, 256) == 16        # 64 steps x 8 bits
+    assert tcq.tcq_ub8_words_per_block(1, 1, 100) == 7         # 100 steps x 2 bits
+    assert tcq.tcq_ub8_words_per_block(3, 0, 9) == 1
+    assert tcq.tcq_ub8_words_per_block(8, 8, 4096) == 144      # 512 steps x 9 bits
+    assert tcq.tcq_ub8_words_per_block(4, 7, 255) == -1       # V does not divide T
+    assert tcq.tcq_ub8_words_per_block(9, 1, 9) == -1
+    assert tcq.tcq_ub8_words_per_block(1, 9, 8) == -1
+    assert tcq.tcq_ub8_words_per_block(1, 1, 513) == -1        # more than 512 steps
+    assert tcq.tcq_ub8_words_per_block(0, 1, 8) == -1
+
+    def enc(**o):
+        return tcq.tcq_ub8_encode(o.get("x", fake), o.get("d", None), o.get("cb", fake),
+                                  o.get("dt", F32), o.get("V", 4), o.get("m", 7), o.get("T", 256),
+                                  o.get("n", 4), o.get("fs", None), o.get("st", fake),
+                                  o.get("bits", fake), o.get("cost", fake), None)
+
+    assert enc(n=0, x=None, cb=None, st=None, bits=None, cost=None) == tcq.TCQ_OK
+    assert enc(n=-1) == tcq.TCQ_ERR_INVALID_ARG
+    assert enc(x=None) == tcq.TCQ_ERR_INVALID_ARG
+    assert enc(cost=None) == tcq.TCQ_ERR_INVALID_ARG
+    assert enc(x=ctypes.c_void_p(0x10002)) == tcq.TCQ_ERR_INVALID_ARG
+    assert enc(fs=ctypes.c_void_p(0x10001)) == tcq.TCQ_ERR_INVALID_ARG
+    assert enc(dt=F16, cb=ctypes.c_void_p(0x10001)) == tcq.TCQ_ERR_INVALID_ARG
+    assert enc(dt=tcq.TCQ_MAD, cb=None) == tcq.TCQ_ERR_UNSUPPORTED
+    assert enc(dt=7) == tcq.TCQ_ERR_INVALID_ARG
+    assert enc(T=254) == tcq.TCQ_ERR_UNSUPPORTED
+    assert enc(V=9, T=261) == tcq.TCQ_ERR_UNSUPPORTED
+    assert enc(m=9) == tcq.TCQ_ERR_UNSUPPORTED
+    assert enc(V=1, T=600) == tcq.TCQ_ERR_UNSUPPORTED
+
+    def dec(**o):
+        return tcq.tcq_ub8_decode(o.get("bits", fake), o.get("st", fake), o.get("cb", fake),
+                                  o.get("dt", F32), o.get("V", 4), o.get("m", 7), o.get("T", 256),
+                                  o.get("n", 4), o.get("y", fake), None)
+
+    assert dec(n=0, bits=None, st=None, cb=None, y=None) == tcq.TCQ_OK
+    assert dec(y=None) == tcq.TCQ_ERR_INVALID_ARG
+    assert dec(st=ctypes.c_void_p(0x10002)) == tcq.TCQ_ERR_INVALID_ARG
+    assert dec(m=-1) == tcq.TCQ_ERR_UNSUPPORTED
+    assert dec(dt=tcq.TCQ_MAD, cb=None) == tcq.TCQ_ERR_UNSUPPORTED
+    assert dec(n=-3) == tcq.TCQ_ERR_INVALID_ARG

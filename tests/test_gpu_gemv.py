@@ -4,7 +4,11 @@ Tolerance: each product scale * c * x reaches y through at most
 13 + ceil(cols / 256) fp32 roundings: at most 5 in the FMA chains of its quad or
 8-weight item, at most 4 into a lane's per-fetch sum, one addition per fetch
 (512 or 256 columns, depending on the kernel) into the lane's row sum, and a
-5-level warp reduction.  So
+5-level warp reduction.  The kernel for L = 16, k = 2, T = 256 and 4096-column
+chunks (lanes on half blocks, two rows per item) has at most 23 + cols / 4096:
+8 in a stream word's FMA chain, 8 into a block sum, 1 for the two block sums,
+1 for the scale, one per 4096-column chunk and 5 in the warp reduction (its
+rows left for a last partial round: 4 + 1 + 1 + cols / 4096 + 5 + 16).  So
 |y_gpu - y_exact| <= (13 + ceil(cols / 256)) * 2^-24 * sum |scale * c * x|.
 """
 import ctypes
@@ -111,3 +115,63 @@ def test_gemv_rejections(cuda_device):
     assert call(x=ctypes.c_void_p(0x10004)) == tcq.TCQ_ERR_INVALID_ARG
     assert call(y=None) == tcq.TCQ_ERR_INVALID_ARG
     assert call(L=17) == tcq.TCQ_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("rows,nb,code", [
+    (5000, 16, "f16"),    # two rows per item for every warp, then one row per CTA
+    (5000, 16, "mad"),
+    (4737, 32, "f16"),    # two 4096-column chunks per row; an odd row left for the last round
+    (4801, 32, "mad"),
+    (9473, 16, "mad"),    # several items per warp, 1 row in the last round
+    (37, 16, "f16"),      # fewer rows than warps: only the per-CTA rows
+])
+@pytest.mark.parametrize("scaled", [False, True])
+def test_gemv_half_block_kernel(rows, nb, code, scaled, cuda_device):
+    """L = 16, k = 2, T = 256 with cols a multiple of 4096: the kernel that takes
+    half a coding block per lane and two rows per item, in both of its phases
+    (every warp's share of row pairs, then the rows left, one per CTA)."""
+    import torch
+    from oracle import oracle_mad_codebook
+
+    L, k, T = 16, 2, 256
+    rng = np.random.default_rng(rows + nb + (1 if code == "mad" else 0) + (2 if scaled else 0))
+    cols = nb * T
+    bits, start = _rand_stream(rng, rows * nb, k, T)
+    scale = rng.lognormal(0.0, 0.5, rows * nb).astype(np.float32) if scaled else None
+    x = rng.standard_normal(cols).astype(np.float32)
+    if code == "mad":
+        dev = torch.device("cuda", 0)
+        b = torch.from_numpy(np.ascontiguousarray(bits).view(np.int32)).to(dev)
+        s = torch.from_numpy(np.ascontiguousarray(start).view(np.int32)).to(dev)
+        sc = None if scale is None else torch.from_numpy(scale).to(dev)
+        y = tcq.gemv(b, s, sc, tcq.MAD, L, k, T, rows, cols, torch.from_numpy(x).to(dev))
+        torch.cuda.synchronize()
+        y = y.cpu().numpy()
+        cb = oracle_mad_codebook(L).astype(np.float16)
+    else:
+        cb = rng.standard_normal(1 << L).astype(np.float16)
+        y = _gpu_gemv(bits, start, scale, cb, L, k, T, rows, cols, x)
+    _check(bits, start, scale, cb, L, k, T, rows, cols, x, y)
+
+
+def test_gemv_misaligned_bits_take_the_general_kernel(cuda_device):
+    """Bits that are 4-byte but not 16-byte aligned are legal: the call takes a
+    kernel without 16-byte loads and gives the same product within the bound."""
+    import torch
+
+    L, k, T, rows, nb = 16, 2, 256, 40, 16
+    rng = np.random.default_rng(77)
+    cols = nb * T
+    bits, start = _rand_stream(rng, rows * nb, k, T)
+    cb = rng.standard_normal(1 << L).astype(np.float16)
+    x = rng.standard_normal(cols).astype(np.float32)
+    dev = torch.device("cuda", 0)
+    padded = torch.zeros(bits.size + 1, dtype=torch.int32, device=dev)
+    padded[1:] = torch.from_numpy(np.ascontiguousarray(bits).view(np.int32).reshape(-1)).to(dev)
+    b = padded[1:]
+    assert b.data_ptr() % 16 == 4
+    s = torch.from_numpy(np.ascontiguousarray(start).view(np.int32)).to(dev)
+    y = tcq.gemv(b, s, None, torch.from_numpy(cb).to(dev), L, k, T, rows, cols,
+                 torch.from_numpy(x).to(dev))
+    torch.cuda.synchronize()
+    _check(bits, start, None, cb, L, k, T, rows, cols, x, y.cpu().numpy())

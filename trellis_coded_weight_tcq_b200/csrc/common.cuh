@@ -100,6 +100,31 @@ struct BcjrArgs {
     size_t slot_bytes;
 };
 
+// Encode over the 8-state set-partitioned trellis (ub8.cu): n_blocks blocks of
+// T weights, T / V steps of V weights and 1 + m bits each.
+struct Ub8EncodeArgs {
+    const float* x;               // [n_blocks, T]
+    const float* d;               // [n_blocks, T] or nullptr (d = 1)
+    const void* cb;               // union codebook [4 * 2^m, V]
+    int cb_f16;
+    int V, m, T, W;               // W = words per block
+    long long n_blocks;
+    const uint32_t* fixed_start;  // [n_blocks] (low 3 bits) or nullptr: free start
+    uint32_t* start_state;        // [n_blocks]
+    uint32_t* bits;               // [n_blocks, W]
+    float* path_cost;             // [n_blocks]
+};
+
+struct Ub8DecodeArgs {
+    const uint32_t* bits;         // [n_blocks, W]
+    const uint32_t* start_state;  // [n_blocks], low 3 bits read
+    const void* cb;
+    int cb_f16;
+    int V, m, T, W;
+    long long n_blocks;
+    float* y;                     // [n_blocks, T]
+};
+
 // One codebook entry, widened exactly to fp32.
 __device__ __forceinline__ float load_codeword(const void* cb, int f16, uint32_t s)
 {
@@ -189,5 +214,10 @@ cudaError_t launch_gemv_vec(const GemvArgs& a, int V, int num_sms, cudaStream_t 
 // Drops [base, base + bytes) from L2 without write-back (base 128-byte aligned).
 cudaError_t launch_discard_l2(void* base, size_t bytes, int num_sms, cudaStream_t stream);
 cudaError_t launch_gemv(const GemvArgs& a, int num_sms, cudaStream_t stream);
+// 8-state set-partitioned trellis: shared memory per CTA, and the launches
+size_t ub8_encode_smem_bytes(int V, int m, int T);
+size_t ub8_decode_smem_bytes(int V, int m, int T);
+cudaError_t launch_ub8_encode(const Ub8EncodeArgs& a, int num_sms, cudaStream_t stream);
+cudaError_t launch_ub8_decode(const Ub8DecodeArgs& a, int num_sms, cudaStream_t stream);
 
 }  // namespace tcq

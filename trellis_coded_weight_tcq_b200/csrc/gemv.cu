@@ -461,6 +461,270 @@ __global__ void __launch_bounds__(kMadRowsThreads, 1) gemv_rows_kernel(GemvArgs 
     }
 }
 
+// ---------------------------------------------------------------------------
+// L = 16, k = 2, T = 256, cols a multiple of 4096: the layout for the matrices
+// a model layer has.  A warp's lane (j, h) = (lane >> 1, lane & 1) takes half h
+// (128 weights, 8 stream words) of the coding block j of a 16-block (4096
+// column) chunk, for two rows at a time: the lane's x values are then the same
+// for both rows, its words are two 16-byte loads per row (a half-warp reads
+// 1 KiB of one row contiguously), the window before its first weight is the
+// block's start state (h = 0) or the block's word 7 (h = 1), and the row sums
+// need one 5-step warp reduction per row.  x sits in shared memory with 16
+// bytes of padding after every 128 values, so the 16-byte loads of 8
+// consecutive lanes hit 8 different bank quads.
+//
+// States, 16 windows per stream word lo (with hi the word before): window i
+// (i = 1..16) is bits [32 - 2i, 48 - 2i) of the 64-bit hi:lo.  Seven funnel
+// shifts give "views" of the pair at bit offsets 2, 4, 6, 16, 18, 20, 22, in
+// which every window starts at bit 0, 8 or 16, so each state is then one
+// byte permutation, mask or shift (23 instructions per 16 states instead of 2
+// per state).
+//
+// Rows: phase A gives every warp of the grid the same number of row pairs;
+// the rows left over (fewer than two per warp of the grid) are phase B, one row
+// per CTA at a time, each warp taking coding blocks w, w + 16, ... with lanes
+// on 8-weight items, and the CTA summing its 16 warp sums in a fixed order, so
+// that the last round costs a sixteenth of a row instead of a whole row pair.
+// Every sum has a fixed order: the result does not depend on timing.
+//
+// Rounding depth of a product (the tolerance tests/test_gpu_gemv.py uses):
+// phase A, 8 in a word's FMA chain, 8 over the words into the block sum, 1 for
+// the two block sums, 1 for the scale, c = cols / 4096 over the chunks, 5 in
+// the warp reduction: 23 + c <= 13 + cols / 256.  Phase B: 4 + 1 + 1 +
+// cols / 4096 + 5 + 16 <= 13 + cols / 256.
+// ---------------------------------------------------------------------------
+constexpr int kPairThreads = 512;
+constexpr int kPairWarps = kPairThreads / 32;
+constexpr int kPairRows = 2;  // rows per warp item
+
+// padded position of x[i] in shared memory: 4 floats of padding per 128
+__device__ __forceinline__ int xpad(int i) { return i + ((i >> 7) << 2); }
+
+// byte permutation of (b:a) with selector sel (PTX prmt, default mode)
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
+{
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+// The 16 states of stream word lo (hi is the word before), in stream order.
+__device__ __forceinline__ void states16(uint32_t hi, uint32_t lo, uint32_t (&s)[16])
+{
+    const uint32_t v2 = __funnelshift_r(lo, hi, 2), v4 = __funnelshift_r(lo, hi, 4);
+    const uint32_t v6 = __funnelshift_r(lo, hi, 6), v16 = __funnelshift_r(lo, hi, 16);
+    const uint32_t v18 = __funnelshift_r(lo, hi, 18), v20 = __funnelshift_r(lo, hi, 20);
+    const uint32_t v22 = __funnelshift_r(lo, hi, 22);
+    // window i starts at bit 32 - 2i of hi:lo; 0x4421 picks bytes 1, 2 and two zero
+    // bytes of the second operand (0): bits 8..23
+    s[0] = prmt(v22, 0u, 0x4421);   // i = 1, bit 30 = 22 + 8
+    s[1] = prmt(v20, 0u, 0x4421);   // i = 2, bit 28
+    s[2] = prmt(v18, 0u, 0x4421);   // i = 3, bit 26
+    s[3] = prmt(v16, 0u, 0x4421);   // i = 4, bit 24
+    s[4] = v22 & 0xFFFFu;           // i = 5, bit 22
+    s[5] = v20 & 0xFFFFu;           // i = 6, bit 20
+    s[6] = v18 & 0xFFFFu;           // i = 7, bit 18
+    s[7] = v16 & 0xFFFFu;           // i = 8, bit 16
+    s[8] = prmt(v6, 0u, 0x4421);    // i = 9, bit 14
+    s[9] = prmt(v4, 0u, 0x4421);    // i = 10, bit 12
+    s[10] = prmt(v2, 0u, 0x4421);   // i = 11, bit 10
+    s[11] = prmt(lo, 0u, 0x4421);   // i = 12, bit 8
+    s[12] = v6 & 0xFFFFu;           // i = 13, bit 6
+    s[13] = v4 & 0xFFFFu;           // i = 14, bit 4
+    s[14] = v2 & 0xFFFFu;           // i = 15, bit 2
+    s[15] = lo & 0xFFFFu;           // i = 16, bit 0
+}
+
+// Codeword of state s: the computed code as 128 c (n - 255, exact; the 2^-7 goes
+// with the block scale), or the binary16 table entry.
+template <int CODE>
+__device__ __forceinline__ float pair_codeword(uint32_t s, const __half* tab)
+{
+    if constexpr (CODE == kCodeMad) {
+        const uint32_t nb23 = __dp4a(s * kMadA, 0x01010000u, 0x4B000000u);  // bits of 2^23 + n
+        return __uint_as_float(nb23) - 8388863.0f;
+    } else {
+        return __half2float(tab[s]);
+    }
+}
+
+// sum over the 16 weights of stream word lo of c[s] x, as two chains of 8
+template <int CODE>
+__device__ __forceinline__ void word_dot(uint32_t hi, uint32_t lo, const float* __restrict__ xq,
+                                         const __half* tab, float& acc0, float& acc1)
+{
+    uint32_t st[16];
+    states16(hi, lo, st);
+    float xv[16];
+#pragma unroll
+    for (int e = 0; e < 16; e += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(xq + e);
+        xv[e] = v.x;
+        xv[e + 1] = v.y;
+        xv[e + 2] = v.z;
+        xv[e + 3] = v.w;
+    }
+    float p0 = pair_codeword<CODE>(st[0], tab) * xv[0];
+    float p1 = pair_codeword<CODE>(st[1], tab) * xv[1];
+#pragma unroll
+    for (int e = 2; e < 16; e += 2) {
+        p0 = fmaf(pair_codeword<CODE>(st[e], tab), xv[e], p0);
+        p1 = fmaf(pair_codeword<CODE>(st[e + 1], tab), xv[e + 1], p1);
+    }
+    acc0 += p0;
+    acc1 += p1;
+}
+
+template <int CODE>
+__global__ void __launch_bounds__(kPairThreads, 1) gemv_pair_kernel(GemvArgs a)
+{
+    constexpr int T = 256, W = 16;
+    extern __shared__ __align__(16) unsigned char gsm[];
+    constexpr size_t TAB = CODE == kCodeMad ? 0 : ((size_t)1 << 16) * 2;
+    const __half* tab = reinterpret_cast<const __half*>(gsm);
+    float* xs = reinterpret_cast<float*>(gsm + TAB);
+    float* wsum = xs + xpad((int)a.cols);  // kPairWarps partial sums of phase B
+    // stage the table (16-byte asynchronous copies) and x (padded)
+    if constexpr (CODE != kCodeMad) {
+        const char* src = reinterpret_cast<const char*>(a.cb);
+        const uint32_t dst = (uint32_t)__cvta_generic_to_shared(gsm);
+        for (int i = threadIdx.x; i < (int)(TAB / 16); i += blockDim.x)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + 16 * i),
+                         "l"(src + 16 * (size_t)i) : "memory");
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    }
+    for (int i = threadIdx.x; i < (int)(a.cols / 4); i += blockDim.x) {
+        const float4 v = reinterpret_cast<const float4*>(a.x)[i];
+        *reinterpret_cast<float4*>(xs + xpad(4 * i)) = v;
+    }
+    if constexpr (CODE != kCodeMad) asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int jl = lane >> 1, h = lane & 1;  // block of the 16-block chunk, half
+    const long long nb = a.cols / T;
+    const int nch = (int)(nb / 16);          // 4096-column chunks per row
+    const float sc_code = CODE == kCodeMad ? 0.0078125f : 1.f;
+    const long long gw = (long long)blockIdx.x * kPairWarps + warp;
+    const long long nw = (long long)gridDim.x * kPairWarps;
+    const long long pairs = a.rows / kPairRows;
+    const long long rounds = pairs / nw;     // phase A: the same number for every warp
+
+    // ---- phase A
+    struct Item {
+        uint4 w[kPairRows][2];
+        uint32_t prev[kPairRows];
+        float sc[kPairRows];
+    };
+    auto fetch = [&](Item& it, long long r0, int c) {
+#pragma unroll
+        for (int i = 0; i < kPairRows; ++i) {
+            const long long b = (r0 + i) * nb + 16LL * c + jl;
+            const uint4* wp = reinterpret_cast<const uint4*>(a.bits + b * W + 8 * h);
+            it.w[i][0] = wp[0];
+            it.w[i][1] = wp[1];
+            it.prev[i] = h ? a.bits[b * W + 7] : a.start_state[b];
+            it.sc[i] = (a.scale ? a.scale[b] : 1.f) * sc_code;
+        }
+    };
+    auto consume = [&](const Item& it, int c, float (&row)[kPairRows]) {
+        const float* xl = xs + xpad(c * 4096 + 128 * lane);  // the lane's 128 x values, unpadded inside
+        float a0[kPairRows], a1[kPairRows];
+#pragma unroll
+        for (int i = 0; i < kPairRows; ++i) a0[i] = a1[i] = 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+#pragma unroll
+            for (int i = 0; i < kPairRows; ++i) {
+                const uint32_t* wd = reinterpret_cast<const uint32_t*>(&it.w[i][0]);
+                const uint32_t hi = q == 0 ? it.prev[i] : wd[q - 1];
+                word_dot<CODE>(hi, wd[q], xl + 16 * q, tab, a0[i], a1[i]);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kPairRows; ++i) row[i] = fmaf(it.sc[i], a0[i] + a1[i], row[i]);
+    };
+    if (rounds > 0) {
+        // items (pair, chunk) of this warp in order; two buffers, no copies
+        const long long n_items = rounds * nch;
+        auto item_row = [&](long long t) { return (gw + (t / nch) * nw) * kPairRows; };
+        Item A, B;
+        fetch(A, item_row(0), 0);
+        float row[kPairRows];
+#pragma unroll
+        for (int i = 0; i < kPairRows; ++i) row[i] = 0.f;
+        auto finish = [&](long long t) {  // item t was the last chunk of its pair
+            const long long r0 = item_row(t);
+#pragma unroll
+            for (int i = 0; i < kPairRows; ++i) {
+                float v = row[i];
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                if (lane == 0) a.y[r0 + i] = v;
+                row[i] = 0.f;
+            }
+        };
+        for (long long t = 0; t < n_items; t += 2) {
+            if (t + 1 < n_items) fetch(B, item_row(t + 1), (int)((t + 1) % nch));
+            consume(A, (int)(t % nch), row);
+            if ((t + 1) % nch == 0) finish(t);
+            if (t + 1 >= n_items) break;
+            if (t + 2 < n_items) fetch(A, item_row(t + 2), (int)((t + 2) % nch));
+            consume(B, (int)((t + 1) % nch), row);
+            if ((t + 2) % nch == 0) finish(t + 1);
+        }
+    }
+
+    // ---- phase B: the remaining rows, one per CTA at a time; warp w takes
+    // blocks w, w + 16, ... of the row, lane l the 8 weights [8l, 8l + 8)
+    const long long first_b = rounds * nw * kPairRows;
+    const int p0 = 16 * lane - 14;  // stream bit of the item's first window (k = 2, L = 16)
+    const int wi = p0 >> 5, off = p0 & 31;  // word -1 is the start state
+    for (long long r = first_b + blockIdx.x; r < a.rows; r += gridDim.x) {
+        float acc = 0.f;
+        for (long long j = warp; j < nb; j += kPairWarps) {
+            const long long b = r * nb + j;
+            const uint32_t* wb = a.bits + b * W;
+            const uint32_t hi = wi < 0 ? a.start_state[b] : wb[wi];
+            const uint32_t lo = wi + 1 < W ? wb[wi + 1] : 0u;  // lane 31 ends on the last word
+            const uint32_t w = __funnelshift_l(lo, hi, off);
+            const float* xq = xs + xpad((int)(j * T) + 8 * lane);
+            float q0 = 0.f, q1 = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+                q0 = fmaf(pair_codeword<CODE>((w >> (16 - 2 * e)) & 0xFFFFu, tab), xq[e], q0);
+                q1 = fmaf(pair_codeword<CODE>((w >> (14 - 2 * e)) & 0xFFFFu, tab), xq[e + 1], q1);
+            }
+            acc = fmaf((a.scale ? a.scale[b] : 1.f) * sc_code, q0 + q1, acc);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) wsum[warp] = acc;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float t = wsum[0];
+            for (int i = 1; i < kPairWarps; ++i) t += wsum[i];
+            a.y[r] = t;
+        }
+        __syncthreads();
+    }
+}
+
+cudaError_t launch_gemv_pair(const GemvArgs& a, int num_sms, cudaStream_t stream, bool mad)
+{
+    const size_t tab = mad ? 0 : ((size_t)1 << 16) * 2;
+    const size_t smem = tab + (size_t)(a.cols + (a.cols / 128) * 4) * 4 + kPairWarps * 4;
+    const void* fn = mad ? reinterpret_cast<const void*>(&gemv_pair_kernel<kCodeMad>)
+                         : reinterpret_cast<const void*>(&gemv_pair_kernel<kCodeF16>);
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int grid = num_sms;  // one CTA of 16 warps per SM
+    if (mad)
+        gemv_pair_kernel<kCodeMad><<<grid, kPairThreads, smem, stream>>>(a);
+    else
+        gemv_pair_kernel<kCodeF16><<<grid, kPairThreads, smem, stream>>>(a);
+    return cudaGetLastError();
+}
 template <int L, int K, int N, int T, int CODE>
 cudaError_t launch_gemv_rows(const GemvArgs& a, int grid, cudaStream_t stream)
 {
@@ -511,7 +775,13 @@ cudaError_t launch_gemv(const GemvArgs& a, int num_sms, cudaStream_t stream)
     long long grid = (a.rows + warps_per_cta - 1) / warps_per_cta;
     if (grid > num_sms) grid = num_sms;
     if (grid < 1) grid = 1;
-    // computed code at T = 256: whole rows per warp, constant per-lane offsets
+    // L = 16, k = 2, T = 256 and 4096-column chunks: two rows per warp item, lanes on
+    // half blocks (16-byte loads of the bits and, for the table, of the codebook)
+    if (a.L == 16 && a.K == 2 && a.T == 256 && a.cols % 4096 == 0 && (code == kCodeMad || code == kCodeF16) &&
+        (reinterpret_cast<uintptr_t>(a.bits) & 15) == 0 &&
+        (code == kCodeMad || (reinterpret_cast<uintptr_t>(a.cb) & 15) == 0) &&
+        (code == kCodeMad ? 0 : 131072) + (size_t)(a.cols + a.cols / 32) * 4 + 64 <= 220 * 1024)
+        return launch_gemv_pair(a, num_sms, stream, code == kCodeMad);
     // T = 256: whole rows per warp, constant per-lane offsets
     const bool rows_ok = xsmem && a.T == 256 && (a.cols / 256) % kMadRowsChunk == 0;
 #define TCQ_GEMV_ROWS(LL, KK, NN, CC) \

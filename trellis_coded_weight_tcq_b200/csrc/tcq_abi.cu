@@ -637,6 +637,81 @@ tcq_status tcq_gemv_vec(const uint32_t* bits, const uint32_t* start_state, const
     return e == cudaSuccess ? TCQ_OK : TCQ_ERR_CUDA;
 }
 
+int tcq_ub8_words_per_block(int V, int m, int T)
+{
+    if (V < 1 || V > TCQ_UB8_MAX_V || m < 0 || m > TCQ_UB8_MAX_M || T < 1 || T % V != 0 ||
+        T / V > TCQ_UB8_MAX_STEPS)
+        return -1;
+    return (T / V * (1 + m) + 31) / 32;
+}
+
+tcq_status tcq_ub8_encode(const float* x, const float* d, const void* codebook, tcq_dtype cb_dtype,
+                          int V, int m, int T, int64_t n_blocks, const uint32_t* fixed_start,
+                          uint32_t* start_state, uint32_t* bits, float* path_cost,
+                          tcq_stream_t stream)
+{
+    if (n_blocks < 0) return TCQ_ERR_INVALID_ARG;
+    if (!valid_dtype(cb_dtype)) return TCQ_ERR_INVALID_ARG;
+    if (cb_dtype == TCQ_MAD) return TCQ_ERR_UNSUPPORTED;  // the union codebook is a table
+    const int W = tcq_ub8_words_per_block(V, m, T);
+    if (W < 0) return TCQ_ERR_UNSUPPORTED;
+    if (n_blocks == 0) return TCQ_OK;
+    if (!x || !codebook_ok(codebook, cb_dtype) || !start_state || !bits || !path_cost)
+        return TCQ_ERR_INVALID_ARG;
+    if (!aligned(x, 4) || (d && !aligned(d, 4)) || (fixed_start && !aligned(fixed_start, 4)) ||
+        !aligned(start_state, 4) || !aligned(bits, 4) || !aligned(path_cost, 4))
+        return TCQ_ERR_INVALID_ARG;
+    if ((unsigned long long)n_blocks > (1ull << 40)) return TCQ_ERR_INVALID_ARG;
+    const int sms = current_sms();
+    if (sms <= 0) return TCQ_ERR_CUDA;
+    Ub8EncodeArgs a;
+    a.x = x;
+    a.d = d;
+    a.cb = codebook;
+    a.cb_f16 = cb_dtype == TCQ_F16 ? 1 : 0;
+    a.V = V;
+    a.m = m;
+    a.T = T;
+    a.W = W;
+    a.n_blocks = n_blocks;
+    a.fixed_start = fixed_start;
+    a.start_state = start_state;
+    a.bits = bits;
+    a.path_cost = path_cost;
+    const cudaError_t e = launch_ub8_encode(a, sms, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TCQ_OK : TCQ_ERR_CUDA;
+}
+
+tcq_status tcq_ub8_decode(const uint32_t* bits, const uint32_t* start_state, const void* codebook,
+                          tcq_dtype cb_dtype, int V, int m, int T, int64_t n_blocks, float* y,
+                          tcq_stream_t stream)
+{
+    if (n_blocks < 0) return TCQ_ERR_INVALID_ARG;
+    if (!valid_dtype(cb_dtype)) return TCQ_ERR_INVALID_ARG;
+    if (cb_dtype == TCQ_MAD) return TCQ_ERR_UNSUPPORTED;
+    const int W = tcq_ub8_words_per_block(V, m, T);
+    if (W < 0) return TCQ_ERR_UNSUPPORTED;
+    if (n_blocks == 0) return TCQ_OK;
+    if (!bits || !start_state || !codebook_ok(codebook, cb_dtype) || !y) return TCQ_ERR_INVALID_ARG;
+    if (!aligned(bits, 4) || !aligned(start_state, 4) || !aligned(y, 4)) return TCQ_ERR_INVALID_ARG;
+    if ((unsigned long long)n_blocks > (1ull << 40)) return TCQ_ERR_INVALID_ARG;
+    const int sms = current_sms();
+    if (sms <= 0) return TCQ_ERR_CUDA;
+    Ub8DecodeArgs a;
+    a.bits = bits;
+    a.start_state = start_state;
+    a.cb = codebook;
+    a.cb_f16 = cb_dtype == TCQ_F16 ? 1 : 0;
+    a.V = V;
+    a.m = m;
+    a.T = T;
+    a.W = W;
+    a.n_blocks = n_blocks;
+    a.y = y;
+    const cudaError_t e = launch_ub8_decode(a, sms, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TCQ_OK : TCQ_ERR_CUDA;
+}
+
 const char* tcq_status_string(tcq_status status)
 {
     switch (status) {

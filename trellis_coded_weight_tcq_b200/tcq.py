@@ -97,6 +97,12 @@ def load_library() -> ctypes.CDLL:
     lib.tcq_bcjr_workspace_bytes.restype = sz
     lib.tcq_bcjr.argtypes = [vp, vp, vp, ci, ci, ci, ci, i64, ctypes.c_float, vp, vp, vp, sz, vp]
     lib.tcq_bcjr.restype = ci
+    lib.tcq_ub8_words_per_block.argtypes = [ci, ci, ci]
+    lib.tcq_ub8_words_per_block.restype = ci
+    lib.tcq_ub8_encode.argtypes = [vp, vp, vp, ci, ci, ci, ci, i64, vp, vp, vp, vp, vp]
+    lib.tcq_ub8_encode.restype = ci
+    lib.tcq_ub8_decode.argtypes = [vp, vp, vp, ci, ci, ci, ci, i64, vp, vp]
+    lib.tcq_ub8_decode.restype = ci
     _lib = lib
     return lib
 
@@ -183,6 +189,21 @@ def tcq_bcjr(x, d, codebook, cb_dtype, L, k, T, n_blocks, tau, y_soft, free_ener
              workspace_bytes, stream) -> int:
     return int(load_library().tcq_bcjr(x, d, codebook, cb_dtype, L, k, T, n_blocks, tau, y_soft,
                                        free_energy, workspace, workspace_bytes, stream))
+
+
+def tcq_ub8_words_per_block(V: int, m: int, T: int) -> int:
+    return int(load_library().tcq_ub8_words_per_block(V, m, T))
+
+
+def tcq_ub8_encode(x, d, codebook, cb_dtype, V, m, T, n_blocks, fixed_start, start_state, bits,
+                   path_cost, stream) -> int:
+    return int(load_library().tcq_ub8_encode(x, d, codebook, cb_dtype, V, m, T, n_blocks,
+                                             fixed_start, start_state, bits, path_cost, stream))
+
+
+def tcq_ub8_decode(bits, start_state, codebook, cb_dtype, V, m, T, n_blocks, y, stream) -> int:
+    return int(load_library().tcq_ub8_decode(bits, start_state, codebook, cb_dtype, V, m, T,
+                                             n_blocks, y, stream))
 
 
 def tcq_status_string(status: int) -> str:
@@ -448,6 +469,58 @@ def decode_vec(bits, start_state, codebook, L: int, k: int, V: int, T: int, out=
         raise ValueError("decode_vec: out must be a contiguous float32 tensor of n_blocks * T")
     _check(tcq_decode_vec(_ptr(bits), _ptr(start_state), _ptr(codebook), cb_dtype_of(codebook), L,
                           k, V, T, n, _ptr(out), _stream_handle(stream)), "tcq_decode_vec")
+    return out
+
+
+def ub8_encode(x, d, codebook, V: int, m: int, fixed_start=None, out=None,
+               stream=None) -> Encoded:
+    """TCQ over the 8-state set-partitioned trellis of every row of ``x`` (fp32
+    CUDA [n_blocks, T], T / V steps of V weights); ``codebook`` holds 4 * 2^m rows
+    of V values (row r in subset r mod 4).  A free start state per block, or the
+    int32 tensor ``fixed_start``."""
+    torch = _torch()
+    if x.dim() != 2 or x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous float32 CUDA tensor [n_blocks, T]")
+    n, T = x.shape
+    if d is not None and (d.shape != x.shape or d.dtype != torch.float32 or not d.is_contiguous()):
+        raise ValueError("d must be None or a contiguous float32 tensor shaped like x")
+    if codebook is MAD or codebook.numel() != (4 << m) * V:
+        raise ValueError("codebook must be a table of 4 * 2^m rows of V entries")
+    W = tcq_ub8_words_per_block(V, m, T)
+    if W < 0:
+        raise TCQError(TCQ_ERR_UNSUPPORTED, "tcq_ub8_words_per_block")
+    if out is None:
+        out = Encoded(torch.empty(n, dtype=torch.int32, device=x.device),
+                      torch.empty((n, W), dtype=torch.int32, device=x.device),
+                      torch.empty(n, dtype=torch.float32, device=x.device))
+    elif out.start_state.numel() < n or out.bits.numel() < n * W or out.path_cost.numel() < n:
+        raise ValueError("ub8_encode: out is smaller than the blocks need")
+    if fixed_start is not None and (fixed_start.numel() < n or fixed_start.dtype != torch.int32
+                                    or not fixed_start.is_cuda):
+        raise ValueError("fixed_start must be an int32 CUDA tensor of n_blocks start states")
+    _check(tcq_ub8_encode(_ptr(x), _ptr(d), _ptr(codebook), cb_dtype_of(codebook), V, m, T, n,
+                          _ptr(fixed_start), _ptr(out.start_state), _ptr(out.bits),
+                          _ptr(out.path_cost), _stream_handle(stream)), "tcq_ub8_encode")
+    return out
+
+
+def ub8_decode(bits, start_state, codebook, V: int, m: int, T: int, out=None, stream=None):
+    """Values [n_blocks, T] of 8-state set-partitioned trellis streams."""
+    torch = _torch()
+    n = start_state.shape[0]
+    W = tcq_ub8_words_per_block(V, m, T)
+    if W < 0:
+        raise TCQError(TCQ_ERR_UNSUPPORTED, "tcq_ub8_words_per_block")
+    if bits.numel() < n * W:
+        raise ValueError("ub8_decode: bits holds fewer than n_blocks * W words")
+    if codebook is MAD or codebook.numel() != (4 << m) * V:
+        raise ValueError("codebook must be a table of 4 * 2^m rows of V entries")
+    if out is None:
+        out = torch.empty((n, T), dtype=torch.float32, device=bits.device)
+    elif out.numel() < n * T or out.dtype != torch.float32 or not out.is_contiguous():
+        raise ValueError("ub8_decode: out must be a contiguous float32 tensor of n_blocks * T")
+    _check(tcq_ub8_decode(_ptr(bits), _ptr(start_state), _ptr(codebook), cb_dtype_of(codebook), V,
+                          m, T, n, _ptr(out), _stream_handle(stream)), "tcq_ub8_decode")
     return out
 
 

@@ -245,3 +245,20 @@ def ldlq_dyadic_exact(L: int, k: int, T: int, rows: int, cols: int, weighted: bo
     cb = rng.integers(-16, 17, 1 << L) / 8.0
     cb = cb.astype(np.float16) if cb_dtype == "f16" else cb.astype(np.float32)
     return LdlqWorkload(f"ldlq_dyadic_L{L}_k{k}_T{T}_{rows}x{cols}", L, k, T, w, u, d, cb)
+
+
+def ub8_gaussian_codebook(V: int, m: int, dtype: str = "f16", seed: int = SEED_CB + 8) -> np.ndarray:
+    """Union codebook of 4 * 2^m rows of V values for the 8-state set-partitioned
+    trellis (row r in subset r mod 4).  V = 1: the N(0,1) quantiles
+    Phi^{-1}((i + 1/2) / N) in increasing order, so that the subsets interleave
+    along the line as in Ungerboeck's partition; V > 1: seeded N(0,1) vectors."""
+    n = 4 << m
+    if V == 1:
+        import torch
+
+        u = (torch.arange(n, dtype=torch.float64) + 0.5) / n
+        cb = torch.special.ndtri(u).numpy()
+    else:
+        cb = np.random.default_rng(seed).standard_normal((n, V))
+    cb = cb.reshape(-1)
+    return cb.astype(np.float16) if dtype == "f16" else cb.astype(np.float32)
