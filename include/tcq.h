@@ -35,8 +35,8 @@
  * Conventions for every entry point:
  *   - All array pointers are DEVICE pointers owned by the caller.  The library
  *     never allocates, never frees and keeps no global state (thread-safe),
- *     with one documented exception: tcq_encode_static_scratch's fixed device
- *     array (see there).
+ *     with two documented exceptions: tcq_encode_static_scratch's fixed device
+ *     array and the device error word read by tcq_device_errors (see there).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
  *     default stream) and never synchronise.  Device-side failures surface on
  *     the stream like any kernel failure.
@@ -385,6 +385,30 @@ tcq_status tcq_ub8_encode(const float* x, const float* d, const void* codebook, 
 tcq_status tcq_ub8_decode(const uint32_t* bits, const uint32_t* start_state, const void* codebook,
                           tcq_dtype cb_dtype, int V, int m, int T, int64_t n_blocks, float* y,
                           tcq_stream_t stream);
+
+/*
+ * Device-side failures that do not fault the GPU.  (The sources have no
+ * counterpart: this is an engineering part of this library.)  Kernels OR a
+ * flag into one error word per device:
+ *   TCQ_DEVERR_WAIT_TIMEOUT  a bounded wait gave up: the tensor-core feedback
+ *                            product of tcq_ldlq stopped issuing work, waited
+ *                            (bounded) for what it had issued, wrote NaN
+ *                            targets for its rows and freed its tensor memory;
+ *                            the affected blocks then carry non-finite costs.
+ *   TCQ_DEVERR_BOUNDS        an index failed its bounds check and the access
+ *                            was skipped (only the TCQ_DEBUG build,
+ *                            libtcq_debug.so, checks indices).
+ * tcq_device_errors synchronises `stream`, returns the current device's flags
+ * in *flags (if not NULL) and clears them: TCQ_OK when none is set,
+ * TCQ_ERR_INTERNAL when any is, TCQ_ERR_CUDA if the stream or the copy failed.
+ * It allocates nothing.  The word is shared by every stream and host thread on
+ * the device (the second piece of device state this library keeps, next to
+ * tcq_encode_static_scratch's array): read it while no other call runs.
+ */
+#define TCQ_DEVERR_WAIT_TIMEOUT 0x1u
+#define TCQ_DEVERR_BOUNDS 0x2u
+
+tcq_status tcq_device_errors(tcq_stream_t stream, uint32_t* flags);
 
 /* Static, human-readable name of a status code. */
 const char* tcq_status_string(tcq_status status);

@@ -220,3 +220,25 @@ def test_set_partitioned_trellis_entry_points_reject_on_the_host(lib):
     assert dec(m=-1) == tcq.TCQ_ERR_UNSUPPORTED
     assert dec(dt=tcq.TCQ_MAD, cb=None) == tcq.TCQ_ERR_UNSUPPORTED
     assert dec(n=-3) == tcq.TCQ_ERR_INVALID_ARG
+
+
+def test_debug_build_exports_every_declared_function(lib):
+    """The bounds-checked build compiles (sm_100a, relocatable device code) and
+    exports the same C ABI; checked in a process of its own, since one process
+    loads only one build of the library."""
+    import os
+    import subprocess
+    import sys
+
+    from trellis_coded_weight_tcq_b200 import build
+
+    path = build.build(debug=True)
+    code = ("import ctypes, sys; sys.path.insert(0, %r); "
+            "from trellis_coded_weight_tcq_b200 import tcq; "
+            "assert tcq.LIB_PATH.endswith('libtcq_debug.so'); lib = tcq.load_library(); "
+            "missing = [n for n in tcq.header_functions() if not hasattr(lib, n)]; "
+            "assert not missing, missing; print('exports ok')" % build.ROOT)
+    r = subprocess.run([sys.executable, "-c", code], env=dict(os.environ, TCQ_LIBRARY="debug"),
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and "exports ok" in r.stdout, r.stderr[-2000:]
+    assert os.path.exists(path)

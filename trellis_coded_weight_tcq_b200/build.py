@@ -1,10 +1,14 @@
 """Build the sm_100a CUDA library ``libtcq.so`` in-tree with nvcc.
 
-    python -m trellis_coded_weight_tcq_b200.build [--verbose]
+    python -m trellis_coded_weight_tcq_b200.build [--verbose] [--debug]
 
 The library links the CUDA runtime statically, so it loads next to PyTorch's
 own runtime without a version clash; device pointers and streams are shared
-through the primary context.
+through the primary context.  ``--debug`` also builds ``libtcq_debug.so``: the
+same sources with TCQ_DEBUG defined (every global-memory index of the encode,
+decode and matrix-vector kernels checked against its buffer, a failure
+recorded in the device error word and the access skipped) and relocatable
+device code, so that one error word serves every kernel file.
 """
 from __future__ import annotations
 
@@ -19,6 +23,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libtcq.so")
+DEBUG_LIB = os.path.join(PKG, "libtcq_debug.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -40,24 +45,28 @@ def _inputs() -> list[str]:
     ]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every .cu under csrc/ into libtcq.so (skipped when up to date)."""
-    if not force and up_to_date():
-        return LIB
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Compile every .cu under csrc/ into libtcq.so, or with ``debug`` into the
+    bounds-checked libtcq_debug.so (skipped when up to date)."""
+    lib = DEBUG_LIB if debug else LIB
+    if not force and up_to_date(lib):
+        return lib
     nvcc = _nvcc()
-    objdir = os.path.join(PKG, "_build")
+    objdir = os.path.join(PKG, "_build_debug" if debug else "_build")
     os.makedirs(objdir, exist_ok=True)
     common = [
         "-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC",
         "-I", os.path.join(ROOT, "include"),
     ]
+    if debug:
+        common += ["-DTCQ_DEBUG", "-rdc=true"]
     if verbose:
         common += ["-Xptxas", "-v"]
     procs, objs = [], []
@@ -76,18 +85,21 @@ def build(force: bool = False, verbose: bool = False) -> str:
             failed.append(src)
     if failed:
         raise RuntimeError(f"nvcc failed on {failed}")
-    tmp = LIB + f".tmp{os.getpid()}"
-    subprocess.check_call([nvcc, *ARCH, "-shared", "-o", tmp, *objs])
-    os.replace(tmp, LIB)
-    return LIB
+    tmp = lib + f".tmp{os.getpid()}"
+    subprocess.check_call([nvcc, *ARCH, "-shared", *(["-rdc=true"] if debug else []), "-o", tmp, *objs])
+    os.replace(tmp, lib)
+    return lib
 
 
 def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--verbose", action="store_true", help="pass -Xptxas -v")
     ap.add_argument("--force", action="store_true")
+    ap.add_argument("--debug", action="store_true", help="also build the bounds-checked libtcq_debug.so")
     args = ap.parse_args()
     print(build(force=args.force or args.verbose, verbose=args.verbose))
+    if args.debug:
+        print(build(force=args.force, verbose=args.verbose, debug=True))
 
 
 if __name__ == "__main__":

@@ -56,6 +56,12 @@ __global__ void __launch_bounds__(kGenericThreads) acs_generic_kernel(EncodeArgs
     float* Mbase = generic_metrics_in_smem(L, K)
                        ? gsm
                        : reinterpret_cast<float*>(slot + generic_bp_bytes(L, K, NS));
+#ifdef TCQ_DEBUG
+    const long long x_n = (a.n_blocks - 1) * a.x_stride + a.T, d_n = (a.n_blocks - 1) * a.d_stride + a.T;
+    const long long o_n = (a.n_blocks - 1) * a.out_stride + 1;
+    const long long ws_n = (long long)gridDim.x * (long long)a.slot_bytes;
+    const long long cb_n = (1LL << L) * V;
+#endif
 
     for (long long b = blockIdx.x; b < a.n_blocks; b += gridDim.x) {
         const float* xb = a.x + b * a.x_stride;
@@ -63,16 +69,17 @@ __global__ void __launch_bounds__(kGenericThreads) acs_generic_kernel(EncodeArgs
         float bestv = __int_as_float(0x7f800000);
         uint32_t bests = 0xffffffffu;
         // a fixed start s_0 leaves only its successors reachable at step 1
-        const uint32_t s0 = a.fixed_start ? (a.fixed_start[b] & (NU - 1u)) : 0xffffffffu;
+        const uint32_t s0 = a.fixed_start && TCQ_IN_BOUNDS(b, a.n_blocks) ? (a.fixed_start[b] & (NU - 1u)) : 0xffffffffu;
         for (int t = 1; t <= NS; ++t) {
             float ca[kMaxV], cx[kMaxV];
 #pragma unroll
             for (int v = 0; v < kMaxV; ++v) {
                 if (v < V) {
                     const int i = (t - 1) * V + v;
-                    const float sd = db ? sqrtf(db[i]) : 1.f;
+                    const bool ok = TCQ_IN_BOUNDS(xb + i - a.x, x_n) && (!db || TCQ_IN_BOUNDS(db + i - a.d, d_n));
+                    const float sd = db && ok ? sqrtf(db[i]) : 1.f;
                     ca[v] = -sd;
-                    cx[v] = sd * xb[i];
+                    cx[v] = ok ? sd * xb[i] : 0.f;
                 }
             }
             const float* Mp = Mbase + ((t - 1) & 1) * NU;
@@ -87,7 +94,8 @@ __global__ void __launch_bounds__(kGenericThreads) acs_generic_kernel(EncodeArgs
 #pragma unroll
                     for (int w = 0; w < kMaxV; ++w) {
                         if (w < V) {
-                            const float e = fmaf(ca[w], load_codeword(a.cb, a.cb_f16, s * V + w), cx[w]);
+                            const float c = TCQ_IN_BOUNDS((long long)s * V + w, cb_n) ? load_codeword(a.cb, a.cb_f16, s * V + w) : 0.f;
+                            const float e = fmaf(ca[w], c, cx[w]);
                             v = fmaf(e, e, v);
                         }
                     }
@@ -98,7 +106,7 @@ __global__ void __launch_bounds__(kGenericThreads) acs_generic_kernel(EncodeArgs
                 }
                 if (t < NS) {
                     Mn[u] = best;
-                    bp[(size_t)(t - 1) * NU + u] = (uint8_t)bh;
+                    if (TCQ_IN_BOUNDS(bp + (size_t)(t - 1) * NU + u - a.ws, ws_n)) bp[(size_t)(t - 1) * NU + u] = (uint8_t)bh;
                 } else {
                     keep_best(best, (bh << LK) | u, bestv, bests);
                 }
@@ -136,6 +144,9 @@ __global__ void __launch_bounds__(kGenericThreads) acs_generic_kernel(EncodeArgs
             for (int t = NS; t >= 1; --t) {
                 for (int w = 0; w < V; ++w) {
                     const int i = (t - 1) * V + w;
+                    if (!TCQ_IN_BOUNDS(xb + i - a.x, x_n) || (db && !TCQ_IN_BOUNDS(db + i - a.d, d_n)) ||
+                        !TCQ_IN_BOUNDS((long long)s * V + w, cb_n))
+                        continue;
                     const float dv = db ? db[i] : 1.f;
                     const double e = (double)xb[i] - (double)load_codeword(a.cb, a.cb_f16, s * V + w);
                     cost += (double)dv * e * e;
@@ -143,13 +154,15 @@ __global__ void __launch_bounds__(kGenericThreads) acs_generic_kernel(EncodeArgs
                 bw.put(t, K, s & (uint32_t)(H - 1));
                 if (t > 1) {
                     const uint32_t u = s >> K;
-                    const uint32_t h = bp[(size_t)(t - 2) * NU + u];
+                    const uint32_t h = TCQ_IN_BOUNDS(bp + (size_t)(t - 2) * NU + u - a.ws, ws_n) ? bp[(size_t)(t - 2) * NU + u] : 0u;
                     s = (h << LK) | u;
                 }
             }
             bw.finish();
-            a.start_state[b * a.out_stride] = s >> K;
-            a.path_cost[b * a.out_stride] = (float)cost;
+            if (TCQ_IN_BOUNDS(b * a.out_stride, o_n)) {
+                a.start_state[b * a.out_stride] = s >> K;
+                a.path_cost[b * a.out_stride] = (float)cost;
+            }
         }
         __syncthreads();
     }

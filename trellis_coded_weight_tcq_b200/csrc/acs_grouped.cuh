@@ -161,7 +161,7 @@ struct Codewords<C, false> {  // fp32
                 for (int j = 0; j < C::H; ++j) {
                     const uint32_t g = (uint32_t)(tid + i * C::NT);
                     const uint32_t s = ((uint32_t)h << C::LK) | (g << C::K) | (uint32_t)j;
-                    w[i][h][j] = load_codeword(cb, f16, s);
+                    w[i][h][j] = TCQ_IN_BOUNDS(s, 1 << C::L) ? load_codeword(cb, f16, s) : 0.f;
                 }
     }
     __device__ __forceinline__ float get(int i, int h, int j) const { return w[i][h][j]; }
@@ -182,7 +182,8 @@ struct Codewords<C, true> {  // binary16 pairs; the input codebook is binary16
                 for (int j = 0; j < C::H; j += 2) {
                     const uint32_t g = (uint32_t)(tid + i * C::NT);
                     const uint32_t s = ((uint32_t)h << C::LK) | (g << C::K) | (uint32_t)j;
-                    w[i][h][j / 2] = (uint32_t)c[s] | ((uint32_t)c[s + 1] << 16);
+                    w[i][h][j / 2] = TCQ_IN_BOUNDS(s + 1, 1 << C::L)
+                                         ? (uint32_t)c[s] | ((uint32_t)c[s + 1] << 16) : 0u;
                 }
     }
     // c - x in one rounding: sm_100's mixed-precision add takes the binary16
@@ -351,6 +352,10 @@ struct Tracer {
     uint32_t s;         // s_tau
     int tau;            // step about to be stored (T .. 1)
     unit_t unit;        // load in flight
+#ifdef TCQ_DEBUG
+    const unsigned char* ws;  // the workspace and its size, for the index checks
+    long long ws_n;
+#endif
 
     __device__ __forceinline__ void start(long long blk, uint32_t sT, const unit_t* p,
                                           uint16_t* pth, int T)
@@ -366,7 +371,8 @@ struct Tracer {
     {
         if (tau > 1) {  // bp_{tau-1}[s_tau >> k] decides s_{tau-1}
             const uint32_t g = s >> (2 * C::K);
-            unit = bp[(size_t)((tau - 2) / C::SPU) * C::NT + (g % C::NT)];
+            const unit_t* p = bp + (size_t)((tau - 2) / C::SPU) * C::NT + (g % C::NT);
+            unit = TCQ_IN_BOUNDS((const unsigned char*)p - ws, ws_n - (long long)sizeof(unit_t) + 1) ? *p : unit_t(0);
         }
     }
 
@@ -374,7 +380,7 @@ struct Tracer {
     // tracer holds the same state, thread 0 of the team stores it
     __device__ __forceinline__ bool retire(bool store)
     {
-        if (store) path[tau - 1] = (uint16_t)s;
+        if (store && TCQ_IN_BOUNDS((const unsigned char*)(path + tau - 1) - ws, ws_n - 1)) path[tau - 1] = (uint16_t)s;
         if (tau == 1) return true;
         const uint32_t u = s >> C::K;
         const uint32_t g = u >> C::K, j = u & (C::H - 1);
@@ -432,10 +438,18 @@ __device__ __forceinline__ void finish_block(const GroupedArgs& a, long long b,
 {
     const int T = a.T;
     double acc = 0.0;
+#ifdef TCQ_DEBUG
+    const long long x_n = (a.n_blocks - 1) * a.x_stride + T, d_n = (a.n_blocks - 1) * a.d_stride + T;
+    const long long o_n = (a.n_blocks - 1) * a.out_stride + 1;
+    const long long ws_n = (long long)gridDim.x * (long long)a.slot_bytes;
+#endif
     if (b >= 0) {
         const float* xb = a.x + b * opaque(a.x_stride);
         const float* db = a.d ? a.d + b * opaque(a.d_stride) : nullptr;
         for (int t = tid; t < T; t += C::NT) {
+            if (!TCQ_IN_BOUNDS(xb + t - a.x, x_n) || !TCQ_IN_BOUNDS((const unsigned char*)(path + t) - a.ws, ws_n - 1) ||
+                (db && !TCQ_IN_BOUNDS(db + t - a.d, d_n)) || !TCQ_IN_BOUNDS(path[t], 1 << C::L))
+                continue;
             const double e = (double)xb[t] - (double)load_codeword(a.cb, a.cb_f16, path[t]);
             acc += (double)(db ? db[t] : 1.f) * e * e;
         }
@@ -448,11 +462,11 @@ __device__ __forceinline__ void finish_block(const GroupedArgs& a, long long b,
                 const uint32_t sym = path[p / C::K] & (C::H - 1);
                 word |= ((sym >> (C::K - 1 - p % C::K)) & 1u) << (31 - i);
             }
-            a.bits[b * opaque(a.out_stride) * a.W + w] = word;
+            if (TCQ_IN_BOUNDS(b * a.out_stride * a.W + w, o_n * a.W)) a.bits[b * opaque(a.out_stride) * a.W + w] = word;
         }
     }
     const double total = team_sum<C>(acc, redd, m, tid);
-    if (b >= 0 && tid == 0) {
+    if (b >= 0 && tid == 0 && TCQ_IN_BOUNDS(b * a.out_stride, o_n)) {
         a.start_state[b * opaque(a.out_stride)] = (uint32_t)path[0] >> C::K;
         a.path_cost[b * opaque(a.out_stride)] = (float)total;
     }
@@ -519,6 +533,12 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB) acs_grouped_kernel(Group
     cw.load(a.cb, a.cb_f16, tid);
     Tracer<C> tr;
     tr.b = -1;
+#ifdef TCQ_DEBUG
+    const long long x_n = (a.n_blocks - 1) * a.x_stride + T, d_n = (a.n_blocks - 1) * a.d_stride + T;
+    const long long ws_n = (long long)gridDim.x * (long long)a.slot_bytes;
+    tr.ws = a.ws;
+    tr.ws_n = ws_n;
+#endif
 
     for (int r = 0; r < R; ++r) {
         const int par = r & 1;
@@ -531,7 +551,8 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB) acs_grouped_kernel(Group
         if constexpr (C::CB16 && WEIGHTED) {
             float dm = 0.f;
             if (valid)
-                for (int q = tid; q < T; q += C::NT) dm = fmaxf(dm, db ? db[q] : 1.f);
+                for (int q = tid; q < T; q += C::NT)
+                    dm = fmaxf(dm, db && TCQ_IN_BOUNDS(db + q - a.d, d_n) ? db[q] : 1.f);
             dfloor = fmaxf(team_max<C>(dm, redv, m) * 0x1p-60f, 1.17549435e-38f);
         }
         unit_t acc = 0;
@@ -558,6 +579,10 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB) acs_grouped_kernel(Group
             if (tc == 0) {
                 if (valid) {
                     for (int q = tid; q < C::TCHUNK && t + q <= T; q += C::NT) {
+                        if (!TCQ_IN_BOUNDS(xb + t - 1 + q - a.x, x_n) ||
+                            (db && !TCQ_IN_BOUNDS(db + t - 1 + q - a.d, d_n)) ||
+                            (db && t - 1 + q > 0 && !TCQ_IN_BOUNDS(db + t - 2 + q - a.d, d_n)))
+                            continue;
                         const float xv = xb[t - 1 + q];
                         const float dv = (WEIGHTED && db) ? db[t - 1 + q] : 1.f;
                         if constexpr (C::CB16) {
@@ -584,9 +609,10 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB) acs_grouped_kernel(Group
                 float* Mn = Mteam + (t & 1) * C::NU;
                 uint32_t planes[C::K];
                 uint32_t s0 = 0xffffffffu;
-                if constexpr (FIRST && FIXED) s0 = a.fixed_start[b] & (uint32_t)(C::NU - 1);
+                if constexpr (FIRST && FIXED)
+                    if (TCQ_IN_BOUNDS(b, a.n_blocks)) s0 = a.fixed_start[b] & (uint32_t)(C::NU - 1);
                 if constexpr (FIRST && LONG)
-                    if (a.fixed_start) s0 = a.fixed_start[b] & (uint32_t)(C::NU - 1);
+                    if (a.fixed_start && TCQ_IN_BOUNDS(b, a.n_blocks)) s0 = a.fixed_start[b] & (uint32_t)(C::NU - 1);
                 acs_step<C, WEIGHTED, FIRST, LAST>(cw, ax.x, ax.y, Mp, Mn, tid, planes, bestv, bests,
                                                    s0);
                 if constexpr (!LAST) {
@@ -594,13 +620,13 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB) acs_grouped_kernel(Group
 #pragma unroll
                     for (int l = 0; l < C::K; ++l) rec |= (unit_t)planes[l] << (l * C::P);
                     if constexpr (C::SPU == 1) {
-                        *bpw = rec;
+                        if (TCQ_IN_BOUNDS((const unsigned char*)bpw - a.ws, ws_n - (long long)sizeof(unit_t) + 1)) *bpw = rec;
                         bpw += C::NT;
                     } else {
                         const int q = (t - 1) % C::SPU;
                         acc |= rec << (q * C::REC_BITS);
                         if (q == C::SPU - 1 || t == T - 1) {
-                            *bpw = acc;
+                            if (TCQ_IN_BOUNDS((const unsigned char*)bpw - a.ws, ws_n - (long long)sizeof(unit_t) + 1)) *bpw = acc;
                             bpw += C::NT;
                             acc = 0;
                         }
@@ -677,7 +703,37 @@ __global__ void __launch_bounds__(C::NTHREADS, C::MINB) acs_grouped_kernel(Group
         if (tracer && valid) tr.start(b, bests, bp, path, T);
     }
     // the last block of each team has no next round to hide behind
-    if (tracer && tr.b >= 0) {
+    if constexpr (C::NT <= 64 && C::UNIT_BITS == 32) {
+        // small teams: the walk's dependent loads would each wait an L2 round
+        // trip, so the team copies its records into its metric buffer (dead
+        // now) a chunk of rows at a time, with coalesced loads, and the walk
+        // reads them there; every team takes the same barriers (T is common)
+        constexpr int CHR = (2 * C::NU) / C::NT;  // record rows per chunk
+        static_assert(CHR >= 1, "a chunk holds at least one row of records");
+        uint32_t* buf = reinterpret_cast<uint32_t*>(Mteam);
+        const int rows = (T - 2 + C::SPU) / C::SPU;  // rows of records of T - 1 steps
+        // the same in every thread of the team (only the tracer lanes hold tr)
+        const bool walking = R > 0 && first + (long long)(R - 1) * stride + m < nb;
+        const uint32_t* bpt = reinterpret_cast<const uint32_t*>(
+            slot + (size_t)(((R - 1) & 1) * C::NTEAM + m) * team_bytes);
+        for (int hi = rows - 1; hi >= 0; hi -= CHR) {
+            const int lo = hi - CHR + 1 > 0 ? hi - CHR + 1 : 0;
+            if (walking)
+                for (int i = tid; i < (hi - lo + 1) * C::NT; i += C::NT)
+                    if (TCQ_IN_BOUNDS((const unsigned char*)(bpt + (size_t)lo * C::NT + i) - a.ws, ws_n - 3))
+                        buf[i] = bpt[(size_t)lo * C::NT + i];
+            if constexpr (C::NTEAM == 1 || C::NT % 32 != 0) __syncthreads(); else named_barrier(1 + m, C::NT);
+            if (tracer && walking) {
+                while (tr.tau > 1 && (tr.tau - 2) / C::SPU >= lo) {
+                    const uint32_t g = tr.s >> (2 * C::K);
+                    tr.unit = buf[((tr.tau - 2) / C::SPU - lo) * C::NT + (g % C::NT)];
+                    tr.retire(tid == 0);
+                }
+            }
+            if constexpr (C::NTEAM == 1 || C::NT % 32 != 0) __syncthreads(); else named_barrier(1 + m, C::NT);
+        }
+        if (tracer && walking) tr.retire(tid == 0);  // stores s_1
+    } else if (tracer && tr.b >= 0) {
         while (true) {
             tr.issue();
             if (tr.retire(tid == 0)) break;

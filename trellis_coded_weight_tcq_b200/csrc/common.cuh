@@ -29,6 +29,31 @@ struct EncodeArgs {
     int V = 1;             // weights per trellis step (kV bits shifted in; codebook [2^L][V])
 };
 
+// Device-side error flags (tcq_device_errors in tcq.h).
+constexpr unsigned int kDevErrWaitTimeout = TCQ_DEVERR_WAIT_TIMEOUT;
+constexpr unsigned int kDevErrBounds = TCQ_DEVERR_BOUNDS;
+
+// Index checks of the TCQ_DEBUG build: TCQ_IN_BOUNDS(i, n) is true when
+// 0 <= i < n and otherwise ORs kDevErrBounds into the device error word; the
+// caller then skips the access.  In the regular build it is the constant true
+// and its arguments are not evaluated, so the kernels compile unchanged.
+#ifdef TCQ_DEBUG
+extern __device__ unsigned int g_tcq_device_errors;
+__device__ __forceinline__ bool dbg_in_bounds(long long i, long long n)
+{
+    if (i >= 0 && i < n) return true;
+    atomicOr(&g_tcq_device_errors, kDevErrBounds);
+    return false;
+}
+#define TCQ_IN_BOUNDS(i, n) ::tcq::dbg_in_bounds((long long)(i), (long long)(n))
+#else
+#define TCQ_IN_BOUNDS(i, n) true
+#endif
+
+// Host: device address of the current device's error word (looked up on every
+// call made outside stream capture), or nullptr.
+unsigned int* device_error_word(cudaStream_t stream);
+
 // A value the compiler must treat as unknown at each use: a volatile move keeps
 // a per-block product such as b * x_stride at its use instead of being hoisted
 // out of a persistent loop, where the extra live registers slowed the 128-register
@@ -70,6 +95,7 @@ struct FeedbackArgs {
     int n;
     float* x;
     long long x_ld;
+    unsigned int* err;  // device error word (a bounded wait that gave up), or nullptr
 };
 
 struct GemvArgs {

@@ -47,6 +47,10 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a)
 
     const int T = a.T, K = a.K, L = a.L, W = a.W;
     const uint32_t mask = (1u << L) - 1u;
+#ifdef TCQ_DEBUG
+    const long long bits_n = ((a.n_blocks - 1) * a.in_stride + 1) * W;
+    const long long st_n = (a.n_blocks - 1) * a.in_stride + 1, y_n = (a.n_blocks - 1) * a.y_stride + T;
+#endif
     const int Q = (T + 3) >> 2;  // quads per block
     const bool qpow2 = (Q & (Q - 1)) == 0;
     const int qshift = __ffs(Q) - 1;
@@ -88,8 +92,11 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a)
             if (b < a.n_blocks) {
                 const uint32_t* wb = a.bits + b * a.in_stride * W;
                 const int wi = p0 >> 5;  // -1 for the first windows
-                const unsigned long long hi = wi < 0 ? a.start_state[b * a.in_stride] : wb[wi];
-                const unsigned long long lo = wi + 1 < W ? wb[wi + 1] : 0ull;
+                const bool ok = wi < 0 ? TCQ_IN_BOUNDS(b * a.in_stride, st_n)
+                                       : TCQ_IN_BOUNDS(b * a.in_stride * W + wi, bits_n);
+                const bool ok1 = wi + 1 >= W || TCQ_IN_BOUNDS(b * a.in_stride * W + wi + 1, bits_n);
+                const unsigned long long hi = !ok ? 0ull : wi < 0 ? a.start_state[b * a.in_stride] : wb[wi];
+                const unsigned long long lo = wi + 1 < W && ok1 ? wb[wi + 1] : 0ull;
                 f.win[u] = (hi << 32) | lo;
             }
         }
@@ -106,11 +113,12 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a)
                 v[e] = lookup((uint32_t)(f.win[u] >> (64 - f.off[u] - e * K - L)) & mask);
             float* yb = a.y + b * a.y_stride;
             if constexpr (VEC) {
-                __stcs(reinterpret_cast<float4*>(yb + 4 * q), make_float4(v[0], v[1], v[2], v[3]));
+                if (TCQ_IN_BOUNDS(b * a.y_stride + 4 * q + 3, y_n))
+                    __stcs(reinterpret_cast<float4*>(yb + 4 * q), make_float4(v[0], v[1], v[2], v[3]));
             } else {
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
-                    if (4 * q + e < T) yb[4 * q + e] = v[e];
+                    if (4 * q + e < T && TCQ_IN_BOUNDS(b * a.y_stride + 4 * q + e, y_n)) yb[4 * q + e] = v[e];
             }
         }
     };
@@ -181,13 +189,20 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_fast_kernel(DecodeArgs 
     }
     const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
     long long b = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+#ifdef TCQ_DEBUG
+    const long long bits_n = ((a.n_blocks - 1) * a.in_stride + 1) * W;
+    const long long st_n = (a.n_blocks - 1) * a.in_stride + 1, y_n = (a.n_blocks - 1) * a.y_stride + T;
+#endif
     uint32_t hi[QPL], lo[QPL];
     auto fetch = [&](long long blk, uint32_t (&h)[QPL], uint32_t (&l)[QPL]) {
         const uint32_t* wb = a.bits + blk * a.in_stride * W;
 #pragma unroll
         for (int r = 0; r < QPL; ++r) {
-            h[r] = wi[r] < 0 ? a.start_state[blk * a.in_stride] : wb[wi[r]];
-            l[r] = wi[r] + 1 < W ? wb[wi[r] + 1] : 0u;
+            const bool ok = wi[r] < 0 ? TCQ_IN_BOUNDS(blk * a.in_stride, st_n)
+                                      : TCQ_IN_BOUNDS(blk * a.in_stride * W + wi[r], bits_n);
+            const bool ok1 = wi[r] + 1 >= W || TCQ_IN_BOUNDS(blk * a.in_stride * W + wi[r] + 1, bits_n);
+            h[r] = !ok ? 0u : wi[r] < 0 ? a.start_state[blk * a.in_stride] : wb[wi[r]];
+            l[r] = wi[r] + 1 < W && ok1 ? wb[wi[r] + 1] : 0u;
         }
     };
     if (b < a.n_blocks) fetch(b, hi, lo);
@@ -202,7 +217,8 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_fast_kernel(DecodeArgs 
             float v[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) v[e] = lookup((w >> (32 - L - e * K)) & MASK);
-            __stcs(reinterpret_cast<float4*>(yb + 4 * (lane + 32 * r)), make_float4(v[0], v[1], v[2], v[3]));
+            if (TCQ_IN_BOUNDS(b * a.y_stride + 4 * (lane + 32 * r) + 3, y_n))
+                __stcs(reinterpret_cast<float4*>(yb + 4 * (lane + 32 * r)), make_float4(v[0], v[1], v[2], v[3]));
         }
 #pragma unroll
         for (int r = 0; r < QPL; ++r) {

@@ -71,6 +71,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(GemvArgs a)
     const int lane = threadIdx.x & 31;
     const long long warp0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+#ifdef TCQ_DEBUG
+    const long long nblk = a.rows * nb;
+#endif
 
     // A warp's work is the sequence of (row, iteration) items of its rows; the
     // next item's window and scale loads are issued before the current item's
@@ -99,7 +102,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(GemvArgs a)
             f.hi[u] = 0u;
             f.lo[u] = 0u;
             f.sc[u] = 0.f;
-            if (g < nq) {
+            if (g < nq && TCQ_IN_BOUNDS(r * nb + j, nblk)) {
                 const uint32_t* wb = rbits + j * W;
                 const int wi = p0 >> 5;  // -1: the start state is stream word -1
                 f.hi[u] = wi < 0 ? rstart[j] : wb[wi];
@@ -159,7 +162,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(GemvArgs a)
         if (itn == 0) {  // row r complete
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-            if (lane == 0) a.y[r] = acc;
+            if (lane == 0 && TCQ_IN_BOUNDS(r, a.rows)) a.y[r] = acc;
             acc = 0.f;
         }
         r = rn;
@@ -215,6 +218,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_fast_kernel(GemvArgs a)
     const int lane = threadIdx.x & 31;
     const long long warp0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+#ifdef TCQ_DEBUG
+    const long long nblk = a.rows * nb;
+#endif
 
     struct Frag {
         uint32_t hi[U], lo[U];
@@ -237,7 +243,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_fast_kernel(GemvArgs a)
             f.hi[u] = 0u;
             f.lo[u] = 0u;
             f.sc[u] = 0.f;
-            if (i < ni) {
+            if (i < ni && TCQ_IN_BOUNDS(r * nb + j, nblk)) {
                 const uint32_t* wb = rbits + j * W;
                 const int wi = p0 >> 5;  // -1: the start state is stream word -1
                 f.hi[u] = wi < 0 ? rstart[j] : wb[wi];
@@ -304,7 +310,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) gemv_fast_kernel(GemvArgs a)
         if (itn == 0) {
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-            if (lane == 0) a.y[r] = acc;
+            if (lane == 0 && TCQ_IN_BOUNDS(r, a.rows)) a.y[r] = acc;
             acc = 0.f;
         }
         r = rn;
@@ -374,6 +380,7 @@ __global__ void __launch_bounds__(kMadRowsThreads, 1) gemv_rows_kernel(GemvArgs 
         const uint32_t* rbits = a.bits + (r * nb + c * CH) * W;
         const uint32_t* rstart = a.start_state + r * nb + c * CH;
         const float* rscale = a.scale ? a.scale + r * nb + c * CH : nullptr;
+        if (!TCQ_IN_BOUNDS(r * nb + c * CH + CH - 1, a.rows * nb)) return;
 #pragma unroll
         for (int b = 0; b < CH; ++b) {
 #pragma unroll
@@ -441,7 +448,7 @@ __global__ void __launch_bounds__(kMadRowsThreads, 1) gemv_rows_kernel(GemvArgs 
     auto finish_row = [&](long long row) {
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (lane == 0) a.y[row] = acc;
+        if (lane == 0 && TCQ_IN_BOUNDS(row, a.rows)) a.y[row] = acc;
         acc = 0.f;
     };
     while (r < a.rows) {  // r and c are the same in every lane of the warp
@@ -548,6 +555,18 @@ __device__ __forceinline__ float pair_codeword(uint32_t s, const __half* tab)
     }
 }
 
+__device__ __forceinline__ unsigned long long pack2(float a, float b)
+{
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+__device__ __forceinline__ void unpack2(unsigned long long v, float& a, float& b)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+
 // sum over the 16 weights of stream word lo of c[s] x, as two chains of 8
 template <int CODE>
 __device__ __forceinline__ void word_dot(uint32_t hi, uint32_t lo, const float* __restrict__ xq,
@@ -555,6 +574,35 @@ __device__ __forceinline__ void word_dot(uint32_t hi, uint32_t lo, const float* 
 {
     uint32_t st[16];
     states16(hi, lo, st);
+    if constexpr (CODE == kCodeMad) {
+        // two weights per instruction for the float part: (n - 255) of both by
+        // one packed subtraction, both products into the pair of chains by one
+        // packed FMA (each half rounds like the scalar operation, so the sums
+        // are those of two scalar chains)
+        const unsigned long long off = pack2(-8388863.0f, -8388863.0f);
+        unsigned long long p = 0ull;
+#pragma unroll
+        for (int e = 0; e < 16; e += 4) {
+            const float4 v = *reinterpret_cast<const float4*>(xq + e);
+#pragma unroll
+            for (int h = 0; h < 4; h += 2) {
+                const uint32_t n0 = __dp4a(st[e + h] * kMadA, 0x01010000u, 0x4B000000u);
+                const uint32_t n1 = __dp4a(st[e + h + 1] * kMadA, 0x01010000u, 0x4B000000u);
+                unsigned long long c2;
+                asm("add.rn.f32x2 %0, %1, %2;" : "=l"(c2) : "l"(pack2(__uint_as_float(n0), __uint_as_float(n1))), "l"(off));
+                const unsigned long long x2 = h == 0 ? pack2(v.x, v.y) : pack2(v.z, v.w);
+                if (e == 0 && h == 0)
+                    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(p) : "l"(c2), "l"(x2));
+                else
+                    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(c2), "l"(x2), "l"(p));
+            }
+        }
+        float p0, p1;
+        unpack2(p, p0, p1);
+        acc0 += p0;
+        acc1 += p1;
+        return;
+    }
     float xv[16];
 #pragma unroll
     for (int e = 0; e < 16; e += 4) {
@@ -597,8 +645,6 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemv_pair_kernel(GemvArgs a)
         const float4 v = reinterpret_cast<const float4*>(a.x)[i];
         *reinterpret_cast<float4*>(xs + xpad(4 * i)) = v;
     }
-    if constexpr (CODE != kCodeMad) asm volatile("cp.async.wait_all;" ::: "memory");
-    __syncthreads();
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int jl = lane >> 1, h = lane & 1;  // block of the 16-block chunk, half
@@ -620,6 +666,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemv_pair_kernel(GemvArgs a)
 #pragma unroll
         for (int i = 0; i < kPairRows; ++i) {
             const long long b = (r0 + i) * nb + 16LL * c + jl;
+            if (!TCQ_IN_BOUNDS(b, a.rows * nb)) continue;
             const uint4* wp = reinterpret_cast<const uint4*>(a.bits + b * W + 8 * h);
             it.w[i][0] = wp[0];
             it.w[i][1] = wp[1];
@@ -644,12 +691,15 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemv_pair_kernel(GemvArgs a)
 #pragma unroll
         for (int i = 0; i < kPairRows; ++i) row[i] = fmaf(it.sc[i], a0[i] + a1[i], row[i]);
     };
+    // items (pair, chunk) of this warp in order; two buffers, no copies.  The
+    // first item's loads are in flight while the table and x are staged.
+    const long long n_items = rounds * nch;
+    auto item_row = [&](long long t) { return (gw + (t / nch) * nw) * kPairRows; };
+    Item A, B;
+    if (rounds > 0) fetch(A, item_row(0), 0);
+    if constexpr (CODE != kCodeMad) asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
     if (rounds > 0) {
-        // items (pair, chunk) of this warp in order; two buffers, no copies
-        const long long n_items = rounds * nch;
-        auto item_row = [&](long long t) { return (gw + (t / nch) * nw) * kPairRows; };
-        Item A, B;
-        fetch(A, item_row(0), 0);
         float row[kPairRows];
 #pragma unroll
         for (int i = 0; i < kPairRows; ++i) row[i] = 0.f;
@@ -660,7 +710,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemv_pair_kernel(GemvArgs a)
                 float v = row[i];
 #pragma unroll
                 for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                if (lane == 0) a.y[r0 + i] = v;
+                if (lane == 0 && TCQ_IN_BOUNDS(r0 + i, a.rows)) a.y[r0 + i] = v;
                 row[i] = 0.f;
             }
         };
@@ -684,6 +734,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemv_pair_kernel(GemvArgs a)
         float acc = 0.f;
         for (long long j = warp; j < nb; j += kPairWarps) {
             const long long b = r * nb + j;
+            if (!TCQ_IN_BOUNDS(b, a.rows * nb)) continue;
             const uint32_t* wb = a.bits + b * W;
             const uint32_t hi = wi < 0 ? a.start_state[b] : wb[wi];
             const uint32_t lo = wi + 1 < W ? wb[wi + 1] : 0u;  // lane 31 ends on the last word
@@ -704,7 +755,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemv_pair_kernel(GemvArgs a)
         if (threadIdx.x == 0) {
             float t = wsum[0];
             for (int i = 1; i < kPairWarps; ++i) t += wsum[i];
-            a.y[r] = t;
+            if (TCQ_IN_BOUNDS(r, a.rows)) a.y[r] = t;
         }
         __syncthreads();
     }

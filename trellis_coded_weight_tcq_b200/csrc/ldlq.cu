@@ -149,9 +149,12 @@ __global__ void __launch_bounds__(kThreads) feedback_kernel(FeedbackArgs a)
 // offset).  Each K step of 8 is one 128 x 256 x 8 MMA per product, issued by
 // one thread; tcgen05.commit on the stage's mbarrier tells the loaders when
 // the stage may be overwritten, so the next tile's loads overlap the MMAs.
-// Every wait is bounded: after kTcSpinLimit polls the CTA gives up, writes NaN
-// targets (which the encoder then reports as non-finite costs) and frees its
-// tensor memory.
+// Every wait is bounded, and the CTA decides together (__syncthreads_or) on
+// the outcome: after kTcSpinLimit polls it stops loading stages and issuing
+// MMAs, waits (bounded again) for the last commit it issued, skips the tensor
+// memory read, writes NaN targets (which the encoder then reports as non-finite
+// costs), frees its tensor memory and ORs TCQ_DEVERR_WAIT_TIMEOUT into the
+// device error word (tcq_device_errors).
 // ---------------------------------------------------------------------------
 constexpr int TC_M = 128, TC_N = 256, TC_K = 32;
 constexpr int kTcThreads = 256;
@@ -162,7 +165,6 @@ struct __align__(1024) TcSmem {
     float b[2][2][TC_N * TC_K];
     unsigned long long mbar[2];
     uint32_t tmem_base;
-    int failed;
 };
 
 // element offset of (row, k) in a K-major core-matrix tile of TC_K columns
@@ -219,7 +221,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) feedback_tc_kernel(FeedbackArgs
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&S.mbar[0])) : "memory");
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&S.mbar[1])) : "memory");
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        S.failed = 0;
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -258,10 +259,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) feedback_tc_kernel(FeedbackArgs
     };
     if (iters > 0) prefetch(0);
 
+    bool failed = false;
+    int last = -1;  // the last iteration whose MMAs were issued and committed
     for (int it = 0; it < iters; ++it) {
         const int st = it & 1;
-        // the MMAs that last read this stage (iteration it - 2) must be done
-        if (it >= 2 && !mbar_wait(smem_u32(&S.mbar[st]), (uint32_t)(((it >> 1) - 1) & 1))) S.failed = 1;
+        // the MMAs that last read this stage (iteration it - 2) must be done; a
+        // wait that gives up in any thread stops the whole CTA before the stage
+        // is overwritten
+        if (it >= 2) {
+            const bool ok = mbar_wait(smem_u32(&S.mbar[st]), (uint32_t)(((it >> 1) - 1) & 1));
+            if (__syncthreads_or(!ok)) {
+                failed = true;
+                break;
+            }
+        }
         // error tile: lanes take 8 rows x 4 column quads (conflict-free 16-byte stores)
 #pragma unroll
         for (int i = 0; i < AQ; ++i) {
@@ -311,16 +322,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) feedback_tc_kernel(FeedbackArgs
             asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                          ::"r"(smem_u32(&S.mbar[st])) : "memory");
         }
+        last = it;
         if (it + 1 < iters) prefetch((long long)(it + 1) * TC_K);
     }
-    // all MMAs done: the last commit covers every earlier one
-    if (iters > 0) {
-        const int last = iters - 1;
-        if (!mbar_wait(smem_u32(&S.mbar[last & 1]), (uint32_t)((last >> 1) & 1))) S.failed = 1;
+    // all MMAs done: the last commit covers every earlier one (also after a
+    // give-up, so that nothing issued is still running when tensor memory is read
+    // or freed)
+    if (last >= 0) {
+        const bool ok = mbar_wait(smem_u32(&S.mbar[last & 1]), (uint32_t)((last >> 1) & 1));
+        if (__syncthreads_or(!ok)) failed = true;
     }
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     __syncthreads();
-    const bool failed = S.failed != 0;
+    if (failed && tid == 0 && a.err) atomicOr(a.err, kDevErrWaitTimeout);
 
     // epilogue: warp w reads TMEM lanes 32 (w & 3) .. + 31 (its rows), columns
     // 128 (w >> 2) .. + 127, and writes X = W + feedback
@@ -329,8 +343,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) feedback_tc_kernel(FeedbackArgs
 #pragma unroll 1
     for (int j = 0; j < 4; ++j) {
         const int c = 128 * (warp >> 2) + 32 * j;
-        uint32_t v[32];
+        uint32_t v[32] = {};
         const uint32_t taddr = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)c;
+        if (!failed) {  // the same in every thread: tcgen05.ld is warp-collective
         asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
                      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
                      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
@@ -342,6 +357,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) feedback_tc_kernel(FeedbackArgs
                        "=r"(v[30]), "=r"(v[31])
                      : "r"(taddr));
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        }
         if (r < a.rows) {
             const float* wr = a.w + r * a.cols + a.c0 + c;
             float* xr = a.x + r * a.x_ld + c;

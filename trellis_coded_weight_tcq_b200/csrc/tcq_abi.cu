@@ -374,6 +374,7 @@ tcq_status tcq_ldlq(const float* w, const float* u, const float* d, const void* 
     // else the front of the workspace
     float* xbuf = x ? x : reinterpret_cast<float*>(ws);
     const long long x_ld = x ? cols : T;
+    unsigned int* err = device_error_word(st);  // where a feedback give-up is reported
 
     for (int64_t j = 0; j < nb; ++j) {
         const long long c0 = j * (long long)T;
@@ -387,6 +388,7 @@ tcq_status tcq_ldlq(const float* w, const float* u, const float* d, const void* 
         f.n = T;
         f.x = x ? xbuf + c0 : xbuf;
         f.x_ld = x_ld;
+        f.err = err;
         if (launch_feedback(f, st) != cudaSuccess) return TCQ_ERR_CUDA;
 
         EncodeArgs a;

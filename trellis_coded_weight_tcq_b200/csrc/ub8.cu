@@ -96,9 +96,10 @@ __global__ void __launch_bounds__(kUb8Warps * 32) ub8_encode_kernel(Ub8EncodeArg
                 const int t = t0 + 32 * u < S ? t0 + 32 * u : t0;  // a spare lane repeats a valid step
 #pragma unroll
                 for (int v = 0; v < V; ++v) {
-                    const float dv = db ? db[t * V + v] : 1.f;
+                    const bool ok = TCQ_IN_BOUNDS(b * a.T + t * V + v, a.n_blocks * a.T);
+                    const float dv = db && ok ? db[t * V + v] : 1.f;
                     sd[u][v] = sqrtf(dv);
-                    xs[u][v] = sd[u][v] * xb[t * V + v];
+                    xs[u][v] = ok ? sd[u][v] * xb[t * V + v] : 0.f;
                 }
             }
             float best[kUb8Unroll][4];
@@ -154,7 +155,8 @@ __global__ void __launch_bounds__(kUb8Warps * 32) ub8_encode_kernel(Ub8EncodeArg
         const int ja = 2 * q2 + r2;             // its subset (z = q2, p = r2)
         const int jb = 2 * (q2 ^ 1) + r2;       // the subset from sa + 1 (z = q2 ^ 1)
         float M = 0.f;
-        if (a.fixed_start) M = (sg == (int)(a.fixed_start[b] & 7u)) ? 0.f : __int_as_float(0x7f800000);
+        if (a.fixed_start && TCQ_IN_BOUNDS(b, a.n_blocks))
+            M = (sg == (int)(a.fixed_start[b] & 7u)) ? 0.f : __int_as_float(0x7f800000);
         for (int t = 0; t < S; ++t) {
             const float ma = __shfl_sync(0xffffffffu, M, sa);
             const float mb = __shfl_sync(0xffffffffu, M, sa + 1);
@@ -195,7 +197,7 @@ __global__ void __launch_bounds__(kUb8Warps * 32) ub8_encode_kernel(Ub8EncodeArg
                 ROW[t] = (uint16_t)(4 * i + j);
                 s = prev;
             }
-            a.start_state[b] = (uint32_t)s;
+            if (TCQ_IN_BOUNDS(b, a.n_blocks)) a.start_state[b] = (uint32_t)s;
         }
         __syncwarp();
 
@@ -213,7 +215,7 @@ __global__ void __launch_bounds__(kUb8Warps * 32) ub8_encode_kernel(Ub8EncodeArg
                 word |= bits << (32 * w + 32 - p - take);
                 p += take;
             }
-            wb[w] = word;
+            if (TCQ_IN_BOUNDS(b * a.W + w, a.n_blocks * a.W)) wb[w] = word;
         }
         // the path's cost, summed in fp64
         double acc = 0.0;
@@ -221,13 +223,14 @@ __global__ void __launch_bounds__(kUb8Warps * 32) ub8_encode_kernel(Ub8EncodeArg
             const float* row = cbs + (size_t)ROW[t] * V;
 #pragma unroll
             for (int v = 0; v < V; ++v) {
+                if (!TCQ_IN_BOUNDS(b * a.T + t * V + v, a.n_blocks * a.T)) continue;
                 const double e = (double)xb[t * V + v] - (double)row[v];
                 acc += (double)(db ? db[t * V + v] : 1.f) * e * e;
             }
         }
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (lane == 0) a.path_cost[b] = (float)acc;
+        if (lane == 0 && TCQ_IN_BOUNDS(b, a.n_blocks)) a.path_cost[b] = (float)acc;
         __syncwarp();  // the warp's arrays are reused by its next block
     }
 }
@@ -261,11 +264,12 @@ __global__ void __launch_bounds__(kUb8DecWarps * 32) ub8_decode_kernel(Ub8Decode
             uint32_t* Pl = P + lane * PW;
             if (b < a.n_blocks) {
                 const uint32_t* wb = a.bits + b * a.W;
-                int s = (int)(a.start_state[b] & 7u);
+                int s = TCQ_IN_BOUNDS(b, a.n_blocks) ? (int)(a.start_state[b] & 7u) : 0;
                 uint32_t acc = 0;
                 for (int t = 0; t < S; ++t) {
                     const int pos = t * K;  // the branch bit is the symbol's first bit
-                    const int z = (int)((wb[pos >> 5] >> (31 - (pos & 31))) & 1u);
+                    const int z = TCQ_IN_BOUNDS(b * a.W + (pos >> 5), a.n_blocks * a.W)
+                                      ? (int)((wb[pos >> 5] >> (31 - (pos & 31))) & 1u) : 0;
                     acc |= (uint32_t)((s >> 2) & 1) << (t & 31);
                     if ((t & 31) == 31) {
                         Pl[t >> 5] = acc;
@@ -287,14 +291,17 @@ __global__ void __launch_bounds__(kUb8DecWarps * 32) ub8_decode_kernel(Ub8Decode
                 const int pos = t * K;
                 const int w0 = pos >> 5, off = pos & 31;
                 // K <= 9 bits: at most two words
-                const uint32_t hi = wb[w0];
-                const uint32_t lo = (off + K > 32) ? wb[w0 + 1] : 0u;
+                const bool ok = TCQ_IN_BOUNDS(b * a.W + w0, a.n_blocks * a.W) &&
+                                (off + K <= 32 || TCQ_IN_BOUNDS(b * a.W + w0 + 1, a.n_blocks * a.W));
+                const uint32_t hi = ok ? wb[w0] : 0u;
+                const uint32_t lo = (ok && off + K > 32) ? wb[w0 + 1] : 0u;
                 const uint32_t sym = (__funnelshift_l(lo, hi, off) >> (32 - K));
                 const int z = (int)(sym >> a.m);
                 const int p = (int)((P[q * PW + (t >> 5)] >> (t & 31)) & 1u);
                 const float* row = cbs + (size_t)(4 * (sym & imask) + 2 * z + p) * V;
 #pragma unroll
-                for (int v = 0; v < V; ++v) yb[t * V + v] = row[v];
+                for (int v = 0; v < V; ++v)
+                    if (TCQ_IN_BOUNDS(b * a.T + t * V + v, a.n_blocks * a.T)) yb[t * V + v] = row[v];
             }
         }
         __syncwarp();

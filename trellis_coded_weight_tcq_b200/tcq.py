@@ -16,7 +16,10 @@ import re
 from dataclasses import dataclass
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libtcq.so")
+# TCQ_LIBRARY=debug selects the bounds-checked build (libtcq_debug.so, see
+# build.py); load only one of the two builds in a process.
+LIB_PATH = os.path.join(_PKG, "libtcq_debug.so" if os.environ.get("TCQ_LIBRARY") == "debug"
+                        else "libtcq.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "tcq.h")
 
 TCQ_OK = 0
@@ -103,6 +106,8 @@ def load_library() -> ctypes.CDLL:
     lib.tcq_ub8_encode.restype = ci
     lib.tcq_ub8_decode.argtypes = [vp, vp, vp, ci, ci, ci, ci, i64, vp, vp]
     lib.tcq_ub8_decode.restype = ci
+    lib.tcq_device_errors.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
+    lib.tcq_device_errors.restype = ci
     _lib = lib
     return lib
 
@@ -204,6 +209,23 @@ def tcq_ub8_encode(x, d, codebook, cb_dtype, V, m, T, n_blocks, fixed_start, sta
 def tcq_ub8_decode(bits, start_state, codebook, cb_dtype, V, m, T, n_blocks, y, stream) -> int:
     return int(load_library().tcq_ub8_decode(bits, start_state, codebook, cb_dtype, V, m, T,
                                              n_blocks, y, stream))
+
+
+TCQ_DEVERR_WAIT_TIMEOUT = 0x1
+TCQ_DEVERR_BOUNDS = 0x2
+
+
+def tcq_device_errors(stream, flags) -> int:
+    return int(load_library().tcq_device_errors(stream, flags))
+
+
+def device_errors(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error flags."""
+    flags = ctypes.c_uint32(0)
+    st = tcq_device_errors(_stream_handle(stream), ctypes.byref(flags))
+    if st not in (TCQ_OK, TCQ_ERR_INTERNAL):
+        raise TCQError(st, "tcq_device_errors")
+    return int(flags.value)
 
 
 def tcq_status_string(status: int) -> str:
