@@ -26,7 +26,7 @@ def test_debug_build_small_shapes_clean(cuda_device):
     build.build(debug=True)
     env = dict(os.environ, TCQ_LIBRARY="debug")
     r = subprocess.run([sys.executable, os.path.join(ROOT, "tests", "debug_build_run.py")],
-                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=420)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
     assert "DEBUG BUILD OK" in r.stdout
 

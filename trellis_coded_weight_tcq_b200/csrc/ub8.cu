@@ -30,7 +30,7 @@
 //      sums the path's cost in fp64.
 // Nothing needs a workspace: per step the warp keeps 4 metrics, 4 entry
 // indices, one backpointer byte, the symbol and the row in shared memory, which
-// bounds a block to kUb8MaxSteps steps.
+// bounds a block to TCQ_UB8_MAX_STEPS steps.
 //
 // Decoder: the state at every step depends on all earlier branch bits, so a
 // warp first walks 32 blocks at once (one lane per block, only the branch bit
@@ -62,6 +62,28 @@ __device__ __forceinline__ void ub8_stage_codebook(float* dst, const void* cb, i
     for (int i = threadIdx.x; i < n; i += blockDim.x) dst[i] = load_codeword(cb, cb_f16, (uint32_t)i);
 }
 
+// The encoder's copy of the union codebook pairs the subsets (D_0, D_1) and
+// (D_2, D_3) of every entry coordinate by coordinate, so that one packed f32x2
+// operation works on two candidates: value v of row r = 4 i + j sits at
+// ((2 i + (j >> 1)) V + v) 2 + (j & 1).
+__device__ __forceinline__ int ub8_pair_index(int r, int v, int V)
+{
+    return ((2 * (r >> 2) + ((r >> 1) & 1)) * V + v) * 2 + (r & 1);
+}
+
+__device__ __forceinline__ void ub8_stage_pairs(float* dst, const void* cb, int cb_f16, int rows, int V)
+{
+    for (int i = threadIdx.x; i < rows * V; i += blockDim.x)
+        dst[ub8_pair_index(i / V, i % V, V)] = load_codeword(cb, cb_f16, (uint32_t)i);
+}
+
+__device__ __forceinline__ unsigned long long ub8_pack(float a, float b)
+{
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+
 template <int V>
 __global__ void __launch_bounds__(kUb8Warps * 32) ub8_encode_kernel(Ub8EncodeArgs a)
 {
@@ -78,7 +100,7 @@ __global__ void __launch_bounds__(kUb8Warps * 32) ub8_encode_kernel(Ub8EncodeArg
     uint16_t* ROW = SYM + S;                                       // [S]
     uint8_t* BP = reinterpret_cast<uint8_t*>(ROW + S);             // [S]
 
-    ub8_stage_codebook(cbs, a.cb, a.cb_f16, rows * V);
+    ub8_stage_pairs(cbs, a.cb, a.cb_f16, rows, V);
     __syncthreads();
 
     const int n_sub = 1 << a.m;
@@ -90,7 +112,9 @@ __global__ void __launch_bounds__(kUb8Warps * 32) ub8_encode_kernel(Ub8EncodeArg
 
         // ---- 1. nearest entry of every subset, per step
         for (int t0 = lane; t0 < S; t0 += 32 * kUb8Unroll) {
-            float xs[kUb8Unroll][V], sd[kUb8Unroll][V];
+            // per step and coordinate the packed pairs (-sqrt d, -sqrt d) and
+            // (sqrt(d) x, sqrt(d) x): both candidates of a subset pair see them
+            unsigned long long nsd2[kUb8Unroll][V], xs2[kUb8Unroll][V];
 #pragma unroll
             for (int u = 0; u < kUb8Unroll; ++u) {
                 const int t = t0 + 32 * u < S ? t0 + 32 * u : t0;  // a spare lane repeats a valid step
@@ -98,8 +122,10 @@ __global__ void __launch_bounds__(kUb8Warps * 32) ub8_encode_kernel(Ub8EncodeArg
                 for (int v = 0; v < V; ++v) {
                     const bool ok = TCQ_IN_BOUNDS(b * a.T + t * V + v, a.n_blocks * a.T);
                     const float dv = db && ok ? db[t * V + v] : 1.f;
-                    sd[u][v] = sqrtf(dv);
-                    xs[u][v] = ok ? sd[u][v] * xb[t * V + v] : 0.f;
+                    const float sd = sqrtf(dv);
+                    const float xs = ok ? sd * xb[t * V + v] : 0.f;
+                    nsd2[u][v] = ub8_pack(-sd, -sd);
+                    xs2[u][v] = ub8_pack(xs, xs);
                 }
             }
             float best[kUb8Unroll][4];
@@ -112,23 +138,35 @@ __global__ void __launch_bounds__(kUb8Warps * 32) ub8_encode_kernel(Ub8EncodeArg
                     bi[u][j] = 0;
                 }
             for (int i = 0; i < n_sub; ++i) {
-                const float* grp = cbs + (size_t)(4 * i) * V;  // the 4 rows of entry i, one per subset
+                const unsigned long long* grp =
+                    reinterpret_cast<const unsigned long long*>(cbs) + (size_t)(2 * i) * V;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    float c[V];
+                for (int pp = 0; pp < 2; ++pp) {  // subsets (2pp, 2pp + 1)
+                    unsigned long long c2[V];
 #pragma unroll
-                    for (int v = 0; v < V; ++v) c[v] = grp[j * V + v];
+                    for (int v = 0; v < V; ++v) c2[v] = grp[pp * V + v];
 #pragma unroll
                     for (int u = 0; u < kUb8Unroll; ++u) {
-                        float dist = 0.f;
+                        // e = fma(-sqrt d, c, sqrt(d) x), dist = fma(e, e, dist) in each half
+                        unsigned long long dist2 = 0ull;
 #pragma unroll
                         for (int v = 0; v < V; ++v) {
-                            const float e = fmaf(-sd[u][v], c[v], xs[u][v]);
-                            dist = fmaf(e, e, dist);
+                            unsigned long long e2;
+                            asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(e2) : "l"(nsd2[u][v]), "l"(c2[v]), "l"(xs2[u][v]));
+                            if (v == 0)
+                                asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(dist2) : "l"(e2), "l"(e2));
+                            else
+                                asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(dist2) : "l"(e2), "l"(e2), "l"(dist2));
                         }
-                        if (dist < best[u][j]) {
-                            best[u][j] = dist;
-                            bi[u][j] = i;
+                        float d0, d1;
+                        asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(dist2));
+                        if (d0 < best[u][2 * pp]) {
+                            best[u][2 * pp] = d0;
+                            bi[u][2 * pp] = i;
+                        }
+                        if (d1 < best[u][2 * pp + 1]) {
+                            best[u][2 * pp + 1] = d1;
+                            bi[u][2 * pp + 1] = i;
                         }
                     }
                 }
@@ -220,11 +258,11 @@ __global__ void __launch_bounds__(kUb8Warps * 32) ub8_encode_kernel(Ub8EncodeArg
         // the path's cost, summed in fp64
         double acc = 0.0;
         for (int t = lane; t < S; t += 32) {
-            const float* row = cbs + (size_t)ROW[t] * V;
+            const int r = ROW[t];
 #pragma unroll
             for (int v = 0; v < V; ++v) {
                 if (!TCQ_IN_BOUNDS(b * a.T + t * V + v, a.n_blocks * a.T)) continue;
-                const double e = (double)xb[t * V + v] - (double)row[v];
+                const double e = (double)xb[t * V + v] - (double)cbs[ub8_pair_index(r, v, V)];
                 acc += (double)(db ? db[t * V + v] : 1.f) * e * e;
             }
         }
