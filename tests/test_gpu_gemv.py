@@ -7,8 +7,8 @@ Tolerance: each product scale * c * x reaches y through at most
 5-level warp reduction.  The kernel for L = 16, k = 2, T = 256 and 4096-column
 chunks (lanes on half blocks, two rows per item) has at most 23 + cols / 4096:
 8 in a stream word's FMA chain, 8 into a block sum, 1 for the two block sums,
-1 for the scale, one per 4096-column chunk and 5 in the warp reduction (its
-rows left for a last partial round: 4 + 1 + 1 + cols / 4096 + 5 + 16).  So
+1 for the scale, one per 4096-column chunk and 5 in the warp reduction (the
+rows it leaves for a last partial round are summed in the same order).  So
 |y_gpu - y_exact| <= (13 + ceil(cols / 256)) * 2^-24 * sum |scale * c * x|.
 """
 import ctypes
@@ -175,3 +175,27 @@ def test_gemv_misaligned_bits_take_the_general_kernel(cuda_device):
                  torch.from_numpy(x).to(dev))
     torch.cuda.synchronize()
     _check(bits, start, None, cb, L, k, T, rows, cols, x, y.cpu().numpy())
+
+
+def test_gemv_half_block_kernel_rows_bit_identical_across_phases(cuda_device):
+    """Rows with the same blocks give the same bits whether the row falls in the
+    warps' row pairs or among the rows left for the last partial round."""
+    import torch
+
+    L, k, T, nb = 16, 2, 256, 16
+    rows = 4736 + 37  # 148 x 16 warps x 2 rows, then 37 rows for the last round
+    rng = np.random.default_rng(404)
+    bits1, start1 = _rand_stream(rng, nb, k, T)
+    bits = np.tile(bits1, (rows, 1))
+    start = np.tile(start1, rows)
+    cb = rng.standard_normal(1 << L).astype(np.float16)
+    x = rng.standard_normal(nb * T).astype(np.float32)
+    for code in ("f16", "mad"):
+        dev = torch.device("cuda", 0)
+        b = torch.from_numpy(np.ascontiguousarray(bits).view(np.int32)).to(dev)
+        s = torch.from_numpy(np.ascontiguousarray(start).view(np.int32)).to(dev)
+        c = tcq.MAD if code == "mad" else torch.from_numpy(cb).to(dev)
+        y = tcq.gemv(b, s, None, c, L, k, T, rows, nb * T, torch.from_numpy(x).to(dev))
+        torch.cuda.synchronize()
+        y = y.cpu().numpy()
+        assert np.all(y == y[0]), code

@@ -489,16 +489,16 @@ __global__ void __launch_bounds__(kMadRowsThreads, 1) gemv_rows_kernel(GemvArgs 
 //
 // Rows: phase A gives every warp of the grid the same number of row pairs;
 // the rows left over (fewer than two per warp of the grid) are phase B, one row
-// per CTA at a time, each warp taking coding blocks w, w + 16, ... with lanes
-// on 8-weight items, and the CTA summing its 16 warp sums in a fixed order, so
-// that the last round costs a sixteenth of a row instead of a whole row pair.
-// Every sum has a fixed order: the result does not depend on timing.
+// per CTA at a time, its stream words spread over all the CTA's threads (each
+// computes one word's two FMA chains) and then combined by one warp in phase
+// A's order, so that the last round costs a fraction of a row instead of a
+// whole row pair and a row's result is the same bits whichever phase computes
+// it.  Every sum has a fixed order: the result does not depend on timing.
 //
 // Rounding depth of a product (the tolerance tests/test_gpu_gemv.py uses):
-// phase A, 8 in a word's FMA chain, 8 over the words into the block sum, 1 for
-// the two block sums, 1 for the scale, c = cols / 4096 over the chunks, 5 in
-// the warp reduction: 23 + c <= 13 + cols / 256.  Phase B: 4 + 1 + 1 +
-// cols / 4096 + 5 + 16 <= 13 + cols / 256.
+// 8 in a word's FMA chain, 8 over the words into the half-block sum, 1 for the
+// two half-block sums, 1 for the scale, c = cols / 4096 over the chunks, 5 in
+// the warp reduction: 23 + c <= 13 + cols / 256.
 // ---------------------------------------------------------------------------
 constexpr int kPairThreads = 512;
 constexpr int kPairWarps = kPairThreads / 32;
@@ -631,7 +631,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemv_pair_kernel(GemvArgs a)
     constexpr size_t TAB = CODE == kCodeMad ? 0 : ((size_t)1 << 16) * 2;
     const __half* tab = reinterpret_cast<const __half*>(gsm);
     float* xs = reinterpret_cast<float*>(gsm + TAB);
-    float* wsum = xs + xpad((int)a.cols);  // kPairWarps partial sums of phase B
+    float* wsum = xs + xpad((int)a.cols);  // phase B: the (p0, p1) of every word of a row
     // stage the table (16-byte asynchronous copies) and x (padded)
     if constexpr (CODE != kCodeMad) {
         const char* src = reinterpret_cast<const char*>(a.cb);
@@ -725,37 +725,45 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemv_pair_kernel(GemvArgs a)
         }
     }
 
-    // ---- phase B: the remaining rows, one per CTA at a time; warp w takes
-    // blocks w, w + 16, ... of the row, lane l the 8 weights [8l, 8l + 8)
+    // ---- phase B: the remaining rows, one per CTA at a time.  The row's
+    // arithmetic is phase A's exactly, so that a row's result does not depend on
+    // the phase that computes it: every thread takes stream words (the word's two
+    // FMA chains, word_dot from zero), then warp 0, lane = half block, adds the
+    // eight words of its half in order, scales per chunk, and runs the same
+    // five-step butterfly.
     const long long first_b = rounds * nw * kPairRows;
-    const int p0 = 16 * lane - 14;  // stream bit of the item's first window (k = 2, L = 16)
-    const int wi = p0 >> 5, off = p0 & 31;  // word -1 is the start state
     for (long long r = first_b + blockIdx.x; r < a.rows; r += gridDim.x) {
-        float acc = 0.f;
-        for (long long j = warp; j < nb; j += kPairWarps) {
-            const long long b = r * nb + j;
-            if (!TCQ_IN_BOUNDS(b, a.rows * nb)) continue;
-            const uint32_t* wb = a.bits + b * W;
-            const uint32_t hi = wi < 0 ? a.start_state[b] : wb[wi];
-            const uint32_t lo = wi + 1 < W ? wb[wi + 1] : 0u;  // lane 31 ends on the last word
-            const uint32_t w = __funnelshift_l(lo, hi, off);
-            const float* xq = xs + xpad((int)(j * T) + 8 * lane);
-            float q0 = 0.f, q1 = 0.f;
-#pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-                q0 = fmaf(pair_codeword<CODE>((w >> (16 - 2 * e)) & 0xFFFFu, tab), xq[e], q0);
-                q1 = fmaf(pair_codeword<CODE>((w >> (14 - 2 * e)) & 0xFFFFu, tab), xq[e + 1], q1);
+        for (int task = threadIdx.x; task < nch * 256; task += blockDim.x) {
+            const int c = task >> 8, ln = (task >> 3) & 31, q = task & 7;  // chunk, half block (lane), word
+            const int jb = ln >> 1, hb = ln & 1;
+            const long long b = r * nb + 16LL * c + jb;
+            float p0 = 0.f, p1 = 0.f;
+            if (TCQ_IN_BOUNDS(b, a.rows * nb)) {
+                const uint32_t* wb = a.bits + b * W;
+                const uint32_t hi = q > 0 ? wb[8 * hb + q - 1] : hb ? wb[7] : a.start_state[b];
+                word_dot<CODE>(hi, wb[8 * hb + q], xs + xpad(c * 4096 + 128 * ln) + 16 * q, tab, p0, p1);
             }
-            acc = fmaf((a.scale ? a.scale[b] : 1.f) * sc_code, q0 + q1, acc);
+            wsum[2 * task] = p0;
+            wsum[2 * task + 1] = p1;
         }
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (lane == 0) wsum[warp] = acc;
         __syncthreads();
-        if (threadIdx.x == 0) {
-            float t = wsum[0];
-            for (int i = 1; i < kPairWarps; ++i) t += wsum[i];
-            if (TCQ_IN_BOUNDS(r, a.rows)) a.y[r] = t;
+        if (warp == 0) {
+            float v = 0.f;
+            for (int c = 0; c < nch; ++c) {
+                const long long b = r * nb + 16LL * c + jl;
+                float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int task = (c << 8) | (lane << 3) | q;
+                    a0 += wsum[2 * task];
+                    a1 += wsum[2 * task + 1];
+                }
+                const float sc = (a.scale && TCQ_IN_BOUNDS(b, a.rows * nb) ? a.scale[b] : 1.f) * sc_code;
+                v = fmaf(sc, a0 + a1, v);
+            }
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            if (lane == 0 && TCQ_IN_BOUNDS(r, a.rows)) a.y[r] = v;
         }
         __syncthreads();
     }
@@ -764,7 +772,8 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemv_pair_kernel(GemvArgs a)
 cudaError_t launch_gemv_pair(const GemvArgs& a, int num_sms, cudaStream_t stream, bool mad)
 {
     const size_t tab = mad ? 0 : ((size_t)1 << 16) * 2;
-    const size_t smem = tab + (size_t)(a.cols + (a.cols / 128) * 4) * 4 + kPairWarps * 4;
+    // x padded, then phase B's two floats per stream word of a row (cols / 16 words)
+    const size_t smem = tab + (size_t)(a.cols + (a.cols / 128) * 4) * 4 + (size_t)(a.cols / 16) * 2 * 4;
     const void* fn = mad ? reinterpret_cast<const void*>(&gemv_pair_kernel<kCodeMad>)
                          : reinterpret_cast<const void*>(&gemv_pair_kernel<kCodeF16>);
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -831,7 +840,7 @@ cudaError_t launch_gemv(const GemvArgs& a, int num_sms, cudaStream_t stream)
     if (a.L == 16 && a.K == 2 && a.T == 256 && a.cols % 4096 == 0 && (code == kCodeMad || code == kCodeF16) &&
         (reinterpret_cast<uintptr_t>(a.bits) & 15) == 0 &&
         (code == kCodeMad || (reinterpret_cast<uintptr_t>(a.cb) & 15) == 0) &&
-        (code == kCodeMad ? 0 : 131072) + (size_t)(a.cols + a.cols / 32) * 4 + 64 <= 220 * 1024)
+        (code == kCodeMad ? 0 : 131072) + (size_t)(a.cols + a.cols / 32) * 4 + (size_t)(a.cols / 8) * 4 <= 220 * 1024)
         return launch_gemv_pair(a, num_sms, stream, code == kCodeMad);
     // T = 256: whole rows per warp, constant per-lane offsets
     const bool rows_ok = xsmem && a.T == 256 && (a.cols / 256) % kMadRowsChunk == 0;
