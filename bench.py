@@ -193,6 +193,72 @@ def time_workload(name, dev, tcq, workloads, peak_ops, warmup=3, steps=10):
             "kernel": tcq.tcq_encode_path(wl.L, wl.k, tcq.cb_dtype_of(cb))}
 
 
+def run_only(args):
+    """One leg of the hot path on seeded inputs of the workload's shape, for
+    profiling and quick timing (3 warm-ups, median of 10): the matrix-vector
+    product (both codes), the decoder, the 8-state trellis encode, or the
+    error-feedback encode of the first rows of the MLP matrix.  Prints one
+    JSON line; not the benchmark's result line."""
+    import numpy as np
+    import torch
+
+    from trellis_coded_weight_tcq_b200 import tcq, workloads
+
+    tcq.load_library()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    g = torch.Generator(device=dev).manual_seed(5)
+    L, k, T = 16, 2, 256
+
+    def med(fn):
+        for _ in range(3):
+            fn()
+        ev = []
+        for _ in range(10):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            ev.append((a, b))
+        torch.cuda.synchronize()
+        return _median_ms(ev)
+
+    out = {"only": args.only}
+    if args.only in ("gemv", "decode"):
+        rows, cols = 14336, 4096  # the MLP matrix; the kernels do not depend on the bit values
+        n = rows * cols // T
+        bits = torch.randint(-2**31, 2**31 - 1, (n, 16), dtype=torch.int32, device=dev, generator=g)
+        start = torch.randint(0, 1 << 14, (n,), dtype=torch.int32, device=dev, generator=g)
+        cb = torch.from_numpy(workloads.gaussian_sample_codebook_f16(1 << L)).to(dev)
+        if args.only == "gemv":
+            x = torch.randn(cols, device=dev, generator=g)
+            y = torch.empty(rows, device=dev)
+            out["table_ms"] = med(lambda: tcq.gemv(bits, start, None, cb, L, k, T, rows, cols, x, y))
+            out["computed_ms"] = med(lambda: tcq.gemv(bits, start, None, tcq.MAD, L, k, T, rows, cols, x, y))
+        else:
+            y = torch.empty((n, T), device=dev)
+            out["decode_ms"] = med(lambda: tcq.decode(bits, start, cb, L, k, T, y))
+            out["hbm_frac"] = (n * T * 4 + n * 64 + n * 4) / (out["decode_ms"] / 1e3) / 1e9 / peaks_hbm()
+    elif args.only == "ub8":
+        wl = workloads.mlp(0)
+        nb = args.blocks or wl.n_blocks
+        x = torch.from_numpy(np.ascontiguousarray(wl.x[:nb])).to(dev)
+        d = torch.from_numpy(np.ascontiguousarray(wl.d[:nb])).to(dev)
+        cb = torch.from_numpy(workloads.ub8_gaussian_codebook(4, 7, "f16")).to(dev)
+        o = tcq.ub8_encode(x, d, cb, 4, 7)
+        y = tcq.ub8_decode(o.bits, o.start_state, cb, 4, 7, T)
+        out["blocks"] = nb
+        out["encode_ms"] = med(lambda: tcq.ub8_encode(x, d, cb, 4, 7, out=o))
+        out["decode_ms"] = med(lambda: tcq.ub8_decode(o.bits, o.start_state, cb, 4, 7, T, out=y))
+    elif args.only == "ldlq":
+        lw = workloads.ldlq_mlp()
+        r = args.blocks // (lw.cols // lw.T) if args.blocks else lw.rows
+        a = [torch.from_numpy(np.ascontiguousarray(v)).to(dev) for v in (lw.w[:r], lw.u, lw.d, lw.codebook)]
+        out["rows"] = r
+        out["ms"] = med(lambda: tcq.ldlq(*a, lw.L, lw.k, lw.T, keep_targets=False))
+    print(json.dumps(out), flush=True)
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -709,6 +775,9 @@ def main():
     ap.add_argument("--no-ldlq", action="store_true",
                     help="skip the error-feedback encode of the MLP matrix")
     ap.add_argument("--cpu-blocks-per-core", type=int, default=16)
+    ap.add_argument("--only", choices=["gemv", "decode", "ub8", "ldlq"], default=None,
+                    help="run one leg on seeded inputs of the workload's shape and print its "
+                         "timing (profiling); not the benchmark line")
     ap.add_argument("--blocks", type=int, default=0,
                     help="encode only the first N blocks of the workload (a smaller profiling "
                          "case; reported in config.n_blocks)")
@@ -716,7 +785,9 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.impl == "reference":
+    if args.only:
+        run_only(args)
+    elif args.impl == "reference":
         run_reference(args, rank, world)
     else:
         run_ours(args, rank, world, local_rank)

@@ -151,26 +151,46 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a)
 // blocks, and lane l always holds quads l, l + 32, ... of a block, so its
 // window offsets are constants; the four windows of a quad lie in one 32-bit
 // word once it is aligned ((4 - 1) k + L <= 32), so a state is one shift and one
-// mask.  The next block's words are loaded before the current block is written.
+// mask.  The loads decide the speed otherwise (each warp waited on its block's
+// words: 14 long-scoreboard stalls per instruction with one block of
+// look-ahead), so every warp keeps kDecodeRing blocks' words and start states
+// in flight in a shared-memory ring filled by asynchronous 16-byte copies (no
+// registers held): cp.async.wait_group then guarantees the oldest slot has
+// landed.  A table is staged the same way while the first slots load.
+constexpr int kDecodeRing = 8;
+
+template <int W>
+struct DecodeRing {
+    static constexpr int SLOT = W * 4 + 16;  // the block's words, then its start state
+};
+
 template <int L, int K, int T, int MODE>
 __global__ void __launch_bounds__(kDecodeThreads) decode_fast_kernel(DecodeArgs a)
 {
     constexpr int Q = T / 4;    // quads per block
     constexpr int QPL = Q / 32; // quads per lane per block
     constexpr int W = (T * K + 31) / 32;
+    constexpr int D = kDecodeRing;
+    constexpr int SLOT = DecodeRing<W>::SLOT;
     constexpr uint32_t MASK = (1u << L) - 1u;
-    static_assert(Q % 32 == 0 && 3 * K + L <= 32, "shape");
+    static_assert(Q % 32 == 0 && 3 * K + L <= 32 && W % 4 == 0 && W / 4 <= 32, "shape");
     extern __shared__ __align__(16) unsigned char dsm[];
     const int n_entries = 1 << L;
-    if constexpr (MODE == kTableF32) {
+    constexpr size_t TAB = MODE == kTableMad ? 0 : ((size_t)1 << L) * (MODE == kTableF16 ? 2 : 4);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned char* ring = dsm + TAB + (size_t)warp * D * SLOT;
+    const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
+    if constexpr (MODE == kTableF16) {
+        const char* src = reinterpret_cast<const char*>(a.cb);
+        const uint32_t dst = (uint32_t)__cvta_generic_to_shared(dsm);
+        for (int i = threadIdx.x; i < n_entries / 8; i += blockDim.x)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + 16 * i),
+                         "l"(src + 16 * (size_t)i) : "memory");
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    } else if constexpr (MODE == kTableF32) {
         float* tab = reinterpret_cast<float*>(dsm);
         for (int i = threadIdx.x; i < n_entries; i += blockDim.x) tab[i] = load_codeword(a.cb, a.cb_f16, i);
-    } else if constexpr (MODE == kTableF16) {
-        const uint4* s4 = reinterpret_cast<const uint4*>(a.cb);
-        uint4* d4 = reinterpret_cast<uint4*>(dsm);
-        for (int i = threadIdx.x; i < n_entries / 8; i += blockDim.x) d4[i] = s4[i];
     }
-    __syncthreads();
     auto lookup = [&](uint32_t s) -> float {
         if constexpr (MODE == kTableF32)
             return reinterpret_cast<const float*>(dsm)[s];
@@ -179,7 +199,6 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_fast_kernel(DecodeArgs 
         else
             return mad_codeword(s);
     };
-    const int lane = threadIdx.x & 31;
     int wi[QPL], off[QPL];
 #pragma unroll
     for (int r = 0; r < QPL; ++r) {
@@ -188,45 +207,53 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_fast_kernel(DecodeArgs 
         off[r] = p0 & 31;
     }
     const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
-    long long b = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const long long b0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
 #ifdef TCQ_DEBUG
     const long long bits_n = ((a.n_blocks - 1) * a.in_stride + 1) * W;
     const long long st_n = (a.n_blocks - 1) * a.in_stride + 1, y_n = (a.n_blocks - 1) * a.y_stride + T;
 #endif
-    uint32_t hi[QPL], lo[QPL];
-    auto fetch = [&](long long blk, uint32_t (&h)[QPL], uint32_t (&l)[QPL]) {
-        const uint32_t* wb = a.bits + blk * a.in_stride * W;
-#pragma unroll
-        for (int r = 0; r < QPL; ++r) {
-            const bool ok = wi[r] < 0 ? TCQ_IN_BOUNDS(blk * a.in_stride, st_n)
-                                      : TCQ_IN_BOUNDS(blk * a.in_stride * W + wi[r], bits_n);
-            const bool ok1 = wi[r] + 1 >= W || TCQ_IN_BOUNDS(blk * a.in_stride * W + wi[r] + 1, bits_n);
-            h[r] = !ok ? 0u : wi[r] < 0 ? a.start_state[blk * a.in_stride] : wb[wi[r]];
-            l[r] = wi[r] + 1 < W && ok1 ? wb[wi[r] + 1] : 0u;
+    // block blk's words and start state into ring slot sl; every lane commits one
+    // group (possibly empty) per call, so wait_group counts blocks
+    auto prefetch = [&](long long blk, int sl) {
+        if (blk < a.n_blocks) {
+            if (lane < W / 4 && TCQ_IN_BOUNDS(blk * a.in_stride * W + 4 * lane + 3, bits_n))
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ring_s + sl * SLOT + 16 * lane),
+                             "l"(a.bits + blk * a.in_stride * W + 4 * lane) : "memory");
+            else if (lane == 31 && TCQ_IN_BOUNDS(blk * a.in_stride, st_n))
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(ring_s + sl * SLOT + 4 * W),
+                             "l"(a.start_state + blk * a.in_stride) : "memory");
         }
+        asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    if (b < a.n_blocks) fetch(b, hi, lo);
-    while (b < a.n_blocks) {
-        const long long bn = b + nwarps;
-        uint32_t nhi[QPL], nlo[QPL];
-        if (bn < a.n_blocks) fetch(bn, nhi, nlo);
-        float* yb = a.y + b * a.y_stride;
+#pragma unroll
+    for (int d = 0; d < D; ++d) prefetch(b0 + d * nwarps, d);
+    if constexpr (MODE == kTableF16) {
+        // the table's group is older than the ring's: waiting for all but D groups
+        asm volatile("cp.async.wait_group %0;" ::"n"(D) : "memory");
+    }
+    __syncthreads();
+    int sl = 0;
+    for (long long bb = b0; bb < a.n_blocks; bb += nwarps) {
+        asm volatile("cp.async.wait_group %0;" ::"n"(D - 1) : "memory");  // this block's group has landed
+        __syncwarp();
+        const uint32_t* rw = reinterpret_cast<const uint32_t*>(ring + sl * SLOT);
+        float* yb = a.y + bb * a.y_stride;
 #pragma unroll
         for (int r = 0; r < QPL; ++r) {
-            const uint32_t w = __funnelshift_l(lo[r], hi[r], off[r]);
+            const uint32_t hi = wi[r] < 0 ? rw[W] : rw[wi[r]];  // word -1 is the start state
+            const uint32_t lo = wi[r] + 1 < W ? rw[wi[r] + 1] : 0u;
+            const uint32_t w = __funnelshift_l(lo, hi, off[r]);
             float v[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) v[e] = lookup((w >> (32 - L - e * K)) & MASK);
-            if (TCQ_IN_BOUNDS(b * a.y_stride + 4 * (lane + 32 * r) + 3, y_n))
+            if (TCQ_IN_BOUNDS(bb * a.y_stride + 4 * (lane + 32 * r) + 3, y_n))
                 __stcs(reinterpret_cast<float4*>(yb + 4 * (lane + 32 * r)), make_float4(v[0], v[1], v[2], v[3]));
         }
-#pragma unroll
-        for (int r = 0; r < QPL; ++r) {
-            hi[r] = nhi[r];
-            lo[r] = nlo[r];
-        }
-        b = bn;
+        __syncwarp();  // the slot is read: refill it D blocks ahead
+        prefetch(bb + D * nwarps, sl);
+        sl = sl + 1 == D ? 0 : sl + 1;
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
 template <int L, int K, int T, int MODE>
@@ -390,8 +417,12 @@ cudaError_t launch_decode(const DecodeArgs& a, int num_sms, cudaStream_t stream)
         const long long need = (a.n_blocks + kDecodeThreads / 32 - 1) / (kDecodeThreads / 32);
         if (fg > need) fg = need;
         if (fg < 1) fg = 1;
+        const bool cb16_ok = (mode != kTableF16 || (reinterpret_cast<uintptr_t>(a.cb) & 15) == 0) &&
+                             (reinterpret_cast<uintptr_t>(a.bits) & 15) == 0;
+        // the table, then one ring of blocks per warp
+        const size_t ring = (size_t)(kDecodeThreads / 32) * kDecodeRing * (a.K * 256 / 32 * 4 + 16);
 #define TCQ_DECODE_FAST(LL, KK, MM) \
-        if (a.L == LL && a.K == KK && mode == MM) return launch_fast<LL, KK, 256, MM>(a, (int)fg, smem, stream);
+        if (a.L == LL && a.K == KK && mode == MM && cb16_ok) return launch_fast<LL, KK, 256, MM>(a, (int)fg, smem + ring, stream);
         TCQ_DECODE_FAST(16, 2, kTableF16)
         TCQ_DECODE_FAST(16, 2, kTableMad)
         TCQ_DECODE_FAST(16, 3, kTableF16)

@@ -699,40 +699,17 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemv_pair_kernel(GemvArgs a)
     if (rounds > 0) fetch(A, item_row(0), 0);
     if constexpr (CODE != kCodeMad) asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
-    if (rounds > 0) {
-        float row[kPairRows];
-#pragma unroll
-        for (int i = 0; i < kPairRows; ++i) row[i] = 0.f;
-        auto finish = [&](long long t) {  // item t was the last chunk of its pair
-            const long long r0 = item_row(t);
-#pragma unroll
-            for (int i = 0; i < kPairRows; ++i) {
-                float v = row[i];
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                if (lane == 0 && TCQ_IN_BOUNDS(r0 + i, a.rows)) a.y[r0 + i] = v;
-                row[i] = 0.f;
-            }
-        };
-        for (long long t = 0; t < n_items; t += 2) {
-            if (t + 1 < n_items) fetch(B, item_row(t + 1), (int)((t + 1) % nch));
-            consume(A, (int)(t % nch), row);
-            if ((t + 1) % nch == 0) finish(t);
-            if (t + 1 >= n_items) break;
-            if (t + 2 < n_items) fetch(A, item_row(t + 2), (int)((t + 2) % nch));
-            consume(B, (int)((t + 1) % nch), row);
-            if ((t + 2) % nch == 0) finish(t + 1);
-        }
-    }
-
-    // ---- phase B: the remaining rows, one per CTA at a time.  The row's
-    // arithmetic is phase A's exactly, so that a row's result does not depend on
-    // the phase that computes it: every thread takes stream words (the word's two
-    // FMA chains, word_dot from zero), then warp 0, lane = half block, adds the
-    // eight words of its half in order, scales per chunk, and runs the same
-    // five-step butterfly.
+    // ---- phase B, first: the rows phase A leaves, one per CTA at a time (their
+    // loads overlap the staging and phase A's first loads; warp 0's final sums
+    // overlap the other warps' phase A).  The row's arithmetic is phase A's
+    // exactly, so that a row's result does not depend on the phase that
+    // computes it: every thread takes stream words (the word's two FMA chains,
+    // word_dot from zero), then warp 0, lane = half block, adds the eight words
+    // of its half in order, scales per chunk, and runs the same five-step
+    // butterfly.
     const long long first_b = rounds * nw * kPairRows;
     for (long long r = first_b + blockIdx.x; r < a.rows; r += gridDim.x) {
+        if (r != first_b + blockIdx.x) __syncthreads();  // warp 0 has read the previous row's sums
         for (int task = threadIdx.x; task < nch * 256; task += blockDim.x) {
             const int c = task >> 8, ln = (task >> 3) & 31, q = task & 7;  // chunk, half block (lane), word
             const int jb = ln >> 1, hb = ln & 1;
@@ -765,8 +742,35 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemv_pair_kernel(GemvArgs a)
             for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
             if (lane == 0 && TCQ_IN_BOUNDS(r, a.rows)) a.y[r] = v;
         }
-        __syncthreads();
     }
+
+    if (rounds > 0) {
+        float row[kPairRows];
+#pragma unroll
+        for (int i = 0; i < kPairRows; ++i) row[i] = 0.f;
+        auto finish = [&](long long t) {  // item t was the last chunk of its pair
+            const long long r0 = item_row(t);
+#pragma unroll
+            for (int i = 0; i < kPairRows; ++i) {
+                float v = row[i];
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                if (lane == 0 && TCQ_IN_BOUNDS(r0 + i, a.rows)) a.y[r0 + i] = v;
+                row[i] = 0.f;
+            }
+        };
+        for (long long t = 0; t < n_items; t += 2) {
+            if (t + 1 < n_items) fetch(B, item_row(t + 1), (int)((t + 1) % nch));
+            consume(A, (int)(t % nch), row);
+            if ((t + 1) % nch == 0) finish(t);
+            if (t + 1 >= n_items) break;
+            if (t + 2 < n_items) fetch(A, item_row(t + 2), (int)((t + 2) % nch));
+            consume(B, (int)((t + 1) % nch), row);
+            if ((t + 2) % nch == 0) finish(t + 1);
+        }
+    }
+
+
 }
 
 cudaError_t launch_gemv_pair(const GemvArgs& a, int num_sms, cudaStream_t stream, bool mad)
