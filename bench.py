@@ -195,7 +195,8 @@ def time_workload(name, dev, tcq, workloads, peak_ops, warmup=3, steps=10):
 
 def run_only(args):
     """One leg of the hot path on seeded inputs of the workload's shape, for
-    profiling and quick timing (3 warm-ups, median of 10): the matrix-vector
+    profiling and quick timing (--warmup untimed calls, the median of --steps
+    timed ones): the matrix-vector
     product (both codes), the decoder, the 8-state trellis encode, or the
     error-feedback encode of the first rows of the MLP matrix.  Prints one
     JSON line; not the benchmark's result line."""
@@ -211,10 +212,10 @@ def run_only(args):
     L, k, T = 16, 2, 256
 
     def med(fn):
-        for _ in range(3):
+        for _ in range(args.warmup):
             fn()
         ev = []
-        for _ in range(10):
+        for _ in range(max(1, args.steps)):
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
             fn()

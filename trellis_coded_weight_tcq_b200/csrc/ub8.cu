@@ -137,14 +137,25 @@ __global__ void __launch_bounds__(kUb8Warps * 32) ub8_encode_kernel(Ub8EncodeArg
                     best[u][j] = __int_as_float(0x7f800000);
                     bi[u][j] = 0;
                 }
+            // entries two at a time when there are two (m >= 1): half the loop overhead
+#pragma unroll 2
             for (int i = 0; i < n_sub; ++i) {
                 const unsigned long long* grp =
                     reinterpret_cast<const unsigned long long*>(cbs) + (size_t)(2 * i) * V;
 #pragma unroll
                 for (int pp = 0; pp < 2; ++pp) {  // subsets (2pp, 2pp + 1)
                     unsigned long long c2[V];
+                    if constexpr (V % 2 == 0) {  // 16-byte loads: two coordinates' pairs each
 #pragma unroll
-                    for (int v = 0; v < V; ++v) c2[v] = grp[pp * V + v];
+                        for (int v = 0; v < V; v += 2) {
+                            const ulonglong2 q = *reinterpret_cast<const ulonglong2*>(grp + pp * V + v);
+                            c2[v] = q.x;
+                            c2[v + 1] = q.y;
+                        }
+                    } else {
+#pragma unroll
+                        for (int v = 0; v < V; ++v) c2[v] = grp[pp * V + v];
+                    }
 #pragma unroll
                     for (int u = 0; u < kUb8Unroll; ++u) {
                         // e = fma(-sqrt d, c, sqrt(d) x), dist = fma(e, e, dist) in each half
