@@ -158,6 +158,21 @@ def _median_ms(pairs):
     return statistics.median(a.elapsed_time(b) for a, b in pairs)
 
 
+def _hold_gpu(stream=None, ms=5.0):
+    """Keep the GPU busy for about `ms` before a loop of short event-timed calls:
+    the host enqueues every call and event while it waits, and the GPU then runs
+    them back to back, so each event pair times its kernel rather than the
+    host's time per call (longer than a 20 us kernel)."""
+    import torch
+
+    cycles = int(ms * 1e-3 * 2.0e9)
+    if stream is None:
+        torch.cuda._sleep(cycles)
+    else:
+        with torch.cuda.stream(stream):
+            torch.cuda._sleep(cycles)
+
+
 def time_workload(name, dev, tcq, workloads, peak_ops, warmup=3, steps=10):
     """Encode and decode timing of one named workload: `warmup` untimed
     encode + decode passes, then the median of `steps` event-timed passes."""
@@ -173,6 +188,7 @@ def time_workload(name, dev, tcq, workloads, peak_ops, warmup=3, steps=10):
     for _ in range(warmup):
         tcq.encode(x, d, cb, wl.L, wl.k, ws, out)
         tcq.decode(out.bits, out.start_state, cb, wl.L, wl.k, wl.T, y)
+    _hold_gpu()
     enc, dec = [], []
     for _ in range(steps):
         a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
@@ -214,6 +230,7 @@ def run_only(args):
     def med(fn):
         for _ in range(args.warmup):
             fn()
+        _hold_gpu()
         ev = []
         for _ in range(max(1, args.steps)):
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -407,6 +424,7 @@ def run_ours(args, rank, world, local_rank):
         ym = torch.empty(rows_m, device=dev)
         for _ in range(3):
             tcq.gemv(out.bits, out.start_state, scale, cb, L, k, T, rows_m, cols_m, xv, ym)
+        _hold_gpu(stream)
         g_ev = []
         for _ in range(10):
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -427,6 +445,7 @@ def run_ours(args, rank, world, local_rank):
         # each codeword computed in registers
         for _ in range(3):
             tcq.gemv(out.bits, out.start_state, scale, tcq.MAD, L, k, T, rows_m, cols_m, xv, ym)
+        _hold_gpu(stream)
         m_ev = []
         for _ in range(10):
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -604,6 +623,7 @@ def run_ours(args, rank, world, local_rank):
         v_nodes = n * (T // V) * (1 << L)
         # decode of the V = 2 stream: reads k/8 B and writes 4 B per weight
         yv = tcq.decode_vec(vout.bits, vout.start_state, cbv, L, k, V, T)
+        _hold_gpu(stream)
         vd_ev = []
         for _ in range(3):
             a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -627,6 +647,7 @@ def run_ours(args, rank, world, local_rank):
             yg = torch.empty(g_rows, device=dev)
             for _ in range(3):
                 tcq.gemv_vec(vout.bits, vout.start_state, sg, cbv, L, k, V, T, g_rows, g_cols, xg, out=yg)
+            _hold_gpu(stream)
             vg_ev = []
             for _ in range(10):
                 a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

@@ -174,3 +174,28 @@ def test_empty_and_rejected_calls(cuda_device):
         tcq.ub8_encode(torch.zeros((2, 16), device=cuda_device), None, cb[:-1], 1, 3)
     with pytest.raises(tcq.TCQError):  # more than 512 steps
         tcq.ub8_encode(torch.zeros((2, 1024), device=cuda_device), None, cb, 1, 3)
+
+
+def test_decode_into_unaligned_output(cuda_device):
+    """An output that is 4-byte but not 16-byte aligned takes the scalar stores:
+    the same values as an aligned one (and as the oracle)."""
+    import torch
+    from oracle import oracle_ub8_decode
+
+    V, m, T, n = 4, 7, 256, 70
+    rng = np.random.default_rng(61)
+    W = tcq.tcq_ub8_words_per_block(V, m, T)
+    bits = rng.integers(0, 2**32, size=(n, W), dtype=np.uint64).astype(np.uint32)
+    start = rng.integers(0, 8, size=n).astype(np.uint32)
+    cb = workloads.ub8_gaussian_codebook(V, m, "f32")
+    dev = cuda_device
+    b = torch.from_numpy(bits.view(np.int32)).to(dev)
+    s = torch.from_numpy(start.view(np.int32)).to(dev)
+    c = torch.from_numpy(cb).to(dev)
+    buf = torch.full((n * T + 1,), float("nan"), device=dev)
+    y = buf[1:].view(n, T)
+    assert y.data_ptr() % 16 == 4
+    tcq.ub8_decode(b, s, c, V, m, T, out=y)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(y.cpu().numpy(), oracle_ub8_decode(bits, start, cb, V, m, T).astype(np.float32))
+    assert np.isnan(buf[0].item())

@@ -159,10 +159,11 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a)
 // landed.  A table is staged the same way while the first slots load.
 constexpr int kDecodeRing = 8;
 
-template <int W>
-struct DecodeRing {
-    static constexpr int SLOT = W * 4 + 16;  // the block's words, then its start state
-};
+// A slot: three unused words, the start state (word 3), the block's W words
+// (16-byte aligned, from word 4), a zero word (word W + 4, written once), then
+// padding to 16 bytes.  Stream word i (i = -1 the start state) is slot word
+// i + 4, so a window's two words are two plain reads whatever the lane.
+__host__ __device__ constexpr int decode_ring_slot_bytes(int W) { return 16 + W * 4 + 16; }
 
 template <int L, int K, int T, int MODE>
 __global__ void __launch_bounds__(kDecodeThreads) decode_fast_kernel(DecodeArgs a)
@@ -171,7 +172,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_fast_kernel(DecodeArgs 
     constexpr int QPL = Q / 32; // quads per lane per block
     constexpr int W = (T * K + 31) / 32;
     constexpr int D = kDecodeRing;
-    constexpr int SLOT = DecodeRing<W>::SLOT;
+    constexpr int SLOT = decode_ring_slot_bytes(W);
     constexpr uint32_t MASK = (1u << L) - 1u;
     static_assert(Q % 32 == 0 && 3 * K + L <= 32 && W % 4 == 0 && W / 4 <= 32, "shape");
     extern __shared__ __align__(16) unsigned char dsm[];
@@ -217,14 +218,15 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_fast_kernel(DecodeArgs 
     auto prefetch = [&](long long blk, int sl) {
         if (blk < a.n_blocks) {
             if (lane < W / 4 && TCQ_IN_BOUNDS(blk * a.in_stride * W + 4 * lane + 3, bits_n))
-                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ring_s + sl * SLOT + 16 * lane),
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ring_s + sl * SLOT + 16 + 16 * lane),
                              "l"(a.bits + blk * a.in_stride * W + 4 * lane) : "memory");
             else if (lane == 31 && TCQ_IN_BOUNDS(blk * a.in_stride, st_n))
-                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(ring_s + sl * SLOT + 4 * W),
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(ring_s + sl * SLOT + 12),
                              "l"(a.start_state + blk * a.in_stride) : "memory");
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
+    if (lane < D) reinterpret_cast<uint32_t*>(ring + lane * SLOT)[W + 4] = 0u;  // never copied over
 #pragma unroll
     for (int d = 0; d < D; ++d) prefetch(b0 + d * nwarps, d);
     if constexpr (MODE == kTableF16) {
@@ -240,8 +242,8 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_fast_kernel(DecodeArgs 
         float* yb = a.y + bb * a.y_stride;
 #pragma unroll
         for (int r = 0; r < QPL; ++r) {
-            const uint32_t hi = wi[r] < 0 ? rw[W] : rw[wi[r]];  // word -1 is the start state
-            const uint32_t lo = wi[r] + 1 < W ? rw[wi[r] + 1] : 0u;
+            const uint32_t hi = rw[wi[r] + 4];  // wi = -1: the start state
+            const uint32_t lo = rw[wi[r] + 5];  // wi = W - 1: the zero word
             const uint32_t w = __funnelshift_l(lo, hi, off[r]);
             float v[4];
 #pragma unroll
@@ -420,7 +422,7 @@ cudaError_t launch_decode(const DecodeArgs& a, int num_sms, cudaStream_t stream)
         const bool cb16_ok = (mode != kTableF16 || (reinterpret_cast<uintptr_t>(a.cb) & 15) == 0) &&
                              (reinterpret_cast<uintptr_t>(a.bits) & 15) == 0;
         // the table, then one ring of blocks per warp
-        const size_t ring = (size_t)(kDecodeThreads / 32) * kDecodeRing * (a.K * 256 / 32 * 4 + 16);
+        const size_t ring = (size_t)(kDecodeThreads / 32) * kDecodeRing * decode_ring_slot_bytes(a.K * 256 / 32);
 #define TCQ_DECODE_FAST(LL, KK, MM) \
         if (a.L == LL && a.K == KK && mode == MM && cb16_ok) return launch_fast<LL, KK, 256, MM>(a, (int)fg, smem + ring, stream);
         TCQ_DECODE_FAST(16, 2, kTableF16)

@@ -697,6 +697,20 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemv_pair_kernel(GemvArgs a)
     auto item_row = [&](long long t) { return (gw + (t / nch) * nw) * kPairRows; };
     Item A, B;
     if (rounds > 0) fetch(A, item_row(0), 0);
+    // phase B's first row: each thread's first task's two words, loaded before
+    // the staging barrier so that their latency overlaps it
+    const long long first_b = rounds * nw * kPairRows;
+    const long long rb0 = first_b + blockIdx.x;
+    uint32_t pre_hi = 0u, pre_lo = 0u;
+    if (rb0 < a.rows && (int)threadIdx.x < nch * 256) {
+        const int c = threadIdx.x >> 8, ln = (threadIdx.x >> 3) & 31, q = threadIdx.x & 7;
+        const long long b = rb0 * nb + 16LL * c + (ln >> 1);
+        if (TCQ_IN_BOUNDS(b, a.rows * nb)) {
+            const uint32_t* wb = a.bits + b * W;
+            pre_hi = q > 0 ? wb[8 * (ln & 1) + q - 1] : (ln & 1) ? wb[7] : a.start_state[b];
+            pre_lo = wb[8 * (ln & 1) + q];
+        }
+    }
     if constexpr (CODE != kCodeMad) asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
     // ---- phase B, first: the rows phase A leaves, one per CTA at a time (their
@@ -707,9 +721,8 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemv_pair_kernel(GemvArgs a)
     // word_dot from zero), then warp 0, lane = half block, adds the eight words
     // of its half in order, scales per chunk, and runs the same five-step
     // butterfly.
-    const long long first_b = rounds * nw * kPairRows;
-    for (long long r = first_b + blockIdx.x; r < a.rows; r += gridDim.x) {
-        if (r != first_b + blockIdx.x) __syncthreads();  // warp 0 has read the previous row's sums
+    for (long long r = rb0; r < a.rows; r += gridDim.x) {
+        if (r != rb0) __syncthreads();  // warp 0 has read the previous row's sums
         for (int task = threadIdx.x; task < nch * 256; task += blockDim.x) {
             const int c = task >> 8, ln = (task >> 3) & 31, q = task & 7;  // chunk, half block (lane), word
             const int jb = ln >> 1, hb = ln & 1;
@@ -717,8 +730,10 @@ __global__ void __launch_bounds__(kPairThreads, 1) gemv_pair_kernel(GemvArgs a)
             float p0 = 0.f, p1 = 0.f;
             if (TCQ_IN_BOUNDS(b, a.rows * nb)) {
                 const uint32_t* wb = a.bits + b * W;
-                const uint32_t hi = q > 0 ? wb[8 * hb + q - 1] : hb ? wb[7] : a.start_state[b];
-                word_dot<CODE>(hi, wb[8 * hb + q], xs + xpad(c * 4096 + 128 * ln) + 16 * q, tab, p0, p1);
+                const bool pre = r == rb0 && task == (int)threadIdx.x;
+                const uint32_t hi = pre ? pre_hi : q > 0 ? wb[8 * hb + q - 1] : hb ? wb[7] : a.start_state[b];
+                const uint32_t lo = pre ? pre_lo : wb[8 * hb + q];
+                word_dot<CODE>(hi, lo, xs + xpad(c * 4096 + 128 * ln) + 16 * q, tab, p0, p1);
             }
             wsum[2 * task] = p0;
             wsum[2 * task + 1] = p1;

@@ -287,7 +287,14 @@ __global__ void __launch_bounds__(kUb8Warps * 32) ub8_encode_kernel(Ub8EncodeArg
 // ---- decoder
 constexpr int kUb8DecWarps = 8;
 
-template <int V>
+// STAGED: the 32 blocks' stream words (W <= kUb8DecStageWords each) are first
+// copied into shared memory with coalesced loads (the walk's loads would
+// otherwise each wait on memory in turn), rows padded by one word so that the
+// walk's lanes, one per block, hit distinct banks.  VSTORE: rows of V = 2, 4
+// or 8 values leave as 8- or 16-byte stores (the output is aligned for them).
+constexpr int kUb8DecStageWords = 32;
+
+template <int V, bool STAGED, bool VSTORE>
 __global__ void __launch_bounds__(kUb8DecWarps * 32) ub8_decode_kernel(Ub8DecodeArgs a)
 {
     extern __shared__ __align__(16) unsigned char smem[];
@@ -295,9 +302,12 @@ __global__ void __launch_bounds__(kUb8DecWarps * 32) ub8_decode_kernel(Ub8Decode
     float* cbs = reinterpret_cast<float*>(smem);
     const int S = a.T / V;
     const int PW = (S + 31) / 32;  // words of subset-half bits per block
+    const int WP = a.W + 1;        // padded row of staged words
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint32_t* P = reinterpret_cast<uint32_t*>(smem + (((size_t)rows * V * 4 + 15) & ~(size_t)15)) +
                   (size_t)warp * 32 * PW;  // [32 blocks][PW]
+    uint32_t* WB = reinterpret_cast<uint32_t*>(smem + (((size_t)rows * V * 4 + 15) & ~(size_t)15)) +
+                   (size_t)kUb8DecWarps * 32 * PW + (size_t)warp * 32 * WP;  // [32 blocks][W + 1]
     ub8_stage_codebook(cbs, a.cb, a.cb_f16, rows * V);
     __syncthreads();
 
@@ -307,50 +317,76 @@ __global__ void __launch_bounds__(kUb8DecWarps * 32) ub8_decode_kernel(Ub8Decode
     for (long long g = (long long)blockIdx.x * kUb8DecWarps + warp; g < groups;
          g += (long long)gridDim.x * kUb8DecWarps) {
         const long long b0 = g * 32;
+        const int nb = (int)min(32LL, a.n_blocks - b0);
+        if constexpr (STAGED) {
+            // the group's words are contiguous: coalesced loads, eight in flight
+            // per lane, then stores into the padded rows
+            const uint32_t* src = a.bits + b0 * a.W;
+            const int nw = nb * a.W;
+            for (int i0 = 0; i0 < nw; i0 += 8 * 32) {
+                uint32_t r[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int i = i0 + 32 * u + lane;
+                    r[u] = i < nw && TCQ_IN_BOUNDS(b0 * a.W + i, a.n_blocks * a.W) ? src[i] : 0u;
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int i = i0 + 32 * u + lane;
+                    if (i < nw) WB[(i / a.W) * WP + i % a.W] = r[u];
+                }
+            }
+            __syncwarp();
+        }
+        auto word = [&](int q, int w) -> uint32_t {
+            if constexpr (STAGED) return WB[q * WP + w];
+            else return TCQ_IN_BOUNDS((b0 + q) * a.W + w, a.n_blocks * a.W) ? a.bits[(b0 + q) * a.W + w] : 0u;
+        };
         // walk: lane l follows block b0 + l and records p of the state before each step
-        {
+        if (lane < nb) {
             const long long b = b0 + lane;
             uint32_t* Pl = P + lane * PW;
-            if (b < a.n_blocks) {
-                const uint32_t* wb = a.bits + b * a.W;
-                int s = TCQ_IN_BOUNDS(b, a.n_blocks) ? (int)(a.start_state[b] & 7u) : 0;
-                uint32_t acc = 0;
-                for (int t = 0; t < S; ++t) {
-                    const int pos = t * K;  // the branch bit is the symbol's first bit
-                    const int z = TCQ_IN_BOUNDS(b * a.W + (pos >> 5), a.n_blocks * a.W)
-                                      ? (int)((wb[pos >> 5] >> (31 - (pos & 31))) & 1u) : 0;
-                    acc |= (uint32_t)((s >> 2) & 1) << (t & 31);
-                    if ((t & 31) == 31) {
-                        Pl[t >> 5] = acc;
-                        acc = 0;
-                    }
-                    s = ub8_next(s, z);
+            int s = TCQ_IN_BOUNDS(b, a.n_blocks) ? (int)(a.start_state[b] & 7u) : 0;
+            uint32_t acc = 0;
+            for (int t = 0; t < S; ++t) {
+                const int pos = t * K;  // the branch bit is the symbol's first bit
+                const int z = (int)((word(lane, pos >> 5) >> (31 - (pos & 31))) & 1u);
+                acc |= (uint32_t)((s >> 2) & 1) << (t & 31);
+                if ((t & 31) == 31) {
+                    Pl[t >> 5] = acc;
+                    acc = 0;
                 }
-                if (S & 31) Pl[S >> 5] = acc;
+                s = ub8_next(s, z);
             }
+            if (S & 31) Pl[S >> 5] = acc;
         }
         __syncwarp();
         // emit: the whole warp writes one block at a time
-        const int nb = (int)min(32LL, a.n_blocks - b0);
         for (int q = 0; q < nb; ++q) {
             const long long b = b0 + q;
-            const uint32_t* wb = a.bits + b * a.W;
             float* yb = a.y + b * a.T;
             for (int t = lane; t < S; t += 32) {
                 const int pos = t * K;
                 const int w0 = pos >> 5, off = pos & 31;
                 // K <= 9 bits: at most two words
-                const bool ok = TCQ_IN_BOUNDS(b * a.W + w0, a.n_blocks * a.W) &&
-                                (off + K <= 32 || TCQ_IN_BOUNDS(b * a.W + w0 + 1, a.n_blocks * a.W));
-                const uint32_t hi = ok ? wb[w0] : 0u;
-                const uint32_t lo = (ok && off + K > 32) ? wb[w0 + 1] : 0u;
+                const uint32_t hi = word(q, w0);
+                const uint32_t lo = off + K > 32 ? word(q, w0 + 1) : 0u;
                 const uint32_t sym = (__funnelshift_l(lo, hi, off) >> (32 - K));
                 const int z = (int)(sym >> a.m);
                 const int p = (int)((P[q * PW + (t >> 5)] >> (t & 31)) & 1u);
                 const float* row = cbs + (size_t)(4 * (sym & imask) + 2 * z + p) * V;
+                if (!TCQ_IN_BOUNDS(b * a.T + t * V + V - 1, a.n_blocks * a.T)) continue;
+                if constexpr (VSTORE && V == 4) {
+                    *reinterpret_cast<float4*>(yb + t * V) = *reinterpret_cast<const float4*>(row);
+                } else if constexpr (VSTORE && V == 8) {
+                    reinterpret_cast<float4*>(yb + t * V)[0] = reinterpret_cast<const float4*>(row)[0];
+                    reinterpret_cast<float4*>(yb + t * V)[1] = reinterpret_cast<const float4*>(row)[1];
+                } else if constexpr (VSTORE && V == 2) {
+                    *reinterpret_cast<float2*>(yb + t * V) = *reinterpret_cast<const float2*>(row);
+                } else {
 #pragma unroll
-                for (int v = 0; v < V; ++v)
-                    if (TCQ_IN_BOUNDS(b * a.T + t * V + v, a.n_blocks * a.T)) yb[t * V + v] = row[v];
+                    for (int v = 0; v < V; ++v) yb[t * V + v] = row[v];
+                }
             }
         }
         __syncwarp();
@@ -375,23 +411,39 @@ cudaError_t launch_ub8_encode_v(const Ub8EncodeArgs& a, int num_sms, cudaStream_
     return cudaGetLastError();
 }
 
-template <int V>
-cudaError_t launch_ub8_decode_v(const Ub8DecodeArgs& a, int num_sms, cudaStream_t stream)
+template <int V, bool STAGED, bool VSTORE>
+cudaError_t launch_ub8_decode_sv(const Ub8DecodeArgs& a, int num_sms, cudaStream_t stream)
 {
     const size_t smem = ub8_decode_smem_bytes(V, a.m, a.T);
-    cudaError_t e = cudaFuncSetAttribute(ub8_decode_kernel<V>,
+    cudaError_t e = cudaFuncSetAttribute(ub8_decode_kernel<V, STAGED, VSTORE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ub8_decode_kernel<V>, kUb8DecWarps * 32, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ub8_decode_kernel<V, STAGED, VSTORE>,
+                                                      kUb8DecWarps * 32, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const long long groups = (a.n_blocks + 31) / 32;
     const long long need = (groups + kUb8DecWarps - 1) / kUb8DecWarps;
     const long long resident = (long long)num_sms * per_sm;
     const int grid = (int)(need < resident ? need : resident);
-    ub8_decode_kernel<V><<<grid, kUb8DecWarps * 32, smem, stream>>>(a);
+    ub8_decode_kernel<V, STAGED, VSTORE><<<grid, kUb8DecWarps * 32, smem, stream>>>(a);
     return cudaGetLastError();
+}
+
+template <int V>
+cudaError_t launch_ub8_decode_v(const Ub8DecodeArgs& a, int num_sms, cudaStream_t stream)
+{
+    // vector stores when V is 2, 4 or 8 and every row of V values is aligned for them
+    const size_t vb = (V == 2 ? 8 : 16);
+    const bool vst = (V == 2 || V == 4 || V == 8) && (reinterpret_cast<uintptr_t>(a.y) % vb) == 0 &&
+                     ((size_t)a.T * 4) % vb == 0;
+    const bool staged = a.W <= kUb8DecStageWords;
+    if (staged)
+        return vst ? launch_ub8_decode_sv<V, true, true>(a, num_sms, stream)
+                   : launch_ub8_decode_sv<V, true, false>(a, num_sms, stream);
+    return vst ? launch_ub8_decode_sv<V, false, true>(a, num_sms, stream)
+               : launch_ub8_decode_sv<V, false, false>(a, num_sms, stream);
 }
 
 }  // namespace
@@ -407,7 +459,9 @@ size_t ub8_decode_smem_bytes(int V, int m, int T)
 {
     const size_t cb = ((size_t)(4 << m) * V * 4 + 15) & ~(size_t)15;
     const size_t pw = (size_t)((T / V + 31) / 32);
-    return cb + (size_t)kUb8DecWarps * 32 * pw * 4;
+    const size_t W = (size_t)((T / V * (1 + m) + 31) / 32);
+    const size_t staged = W <= (size_t)kUb8DecStageWords ? (size_t)kUb8DecWarps * 32 * (W + 1) * 4 : 0;
+    return cb + (size_t)kUb8DecWarps * 32 * pw * 4 + staged;
 }
 
 cudaError_t launch_ub8_encode(const Ub8EncodeArgs& a, int num_sms, cudaStream_t stream)
