@@ -414,9 +414,11 @@ tcq_status tcq_device_errors(tcq_stream_t stream, uint32_t* flags);
 const char* tcq_status_string(tcq_status status);
 
 /*
- * Static name of the encoder kernel tcq_encode would launch for this shape
- * ("grouped<L,k,...>" for the specialised add-compare-select kernels,
- * "generic" for the runtime-(L,k) kernel), or "unsupported".
+ * Static name of the encoder kernel tcq_encode would launch for this shape with
+ * blocks of at most 1024 steps ("warp<L,k>" for the one-warp-per-block kernel
+ * of small trellises, "grouped<L,k,...>" for the specialised add-compare-select
+ * kernels, "generic" for the runtime-(L,k) kernel), or "unsupported".  Longer
+ * blocks at L = 8, k = 2 take "grouped<8,2,...>".
  */
 const char* tcq_encode_path(int L, int k, tcq_dtype cb_dtype);
 

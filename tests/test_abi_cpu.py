@@ -64,7 +64,8 @@ def test_encode_path_names(lib):
     assert tcq.tcq_encode_path(16, 2, tcq.TCQ_F16).startswith("grouped<16,2")
     assert tcq.tcq_encode_path(16, 3, tcq.TCQ_F16).startswith("grouped<16,3")
     assert tcq.tcq_encode_path(12, 2, tcq.TCQ_F32).startswith("grouped<12,2")
-    assert tcq.tcq_encode_path(8, 2, tcq.TCQ_F32).startswith("grouped<8,2")
+    assert tcq.tcq_encode_path(8, 2, tcq.TCQ_F32) == "warp<8,2>"  # blocks of up to 1024 steps
+    assert tcq.tcq_encode_path(8, 2, tcq.TCQ_F16) == "warp<8,2>"
     assert tcq.tcq_encode_path(16, 2, tcq.TCQ_F32) == "generic"
     assert tcq.tcq_encode_path(3, 2, tcq.TCQ_F16) == "generic"
     assert tcq.tcq_encode_path(17, 2, tcq.TCQ_F32) == "unsupported"

@@ -45,7 +45,9 @@ CASES = [
     (16, 2, 256, 24, "f16", True),    # register-resident encoder
     (16, 3, 256, 12, "f16", True),
     (12, 2, 256, 40, "f32", True),
-    (8, 2, 64, 64, "f32", False),
+    (8, 2, 64, 64, "f32", False),     # one warp per block
+    (8, 2, 1, 40, "f16", True),
+    (8, 2, 1100, 3, "f32", True),     # longer than the warp kernel holds: grouped
     (10, 3, 33, 20, "f32", True),     # runtime-(L,k) encoder
     (16, 2, 1, 9, "f16", True),       # T = 1: only the successors of s_0
     (6, 1, 7, 16, "f32", True),

@@ -117,19 +117,23 @@ def test_gemv_rejections(cuda_device):
     assert call(L=17) == tcq.TCQ_ERR_UNSUPPORTED
 
 
+# 148 CTAs x 16 warps = 2368 warps, three rows per item
 @pytest.mark.parametrize("rows,nb,code", [
-    (5000, 16, "f16"),    # two rows per item for every warp, then one row per CTA
-    (5000, 16, "mad"),
-    (4737, 32, "f16"),    # two 4096-column chunks per row; an odd row left for the last round
-    (4801, 32, "mad"),
-    (9473, 16, "mad"),    # several items per warp, 1 row in the last round
-    (37, 16, "f16"),      # fewer rows than warps: only the per-CTA rows
+    (7204, 16, "f16"),    # one whole round of row groups, then 100 rows, one per CTA
+    (7204, 16, "mad"),
+    (5000, 16, "f16"),    # fewer groups than warps: a partial round, 2 rows of no group
+    (4737, 32, "f16"),    # two 4096-column chunks per row; a partial round
+    (4801, 32, "mad"),    # a partial round and 1 row of no group
+    (9473, 16, "mad"),    # a whole round, a partial round of 789 groups, then 2 rows
+    (14336, 16, "f16"),   # the MLP matrix's rows: two whole rounds, then 128 rows one per CTA
+    (37, 16, "f16"),      # fewer rows than CTAs: only the per-CTA rows
 ])
 @pytest.mark.parametrize("scaled", [False, True])
 def test_gemv_half_block_kernel(rows, nb, code, scaled, cuda_device):
     """L = 16, k = 2, T = 256 with cols a multiple of 4096: the kernel that takes
-    half a coding block per lane and two rows per item, in both of its phases
-    (every warp's share of row pairs, then the rows left, one per CTA)."""
+    half a coding block per lane and three rows per item, in both of its phases
+    (every warp's share of row groups, with the last partial round either kept
+    there or, when it is at most one row per CTA, spread one row per CTA)."""
     import torch
     from oracle import oracle_mad_codebook
 
@@ -179,11 +183,11 @@ def test_gemv_misaligned_bits_take_the_general_kernel(cuda_device):
 
 def test_gemv_half_block_kernel_rows_bit_identical_across_phases(cuda_device):
     """Rows with the same blocks give the same bits whether the row falls in the
-    warps' row pairs or among the rows left for the last partial round."""
+    warps' row groups or among the rows spread one per CTA."""
     import torch
 
     L, k, T, nb = 16, 2, 256, 16
-    rows = 4736 + 37  # 148 x 16 warps x 2 rows, then 37 rows for the last round
+    rows = 7104 + 37  # 148 x 16 warps x 3 rows, then 37 rows, one per CTA
     rng = np.random.default_rng(404)
     bits1, start1 = _rand_stream(rng, nb, k, T)
     bits = np.tile(bits1, (rows, 1))

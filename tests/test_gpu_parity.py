@@ -72,9 +72,11 @@ def test_named_workload_full_size_sampled(name):
 # --------------------------------------------------------------------------
 SHAPES = [
     # (L, k, T, n_blocks, weighted, cb_dtype)
-    (8, 2, 64, 300, False, "f32"),     # grouped, sub-warp teams, ragged team tail
+    (8, 2, 64, 300, False, "f32"),     # one warp per block, ragged last CTA
     (8, 2, 1, 33, True, "f32"),
-    (8, 2, 257, 17, True, "f16"),      # crosses the 256-step staging chunk
+    (8, 2, 257, 17, True, "f16"),
+    (8, 2, 1024, 9, True, "f32"),      # the longest block the warp kernel holds
+    (8, 2, 1025, 9, True, "f32"),      # one step more: the grouped kernel, sub-warp teams
     (12, 2, 256, 700, True, "f32"),    # grouped, several rounds per CTA
     (12, 2, 5, 9, False, "f16"),
     (16, 2, 256, 150, True, "f16"),    # grouped fp16-pair kernel

@@ -224,6 +224,8 @@ struct EncodeKernelInfo {
 
 // nullptr if no specialised grouped kernel exists for (L, k, codebook dtype).
 const EncodeKernelInfo* find_grouped_kernel(int L, int K, int cb_f16);
+// nullptr if no one-warp-per-block kernel exists for (L, k) and blocks of T steps.
+const EncodeKernelInfo* find_warp_kernel(int L, int K, int T);
 const EncodeKernelInfo* generic_kernel_info(int L, int K);
 // nullptr if no compile-time vector-trellis kernel exists for (L, k, V, dtype);
 // its size callbacks take (L, k V, steps per block) like the runtime kernel's.

@@ -55,8 +55,11 @@ tcq_status resolve_table(const void*& cb, tcq_dtype& dt, int L, unsigned char*& 
     return TCQ_OK;
 }
 
-const EncodeKernelInfo* select_kernel(int L, int k, tcq_dtype dt)
+// The encoder for (L, k, T, dtype): the one-warp-per-block kernel for small
+// trellises with blocks it holds, else a grouped kernel, else the generic one.
+const EncodeKernelInfo* select_kernel(int L, int k, int T, tcq_dtype dt)
 {
+    if (const EncodeKernelInfo* w = find_warp_kernel(L, k, T)) return w;
     const EncodeKernelInfo* g = find_grouped_kernel(L, k, table_dtype(dt) == TCQ_F16 ? 1 : 0);
     return g ? g : generic_kernel_info(L, k);
 }
@@ -112,7 +115,7 @@ long long bcjr_grid(int L, int k, long long n_blocks, tcq_dtype dt, int sms)
 tcq_status run_encode(EncodeArgs& a, tcq_dtype cb_dtype, void* workspace, size_t workspace_bytes,
                       cudaStream_t stream)
 {
-    const EncodeKernelInfo* info = select_kernel(a.L, a.K, cb_dtype);
+    const EncodeKernelInfo* info = select_kernel(a.L, a.K, a.T, cb_dtype);
     if (!info) return TCQ_ERR_INTERNAL;
     const size_t slot = info->slot_bytes(a.L, a.K, a.T);
     const int sms = current_sms();
@@ -167,7 +170,7 @@ int tcq_words_per_block(int k, int T)
 size_t tcq_encode_workspace_bytes(int L, int k, int T, int64_t n_blocks, tcq_dtype cb_dtype)
 {
     if (check_shape(L, k, T) != TCQ_OK || n_blocks <= 0 || !valid_dtype(cb_dtype)) return 0;
-    const EncodeKernelInfo* info = select_kernel(L, k, cb_dtype);
+    const EncodeKernelInfo* info = select_kernel(L, k, T, cb_dtype);
     const long long ctas = wanted_ctas(info, L, k, T, n_blocks, current_sms());
     return mad_table_bytes(L, cb_dtype) + (size_t)ctas * info->slot_bytes(L, k, T);
 }
@@ -175,7 +178,7 @@ size_t tcq_encode_workspace_bytes(int L, int k, int T, int64_t n_blocks, tcq_dty
 const char* tcq_encode_path(int L, int k, tcq_dtype cb_dtype)
 {
     if (check_shape(L, k, 1) != TCQ_OK || !valid_dtype(cb_dtype)) return "unsupported";
-    return select_kernel(L, k, cb_dtype)->name;
+    return select_kernel(L, k, 1, cb_dtype)->name;  // blocks of few steps
 }
 
 tcq_status tcq_encode(const float* x, const float* d, const void* codebook, tcq_dtype cb_dtype,
