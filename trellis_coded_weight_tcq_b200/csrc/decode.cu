@@ -324,40 +324,59 @@ __global__ void __launch_bounds__(kVec2DecThreads) decode_vec2_kernel(DecodeArgs
     extern __shared__ __align__(16) uint32_t tab[];  // [kVec2DecSmemStates]
     const uint32_t* cb = reinterpret_cast<const uint32_t*>(a.cb);
     {
-        const uint4* src = reinterpret_cast<const uint4*>(cb);
-        uint4* dst = reinterpret_cast<uint4*>(tab);
-        for (int i = threadIdx.x; i < (int)(kVec2DecSmemStates / 4); i += blockDim.x) dst[i] = __ldg(src + i);
+        // the table by asynchronous 16-byte copies, all in flight at once (a load
+        // and a store per thread and round would wait on each load in turn)
+        const uint32_t dst = (uint32_t)__cvta_generic_to_shared(tab);
+        for (int i = threadIdx.x; i < (int)(kVec2DecSmemStates / 4); i += blockDim.x)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + 16 * i),
+                         "l"(cb + 4 * (size_t)i) : "memory");
+        asm volatile("cp.async.commit_group;" ::: "memory");
     }
-    __syncthreads();
     const int NS = a.T >> 1;
     const int chunks = (NS + 127) >> 7;
     const long long items = a.n_blocks * chunks;
     const int lane = threadIdx.x & 31;
-    for (long long it = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; it < items;
-         it += ((long long)gridDim.x * blockDim.x) >> 5) {
-        const long long b = it / chunks;
+    const long long stride = ((long long)gridDim.x * blockDim.x) >> 5;
+    // the two words of item it that the lane's windows lie in (word -1 of a block
+    // is its start state); a lane with no steps in the item reads nothing
+    auto fetch = [&](long long it, unsigned long long& v) {
+        if (it >= items) return;
+        const long long b = chunks == 1 ? it : it / chunks;
         const int c = (int)(it - b * chunks);
-        const int t0 = (c << 7) + 4 * lane;  // steps t0+1 .. t0+4
-        if (t0 + 4 > NS) continue;           // NS % 4 == 0: a lane's steps are all in or all out
+        if ((c << 7) + 4 * lane + 4 > NS) return;
         const uint32_t* wb = a.bits + b * a.W;
         const int wi = (c << 4) + (lane >> 1);  // word holding the lane's last window end
         const unsigned long long hi = wi >= 1 ? __ldg(wb + wi - 1) : __ldg(a.start_state + b);
-        const unsigned long long v = (hi << 32) | __ldg(wb + wi);
-        float y[8];
+        v = (hi << 32) | __ldg(wb + wi);
+    };
+    long long it = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    unsigned long long v = 0, vn = 0;
+    fetch(it, v);  // the first item's words load while the table is copied
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+    for (; it < items; it += stride) {
+        fetch(it + stride, vn);  // the next item's words are in flight during this one
+        const long long b = chunks == 1 ? it : it / chunks;
+        const int c = (int)(it - b * chunks);
+        const int t0 = (c << 7) + 4 * lane;  // steps t0+1 .. t0+4
+        if (t0 + 4 <= NS) {                  // NS % 4 == 0: a lane's steps are all in or all out
+            float y[8];
 #pragma unroll
-        for (int q = 1; q <= 4; ++q) {
-            // window start relative to bit 0 of v: 16 (lane & 1) + 4q + 16
-            const int sh = 48 - (16 * (lane & 1) + 4 * q + 16);
-            const uint32_t s = (uint32_t)(v >> sh) & 0xffffu;
-            const uint32_t w = s < kVec2DecSmemStates ? tab[s] : __ldg(cb + s);
-            const __half2 h2 = *reinterpret_cast<const __half2*>(&w);
-            const float2 f = __half22float2(h2);
-            y[2 * q - 2] = f.x;
-            y[2 * q - 1] = f.y;
+            for (int q = 1; q <= 4; ++q) {
+                // window start relative to bit 0 of v: 16 (lane & 1) + 4q + 16
+                const int sh = 48 - (16 * (lane & 1) + 4 * q + 16);
+                const uint32_t s = (uint32_t)(v >> sh) & 0xffffu;
+                const uint32_t w = s < kVec2DecSmemStates ? tab[s] : __ldg(cb + s);
+                const __half2 h2 = *reinterpret_cast<const __half2*>(&w);
+                const float2 f = __half22float2(h2);
+                y[2 * q - 2] = f.x;
+                y[2 * q - 1] = f.y;
+            }
+            float4* dst = reinterpret_cast<float4*>(a.y + b * a.y_stride + 2 * (long long)t0);
+            __stcs(dst, make_float4(y[0], y[1], y[2], y[3]));
+            __stcs(dst + 1, make_float4(y[4], y[5], y[6], y[7]));
         }
-        float4* dst = reinterpret_cast<float4*>(a.y + b * a.y_stride + 2 * (long long)t0);
-        __stcs(dst, make_float4(y[0], y[1], y[2], y[3]));
-        __stcs(dst + 1, make_float4(y[4], y[5], y[6], y[7]));
+        v = vn;
     }
 }
 

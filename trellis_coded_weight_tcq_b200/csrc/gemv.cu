@@ -606,26 +606,26 @@ __device__ __forceinline__ void word_dot(uint32_t hi, uint32_t lo, const float* 
         unpack2(p, p0, p1);
         acc0 += p0;
         acc1 += p1;
-        return;
-    }
-    float xv[16];
+    } else {
+        float xv[16];
 #pragma unroll
-    for (int e = 0; e < 16; e += 4) {
-        const float4 v = *reinterpret_cast<const float4*>(xq + e);
-        xv[e] = v.x;
-        xv[e + 1] = v.y;
-        xv[e + 2] = v.z;
-        xv[e + 3] = v.w;
-    }
-    float p0 = pair_codeword<CODE>(st[0], tab) * xv[0];
-    float p1 = pair_codeword<CODE>(st[1], tab) * xv[1];
+        for (int e = 0; e < 16; e += 4) {
+            const float4 v = *reinterpret_cast<const float4*>(xq + e);
+            xv[e] = v.x;
+            xv[e + 1] = v.y;
+            xv[e + 2] = v.z;
+            xv[e + 3] = v.w;
+        }
+        float p0 = pair_codeword<CODE>(st[0], tab) * xv[0];
+        float p1 = pair_codeword<CODE>(st[1], tab) * xv[1];
 #pragma unroll
-    for (int e = 2; e < 16; e += 2) {
-        p0 = fmaf(pair_codeword<CODE>(st[e], tab), xv[e], p0);
-        p1 = fmaf(pair_codeword<CODE>(st[e + 1], tab), xv[e + 1], p1);
+        for (int e = 2; e < 16; e += 2) {
+            p0 = fmaf(pair_codeword<CODE>(st[e], tab), xv[e], p0);
+            p1 = fmaf(pair_codeword<CODE>(st[e + 1], tab), xv[e + 1], p1);
+        }
+        acc0 += p0;
+        acc1 += p1;
     }
-    acc0 += p0;
-    acc1 += p1;
 }
 
 template <int CODE>

@@ -50,11 +50,19 @@ constexpr int kUb8Unroll = 2;   // steps a lane scores per pass over the codeboo
 // the backpointer byte, the symbol and the row (16-bit each)
 constexpr size_t kUb8StepBytes = 4 * 4 + 4 + 1 + 2 + 2;
 
-__device__ __forceinline__ int ub8_next(int s, int z)
+__host__ __device__ constexpr int ub8_next(int s, int z)
 {
-    const int p = (s >> 2) & 1, q = (s >> 1) & 1, r = s & 1;
-    return 4 * (p ^ q) + 2 * (r ^ z) + p;
+    return 4 * (((s >> 2) & 1) ^ ((s >> 1) & 1)) + 2 * ((s & 1) ^ z) + ((s >> 2) & 1);
 }
+
+// the successors of states 0..7 as nibbles (nibble s = ub8_next(s, z)), one table per z
+__host__ __device__ constexpr uint32_t ub8_next_table(int z)
+{
+    uint32_t t = 0;
+    for (int s = 0; s < 8; ++s) t |= (uint32_t)ub8_next(s, z) << (4 * s);
+    return t;
+}
+constexpr uint32_t kUb8Next0 = ub8_next_table(0), kUb8Next1 = ub8_next_table(1);
 
 // Stages the union codebook (rows x V, fp32 or binary16) into shared memory as fp32.
 __device__ __forceinline__ void ub8_stage_codebook(float* dst, const void* cb, int cb_f16, int n)
@@ -294,8 +302,13 @@ constexpr int kUb8DecWarps = 8;
 // or 8 values leave as 8- or 16-byte stores (the output is aligned for them).
 constexpr int kUb8DecStageWords = 32;
 
+// six CTAs per SM (at most 40 registers); the shapes that would spill at 40
+// registers keep the default register count
 template <int V, bool STAGED, bool VSTORE>
-__global__ void __launch_bounds__(kUb8DecWarps * 32) ub8_decode_kernel(Ub8DecodeArgs a)
+constexpr int ub8_dec_min_blocks() { return STAGED && !(V == 8 && VSTORE) ? 6 : 1; }
+
+template <int V, bool STAGED, bool VSTORE>
+__global__ void __launch_bounds__(kUb8DecWarps * 32, (ub8_dec_min_blocks<V, STAGED, VSTORE>())) ub8_decode_kernel(Ub8DecodeArgs a)
 {
     extern __shared__ __align__(16) unsigned char smem[];
     const int rows = 4 << a.m;
@@ -319,22 +332,20 @@ __global__ void __launch_bounds__(kUb8DecWarps * 32) ub8_decode_kernel(Ub8Decode
         const long long b0 = g * 32;
         const int nb = (int)min(32LL, a.n_blocks - b0);
         if constexpr (STAGED) {
-            // the group's words are contiguous: coalesced loads, eight in flight
-            // per lane, then stores into the padded rows
-            const uint32_t* src = a.bits + b0 * a.W;
-            const int nw = nb * a.W;
-            for (int i0 = 0; i0 < nw; i0 += 8 * 32) {
+            // the group's words, row by row (lane w of a row loads word w; the
+            // group's rows are contiguous, so a row is one coalesced read), eight
+            // rows in flight per lane, then stored into the padded rows
+            const uint32_t* src = a.bits + b0 * a.W + lane;
+            uint32_t* dst = WB + lane;
+            for (int q0 = 0; q0 < nb; q0 += 8) {
                 uint32_t r[8];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int i = i0 + 32 * u + lane;
-                    r[u] = i < nw && TCQ_IN_BOUNDS(b0 * a.W + i, a.n_blocks * a.W) ? src[i] : 0u;
-                }
+                for (int u = 0; u < 8; ++u)
+                    r[u] = lane < a.W && q0 + u < nb && TCQ_IN_BOUNDS((b0 + q0 + u) * a.W + lane, a.n_blocks * a.W)
+                               ? src[(q0 + u) * a.W] : 0u;
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int i = i0 + 32 * u + lane;
-                    if (i < nw) WB[(i / a.W) * WP + i % a.W] = r[u];
-                }
+                for (int u = 0; u < 8; ++u)
+                    if (lane < a.W && q0 + u < nb) dst[(q0 + u) * WP] = r[u];
             }
             __syncwarp();
         }
@@ -342,50 +353,62 @@ __global__ void __launch_bounds__(kUb8DecWarps * 32) ub8_decode_kernel(Ub8Decode
             if constexpr (STAGED) return WB[q * WP + w];
             else return TCQ_IN_BOUNDS((b0 + q) * a.W + w, a.n_blocks * a.W) ? a.bits[(b0 + q) * a.W + w] : 0u;
         };
-        // walk: lane l follows block b0 + l and records p of the state before each step
+        // walk: lane l follows block b0 + l and records p of the state before each
+        // step; the successor of state s on branch bit z is nibble s of kUb8Next[z]
         if (lane < nb) {
             const long long b = b0 + lane;
             uint32_t* Pl = P + lane * PW;
-            int s = TCQ_IN_BOUNDS(b, a.n_blocks) ? (int)(a.start_state[b] & 7u) : 0;
+            uint32_t s = TCQ_IN_BOUNDS(b, a.n_blocks) ? (a.start_state[b] & 7u) : 0u;
             uint32_t acc = 0;
-            for (int t = 0; t < S; ++t) {
-                const int pos = t * K;  // the branch bit is the symbol's first bit
-                const int z = (int)((word(lane, pos >> 5) >> (31 - (pos & 31))) & 1u);
-                acc |= (uint32_t)((s >> 2) & 1) << (t & 31);
+            int pos = 0;  // the branch bit is the symbol's first bit
+            for (int t = 0; t < S; ++t, pos += K) {
+                const uint32_t z = (word(lane, pos >> 5) >> (31 - (pos & 31))) & 1u;
+                acc = __funnelshift_r(acc, s >> 2, 1);  // p of step t into bit 31, earlier steps down
                 if ((t & 31) == 31) {
                     Pl[t >> 5] = acc;
                     acc = 0;
                 }
-                s = ub8_next(s, z);
+                s = ((z ? kUb8Next1 : kUb8Next0) >> (4 * s)) & 7u;
             }
-            if (S & 31) Pl[S >> 5] = acc;
+            if (S & 31) Pl[S >> 5] = acc >> (32 - (S & 31));
         }
         __syncwarp();
-        // emit: the whole warp writes one block at a time
-        for (int q = 0; q < nb; ++q) {
-            const long long b = b0 + q;
-            float* yb = a.y + b * a.T;
-            for (int t = lane; t < S; t += 32) {
-                const int pos = t * K;
-                const int w0 = pos >> 5, off = pos & 31;
-                // K <= 9 bits: at most two words
-                const uint32_t hi = word(q, w0);
-                const uint32_t lo = off + K > 32 ? word(q, w0 + 1) : 0u;
-                const uint32_t sym = (__funnelshift_l(lo, hi, off) >> (32 - K));
-                const int z = (int)(sym >> a.m);
-                const int p = (int)((P[q * PW + (t >> 5)] >> (t & 31)) & 1u);
-                const float* row = cbs + (size_t)(4 * (sym & imask) + 2 * z + p) * V;
-                if (!TCQ_IN_BOUNDS(b * a.T + t * V + V - 1, a.n_blocks * a.T)) continue;
+        // emit: the whole warp writes one block at a time, lane l the steps
+        // t = l + 32 r; a step's stream position, word and P bit depend only on
+        // (lane, r), so they are set once per r and the inner loop runs over blocks
+        for (int r = 0; 32 * r < S; ++r) {
+            const int t = lane + 32 * r;
+            if (t >= S) break;
+            const int pos = t * K;
+            const int w0 = pos >> 5, off = pos & 31;
+            const bool two = off + K > 32;  // K <= 9 bits: at most two words
+            float* yt = a.y + b0 * a.T + t * V;   // block q's values at yt + q T
+            const uint32_t* pr = P + r;           // block q's P word at pr + q PW
+            const uint32_t* wq = WB + w0;         // staged: block q's word w0 at wq + q WP
+            for (int q = 0; q < nb; ++q, yt += a.T, pr += PW, wq += WP) {
+                uint32_t hi, lo = 0u;
+                if constexpr (STAGED) {
+                    hi = wq[0];
+                    if (two) lo = wq[1];
+                } else {
+                    hi = word(q, w0);
+                    if (two) lo = word(q, w0 + 1);
+                }
+                const uint32_t sym = __funnelshift_l(lo, hi, off) >> (32 - K);
+                const uint32_t z = sym >> a.m;
+                const uint32_t p = (*pr >> lane) & 1u;
+                const float* row = cbs + (size_t)(((sym & imask) << 2) | (z << 1) | p) * V;
+                if (!TCQ_IN_BOUNDS((b0 + q) * a.T + t * V + V - 1, a.n_blocks * a.T)) continue;
                 if constexpr (VSTORE && V == 4) {
-                    *reinterpret_cast<float4*>(yb + t * V) = *reinterpret_cast<const float4*>(row);
+                    *reinterpret_cast<float4*>(yt) = *reinterpret_cast<const float4*>(row);
                 } else if constexpr (VSTORE && V == 8) {
-                    reinterpret_cast<float4*>(yb + t * V)[0] = reinterpret_cast<const float4*>(row)[0];
-                    reinterpret_cast<float4*>(yb + t * V)[1] = reinterpret_cast<const float4*>(row)[1];
+                    reinterpret_cast<float4*>(yt)[0] = reinterpret_cast<const float4*>(row)[0];
+                    reinterpret_cast<float4*>(yt)[1] = reinterpret_cast<const float4*>(row)[1];
                 } else if constexpr (VSTORE && V == 2) {
-                    *reinterpret_cast<float2*>(yb + t * V) = *reinterpret_cast<const float2*>(row);
+                    *reinterpret_cast<float2*>(yt) = *reinterpret_cast<const float2*>(row);
                 } else {
 #pragma unroll
-                    for (int v = 0; v < V; ++v) yb[t * V + v] = row[v];
+                    for (int v = 0; v < V; ++v) yt[v] = row[v];
                 }
             }
         }
