@@ -42,9 +42,13 @@ __global__ void __launch_bounds__(kGemvVec2Threads) gemv_vec2_kernel(GemvArgs a)
     extern __shared__ __align__(16) uint32_t tab[];  // [kGemvVec2SmemStates]
     const uint32_t* cb = reinterpret_cast<const uint32_t*>(a.cb);
     {
-        const uint4* src = reinterpret_cast<const uint4*>(cb);
-        uint4* dst = reinterpret_cast<uint4*>(tab);
-        for (int i = threadIdx.x; i < (int)(kGemvVec2SmemStates / 4); i += blockDim.x) dst[i] = __ldg(src + i);
+        // the table by asynchronous 16-byte copies, all in flight at once
+        const uint32_t dst = (uint32_t)__cvta_generic_to_shared(tab);
+        for (int i = threadIdx.x; i < (int)(kGemvVec2SmemStates / 4); i += blockDim.x)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + 16 * i),
+                         "l"(cb + 4 * (size_t)i) : "memory");
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        asm volatile("cp.async.wait_all;" ::: "memory");
     }
     __syncthreads();
     const int NS = a.T >> 1;
@@ -64,7 +68,7 @@ __global__ void __launch_bounds__(kGemvVec2Threads) gemv_vec2_kernel(GemvArgs a)
 #pragma unroll
             for (int u = 0; u < kGemvVec2Unroll; ++u) {
                 const long long i = i0 + u;
-                const long long j = i / chunks;
+                const long long j = chunks == 1 ? i : i / chunks;
                 const int c = (int)(i - j * chunks);
                 const int t0 = (c << 7) + 4 * lane;  // steps t0+1 .. t0+4
                 on[u] = i < items && t0 + 4 <= NS;   // NS % 4 == 0
