@@ -205,7 +205,8 @@ def _gemv_vec_check(bits, start, scale, cb, L, k, V, T, rows, cols, x, y):
 
 @pytest.mark.parametrize("L,k,V,T,rows,nb,cbt,cb_offset", [
     (16, 2, 2, 256, 300, 16, "f16", 0),   # compile-time kernel, the MLP shape's blocks
-    (16, 2, 2, 264, 37, 5, "f16", 0),     # 132 steps: a partial second chunk
+    (16, 2, 2, 256, 4773, 16, "f16", 0),  # 4736 warps x one row, then 37 rows split over CTAs
+    (16, 2, 2, 264, 37, 5, "f16", 0),     # 132 steps: a partial second chunk, rows split over CTAs
     (16, 2, 2, 256, 40, 4, "f16", 1),     # unaligned table: runtime kernel
     (16, 2, 2, 30, 20, 3, "f16", 0),      # T % 8 != 0: runtime kernel
     (12, 2, 2, 64, 50, 6, "f32", 0),
@@ -231,6 +232,29 @@ def test_gemv_vec(L, k, V, T, rows, nb, cbt, cb_offset, scaled, cuda_device):
                      cbt_dev, L, k, V, T, rows, cols, torch.from_numpy(x).to(cuda_device))
     torch.cuda.synchronize()
     _gemv_vec_check(bits, start, scale, cb, L, k, V, T, rows, cols, x, y.cpu().numpy())
+
+
+def test_gemv_vec2_rows_bit_identical_across_phases(cuda_device):
+    """Rows with the same blocks give the same bits whether a warp takes the
+    row or the row's items are spread over a CTA's warps (the last round)."""
+    import torch
+    from tests.test_gpu_gemv import _rand_stream
+
+    L, k, V, T, nb = 16, 2, 2, 256, 16
+    rows = 4736 + 37  # 148 CTAs x 32 warps, then 37 rows, one per CTA
+    rng = np.random.default_rng(8650)
+    bits1, start1 = _rand_stream(rng, nb, k * V, T // V)
+    bits = np.tile(bits1, (rows, 1))
+    start = np.tile(start1, rows)
+    cb = rng.standard_normal((1 << L, V)).astype(np.float16)
+    x = rng.standard_normal(nb * T).astype(np.float32)
+    y = tcq.gemv_vec(torch.from_numpy(np.ascontiguousarray(bits).view(np.int32)).to(cuda_device),
+                     torch.from_numpy(np.ascontiguousarray(start).view(np.int32)).to(cuda_device),
+                     None, torch.from_numpy(cb).to(cuda_device), L, k, V, T, rows, nb * T,
+                     torch.from_numpy(x).to(cuda_device))
+    torch.cuda.synchronize()
+    y = y.cpu().numpy()
+    assert np.all(y == y[0])
 
 
 def test_gemv_vec_of_encoded_matrix(cuda_device):

@@ -37,9 +37,68 @@ __device__ __forceinline__ float warp_sum(float v)
     return v;
 }
 
+// One (block, chunk) item of row r for this lane: its share of the item's dot
+// product (four steps, eight weights, one FMA chain) and the block's scale.
+// `on` is false (and part 0) when the lane has no steps in the item.
+struct Vec2Item {
+    unsigned long long v;
+    float4 x0, x1;
+    float sc;
+    bool on;
+};
+
+__device__ __forceinline__ void vec2_item_load(const GemvArgs& a, long long r, long long i, int chunks,
+                                               int NS, long long nb, long long items, int lane, Vec2Item& it)
+{
+    const long long j = chunks == 1 ? i : i / chunks;
+    const int c = (int)(i - j * chunks);
+    const int t0 = (c << 7) + 4 * lane;  // steps t0+1 .. t0+4
+    it.on = i < items && t0 + 4 <= NS;   // NS % 4 == 0
+    it.v = 0ull;
+    it.x0 = it.x1 = make_float4(0.f, 0.f, 0.f, 0.f);
+    it.sc = 0.f;
+    if (it.on) {
+        const long long b = r * nb + j;
+        const uint32_t* wb = a.bits + b * a.W;
+        const int wi = (c << 4) + (lane >> 1);
+        const unsigned long long hi = wi >= 1 ? __ldg(wb + wi - 1) : __ldg(a.start_state + b);
+        it.v = (hi << 32) | __ldg(wb + wi);
+        const float* xb = a.x + j * a.T + 2 * t0;
+        it.x0 = __ldg(reinterpret_cast<const float4*>(xb));
+        it.x1 = __ldg(reinterpret_cast<const float4*>(xb + 4));
+        it.sc = a.scale ? __ldg(a.scale + b) : 1.f;
+    }
+}
+
+__device__ __forceinline__ float vec2_item_part(const Vec2Item& it, const uint32_t* tab, const uint32_t* cb,
+                                                int lane)
+{
+    const float xs[8] = {it.x0.x, it.x0.y, it.x0.z, it.x0.w, it.x1.x, it.x1.y, it.x1.z, it.x1.w};
+    float part = 0.f;
+#pragma unroll
+    for (int q = 1; q <= 4; ++q) {
+        const int sh = 48 - (16 * (lane & 1) + 4 * q + 16);
+        const uint32_t s = (uint32_t)(it.v >> sh) & 0xffffu;
+        const uint32_t w = s < kGemvVec2SmemStates ? tab[s] : __ldg(cb + s);
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w));
+        part = fmaf(f.x, xs[2 * q - 2], part);
+        part = fmaf(f.y, xs[2 * q - 1], part);
+    }
+    return part;
+}
+
+// Rows: whole rounds give every warp one row at a time; the rows of the last,
+// partial round, when they are at most one per CTA and a row's items fit the
+// shared memory left beside the table, go one per CTA with its items spread
+// over the CTA's warps, each lane's share of each item stored and then summed
+// by one warp in item order with the same FMAs, so that a row's result is the
+// same bits either way (14336 rows over 4736 warps left 64 warps a fourth row
+// while the others idled).
+constexpr int kGemvVec2MaxSplitItems = 23;  // items x (32 + 1) floats in the 3 KiB left
+
 __global__ void __launch_bounds__(kGemvVec2Threads) gemv_vec2_kernel(GemvArgs a)
 {
-    extern __shared__ __align__(16) uint32_t tab[];  // [kGemvVec2SmemStates]
+    extern __shared__ __align__(16) uint32_t tab[];  // [kGemvVec2SmemStates], then the split row's shares
     const uint32_t* cb = reinterpret_cast<const uint32_t*>(a.cb);
     {
         // the table by asynchronous 16-byte copies, all in flight at once
@@ -55,58 +114,48 @@ __global__ void __launch_bounds__(kGemvVec2Threads) gemv_vec2_kernel(GemvArgs a)
     const int chunks = (NS + 127) >> 7;
     const long long nb = a.cols / a.T;  // blocks per row
     const long long items = nb * chunks;  // (block, 128-step chunk) pairs of a row
-    const int lane = threadIdx.x & 31;
-    for (long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < a.rows;
-         r += ((long long)gridDim.x * blockDim.x) >> 5) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+    const long long full = (a.rows / nw) * nw;
+    const bool split = items <= kGemvVec2MaxSplitItems && a.rows - full <= (long long)gridDim.x;
+    const long long rows_a = split ? full : a.rows;
+    for (long long r = (long long)blockIdx.x * (blockDim.x >> 5) + warp; r < rows_a; r += nw) {
         float acc = 0.f;
         // kGemvVec2Unroll items at a time: all their loads issue before any use
         for (long long i0 = 0; i0 < items; i0 += kGemvVec2Unroll) {
-            unsigned long long v[kGemvVec2Unroll];
-            float4 x0[kGemvVec2Unroll], x1[kGemvVec2Unroll];
-            float sc[kGemvVec2Unroll];
-            bool on[kGemvVec2Unroll];
+            Vec2Item it[kGemvVec2Unroll];
 #pragma unroll
-            for (int u = 0; u < kGemvVec2Unroll; ++u) {
-                const long long i = i0 + u;
-                const long long j = chunks == 1 ? i : i / chunks;
-                const int c = (int)(i - j * chunks);
-                const int t0 = (c << 7) + 4 * lane;  // steps t0+1 .. t0+4
-                on[u] = i < items && t0 + 4 <= NS;   // NS % 4 == 0
-                v[u] = 0ull;
-                x0[u] = x1[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                sc[u] = 0.f;
-                if (on[u]) {
-                    const long long b = r * nb + j;
-                    const uint32_t* wb = a.bits + b * a.W;
-                    const int wi = (c << 4) + (lane >> 1);
-                    const unsigned long long hi = wi >= 1 ? __ldg(wb + wi - 1) : __ldg(a.start_state + b);
-                    v[u] = (hi << 32) | __ldg(wb + wi);
-                    const float* xb = a.x + j * a.T + 2 * t0;
-                    x0[u] = __ldg(reinterpret_cast<const float4*>(xb));
-                    x1[u] = __ldg(reinterpret_cast<const float4*>(xb + 4));
-                    sc[u] = a.scale ? __ldg(a.scale + b) : 1.f;
-                }
-            }
+            for (int u = 0; u < kGemvVec2Unroll; ++u)
+                vec2_item_load(a, r, i0 + u, chunks, NS, nb, items, lane, it[u]);
 #pragma unroll
-            for (int u = 0; u < kGemvVec2Unroll; ++u) {
-                if (!on[u]) continue;
-                const float xs[8] = {x0[u].x, x0[u].y, x0[u].z, x0[u].w,
-                                     x1[u].x, x1[u].y, x1[u].z, x1[u].w};
-                float part = 0.f;
-#pragma unroll
-                for (int q = 1; q <= 4; ++q) {
-                    const int sh = 48 - (16 * (lane & 1) + 4 * q + 16);
-                    const uint32_t s = (uint32_t)(v[u] >> sh) & 0xffffu;
-                    const uint32_t w = s < kGemvVec2SmemStates ? tab[s] : __ldg(cb + s);
-                    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w));
-                    part = fmaf(f.x, xs[2 * q - 2], part);
-                    part = fmaf(f.y, xs[2 * q - 1], part);
-                }
-                acc = fmaf(sc[u], part, acc);
-            }
+            for (int u = 0; u < kGemvVec2Unroll; ++u)
+                if (it[u].on) acc = fmaf(it[u].sc, vec2_item_part(it[u], tab, cb, lane), acc);
         }
         acc = warp_sum(acc);
         if (lane == 0) a.y[r] = acc;
+    }
+    if (!split) return;
+    float* share = reinterpret_cast<float*>(tab + kGemvVec2SmemStates);  // [items][33]: 32 lanes, the scale
+    for (long long r = full + blockIdx.x; r < a.rows; r += gridDim.x) {
+        for (long long i = warp; i < items; i += blockDim.x >> 5) {
+            Vec2Item it;
+            vec2_item_load(a, r, i, chunks, NS, nb, items, lane, it);
+            share[i * 33 + lane] = it.on ? vec2_item_part(it, tab, cb, lane) : 0.f;
+            if (lane == 0) share[i * 33 + 32] = it.sc;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            float acc = 0.f;
+            for (long long i = 0; i < items; ++i) {
+                const long long j = chunks == 1 ? i : i / chunks;
+                const int c = (int)(i - j * chunks);
+                if ((c << 7) + 4 * lane + 4 <= NS)  // the lanes with steps in the item, as in phase A
+                    acc = fmaf(share[i * 33 + 32], share[i * 33 + lane], acc);
+            }
+            acc = warp_sum(acc);
+            if (lane == 0) a.y[r] = acc;
+        }
+        __syncthreads();
     }
 }
 
@@ -146,7 +195,9 @@ cudaError_t launch_gemv_vec(const GemvArgs& a, int V, int num_sms, cudaStream_t 
 {
     if (a.L == 16 && a.K == 4 && V == 2 && a.cb_f16 == 1 && a.T % 8 == 0 &&
         (reinterpret_cast<uintptr_t>(a.cb) & 15) == 0) {
-        const size_t smem = kGemvVec2SmemStates * sizeof(uint32_t);
+        const long long items = (long long)(a.cols / a.T) * ((a.T / 2 + 127) / 128);
+        const size_t smem = kGemvVec2SmemStates * sizeof(uint32_t) +
+                            (items <= kGemvVec2MaxSplitItems ? (size_t)items * 33 * sizeof(float) : 0);
         const cudaError_t e = cudaFuncSetAttribute(gemv_vec2_kernel,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
