@@ -436,11 +436,22 @@ def run_ours(args, rank, world, local_rank):
         g_ms = _median_ms(g_ev)
         g_bytes = n * W * 4 + n * 4 + n * 4 + cols_m * 4 + rows_m * 4
         peaks_g, _ = _peaks()
+        # the table code is bound by shared memory, not HBM: one table lookup per
+        # weight against one 32-lane wavefront per SM and clock (conflict-free);
+        # 32 random 2-byte lookups over 32 banks cost about 3.5 wavefronts, so
+        # about 1 / 3.5 of this peak is the floor of a random table
+        smem_peak = SMS * 32 * float(peaks_g.get("sm_max_mhz", 1965.0)) * 1e6
+        lookups_per_s = rows_m * cols_m / (g_ms / 1e3)
         gemv = {"rows": rows_m, "cols": cols_m, "ms": g_ms,
                 "weights_per_s": rows_m * cols_m / (g_ms / 1e3),
                 "hbm_gbs": g_bytes / (g_ms / 1e3) / 1e9,
                 "hbm_frac": g_bytes / (g_ms / 1e3) / 1e9 / float(peaks_g.get("hbm_gbs", 6650.0)),
-                "bytes": g_bytes}
+                "bytes": g_bytes,
+                "bound": "smem", "lookups_per_s": lookups_per_s,
+                "smem_frac": lookups_per_s / smem_peak,
+                "smem_peak_basis": f"{SMS} SMs x 32 lookups per clock (one conflict-free wavefront) x "
+                                   f"{peaks_g.get('sm_max_mhz', 1965.0)} MHz; random lookups cost about "
+                                   "3.5 wavefronts, so the attainable fraction is about 0.29"}
         # the same bitstreams read as the computed (lookup-free) code: no table,
         # each codeword computed in registers
         for _ in range(3):
