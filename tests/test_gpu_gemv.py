@@ -117,23 +117,25 @@ def test_gemv_rejections(cuda_device):
     assert call(L=17) == tcq.TCQ_ERR_UNSUPPORTED
 
 
-# 148 CTAs x 16 warps = 2368 warps, three rows per item
+# 148 CTAs x 16 warps = 2368 warps; three rows per item from 3 x 2368 = 7104 rows
+# on, one row per item below
 @pytest.mark.parametrize("rows,nb,code", [
-    (7204, 16, "f16"),    # one whole round of row groups, then 100 rows, one per CTA
+    (7204, 16, "f16"),    # three-row items: one whole round, then 100 rows, one per CTA
     (7204, 16, "mad"),
-    (5000, 16, "f16"),    # fewer groups than warps: a partial round, 2 rows of no group
-    (4737, 32, "f16"),    # two 4096-column chunks per row; a partial round
-    (4801, 32, "mad"),    # a partial round and 1 row of no group
-    (9473, 16, "mad"),    # a whole round, a partial round of 789 groups, then 2 rows
+    (9473, 16, "mad"),    # three-row items: a whole round, a partial round of 789 groups, then 2 rows
     (14336, 16, "f16"),   # the MLP matrix's rows: two whole rounds, then 128 rows one per CTA
+    (5000, 16, "f16"),    # one-row items: two whole rounds, a partial round of 264 rows
+    (4737, 32, "f16"),    # two 4096-column chunks per row; two whole rounds, 1 row one per CTA
+    (4801, 32, "mad"),    # two whole rounds, 65 rows one per CTA
     (37, 16, "f16"),      # fewer rows than CTAs: only the per-CTA rows
 ])
 @pytest.mark.parametrize("scaled", [False, True])
 def test_gemv_half_block_kernel(rows, nb, code, scaled, cuda_device):
     """L = 16, k = 2, T = 256 with cols a multiple of 4096: the kernel that takes
     half a coding block per lane and three rows per item, in both of its phases
-    (every warp's share of row groups, with the last partial round either kept
-    there or, when it is at most one row per CTA, spread one row per CTA)."""
+    (every warp's share of row groups of three rows or one, with the last
+    partial round either kept there or, when it is at most one row per CTA,
+    spread one row per CTA)."""
     import torch
     from oracle import oracle_mad_codebook
 
@@ -181,13 +183,14 @@ def test_gemv_misaligned_bits_take_the_general_kernel(cuda_device):
     _check(bits, start, None, cb, L, k, T, rows, cols, x, y.cpu().numpy())
 
 
-def test_gemv_half_block_kernel_rows_bit_identical_across_phases(cuda_device):
+@pytest.mark.parametrize("rows", [7104 + 37,   # three-row items: one whole round, then 37 rows one per CTA
+                                  2368 + 37])  # one-row items: one whole round, then 37 rows one per CTA
+def test_gemv_half_block_kernel_rows_bit_identical_across_phases(rows, cuda_device):
     """Rows with the same blocks give the same bits whether the row falls in the
     warps' row groups or among the rows spread one per CTA."""
     import torch
 
     L, k, T, nb = 16, 2, 256, 16
-    rows = 7104 + 37  # 148 x 16 warps x 3 rows, then 37 rows, one per CTA
     rng = np.random.default_rng(404)
     bits1, start1 = _rand_stream(rng, nb, k, T)
     bits = np.tile(bits1, (rows, 1))
@@ -203,3 +206,27 @@ def test_gemv_half_block_kernel_rows_bit_identical_across_phases(cuda_device):
         torch.cuda.synchronize()
         y = y.cpu().numpy()
         assert np.all(y == y[0]), code
+
+
+def test_gemv_half_block_kernel_rows_per_item_give_the_same_bits(cuda_device):
+    """The same row through three-row items (7141 rows) and one-row items (2405
+    rows): the same bits, since a row's arithmetic does not depend on the rows
+    an item holds."""
+    import torch
+
+    L, k, T, nb = 16, 2, 256, 16
+    rng = np.random.default_rng(405)
+    bits1, start1 = _rand_stream(rng, nb, k, T)
+    cb = rng.standard_normal(1 << L).astype(np.float16)
+    x = rng.standard_normal(nb * T).astype(np.float32)
+    dev = torch.device("cuda", 0)
+    for code in ("f16", "mad"):
+        c = tcq.MAD if code == "mad" else torch.from_numpy(cb).to(dev)
+        first = []
+        for rows in (7104 + 37, 2368 + 37):
+            b = torch.from_numpy(np.ascontiguousarray(np.tile(bits1, (rows, 1))).view(np.int32)).to(dev)
+            s = torch.from_numpy(np.ascontiguousarray(np.tile(start1, rows)).view(np.int32)).to(dev)
+            y = tcq.gemv(b, s, None, c, L, k, T, rows, nb * T, torch.from_numpy(x).to(dev))
+            torch.cuda.synchronize()
+            first.append(y[0].item())
+        assert first[0] == first[1], code

@@ -507,7 +507,9 @@ __global__ void __launch_bounds__(kMadRowsThreads, 1) gemv_rows_kernel(GemvArgs 
 // ---------------------------------------------------------------------------
 constexpr int kPairThreads = 512;
 constexpr int kPairWarps = kPairThreads / 32;
-constexpr int kPairRows = 3;  // rows per warp item
+// rows per warp item: three when every warp has at least three rows (the x
+// loads serve three rows), else one, so that every warp has work
+constexpr int kPairRowsMax = 3;
 
 // padded position of x[i] in shared memory: 4 floats of padding per 128
 __device__ __forceinline__ int xpad(int i) { return i + ((i >> 7) << 2); }
@@ -628,9 +630,10 @@ __device__ __forceinline__ void word_dot(uint32_t hi, uint32_t lo, const float* 
     }
 }
 
-template <int CODE>
+template <int CODE, int R>
 __global__ void __launch_bounds__(kPairThreads, 1) gemv_pair_kernel(GemvArgs a)
 {
+    constexpr int kPairRows = R;  // rows per warp item
     constexpr int T = 256, W = 16;
     extern __shared__ __align__(16) unsigned char gsm[];
     constexpr size_t TAB = CODE == kCodeMad ? 0 : ((size_t)1 << 16) * 2;
@@ -804,15 +807,22 @@ cudaError_t launch_gemv_pair(const GemvArgs& a, int num_sms, cudaStream_t stream
     const size_t tab = mad ? 0 : ((size_t)1 << 16) * 2;
     // x padded, then phase B's two floats per stream word of a row (cols / 16 words)
     const size_t smem = tab + (size_t)(a.cols + (a.cols / 128) * 4) * 4 + (size_t)(a.cols / 16) * 2 * 4;
-    const void* fn = mad ? reinterpret_cast<const void*>(&gemv_pair_kernel<kCodeMad>)
-                         : reinterpret_cast<const void*>(&gemv_pair_kernel<kCodeF16>);
+    int grid = num_sms;  // one CTA of 16 warps per SM
+    const bool three = a.rows >= (long long)kPairRowsMax * grid * kPairWarps;
+    const void* fn = mad ? (three ? reinterpret_cast<const void*>(&gemv_pair_kernel<kCodeMad, 3>)
+                                  : reinterpret_cast<const void*>(&gemv_pair_kernel<kCodeMad, 1>))
+                         : (three ? reinterpret_cast<const void*>(&gemv_pair_kernel<kCodeF16, 3>)
+                                  : reinterpret_cast<const void*>(&gemv_pair_kernel<kCodeF16, 1>));
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    int grid = num_sms;  // one CTA of 16 warps per SM
-    if (mad)
-        gemv_pair_kernel<kCodeMad><<<grid, kPairThreads, smem, stream>>>(a);
+    if (mad && three)
+        gemv_pair_kernel<kCodeMad, 3><<<grid, kPairThreads, smem, stream>>>(a);
+    else if (mad)
+        gemv_pair_kernel<kCodeMad, 1><<<grid, kPairThreads, smem, stream>>>(a);
+    else if (three)
+        gemv_pair_kernel<kCodeF16, 3><<<grid, kPairThreads, smem, stream>>>(a);
     else
-        gemv_pair_kernel<kCodeF16><<<grid, kPairThreads, smem, stream>>>(a);
+        gemv_pair_kernel<kCodeF16, 1><<<grid, kPairThreads, smem, stream>>>(a);
     return cudaGetLastError();
 }
 template <int L, int K, int N, int T, int CODE>
