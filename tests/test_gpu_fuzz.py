@@ -114,3 +114,48 @@ def test_ub8_random_shape(V, m, T, nb, weighted, cbt, seed, cuda_device):
     y = tcq.ub8_decode(out.bits, out.start_state, ct, V, m, T)
     torch.cuda.synchronize()
     np.testing.assert_array_equal(y.cpu().numpy(), oracle_ub8_decode(got[1], got[0], cb, V, m, T).astype(np.float32))
+
+
+def _gemv_cases(n, seed):
+    rng = np.random.default_rng(seed)
+    out = []
+    for q in range(n):
+        if q % 3 == 0:  # the half-block kernel's shapes: L = 16, k = 2, T = 256, 4096-column chunks
+            L, k, T, nb = 16, 2, 256, 16 * int(rng.integers(1, 3))
+            rows = int(rng.choice([1, 37, 148, 2367, 2369, 4000, 7103, 7105, 9000]))
+            rows = min(rows, 4000) if nb > 16 else rows  # keep the oracle's fp64 product small
+        else:
+            L = int(rng.integers(2, 17))
+            k = int(rng.integers(1, min(4, L) + 1))
+            T = int(rng.choice([4, 8, 24, 64, 100, 256, 512]))
+            nb = int(rng.integers(1, 12))
+            rows = int(rng.integers(1, 400))
+        code = "mad" if (L == 16 and rng.integers(0, 3) == 0) else ("f16" if rng.integers(0, 2) else "f32")
+        if code == "f32" and L >= 15:  # the header's rule: a binary16 table from L = 15 on
+            code = "f16"
+        out.append((L, k, T, rows, nb, code, bool(rng.integers(0, 2)), int(rng.integers(0, 2**31))))
+    return out
+
+
+@pytest.mark.parametrize("L,k,T,rows,nb,code,scaled,seed", _gemv_cases(24, 99003), ids=lambda v: str(v))
+def test_gemv_random_shape(L, k, T, rows, nb, code, scaled, seed, cuda_device):
+    import torch
+    from oracle import oracle_mad_codebook
+    from tests.test_gpu_gemv import _check, _rand_stream
+
+    rng = np.random.default_rng(seed)
+    cols = nb * T
+    bits, start = _rand_stream(rng, rows * nb, k, T)
+    scale = rng.lognormal(0.0, 0.5, rows * nb).astype(np.float32) if scaled else None
+    x = rng.standard_normal(cols).astype(np.float32)
+    if code == "mad":
+        cb, cbt = oracle_mad_codebook(L).astype(np.float16), tcq.MAD
+    else:
+        cb = rng.standard_normal(1 << L).astype(np.float16 if code == "f16" else np.float32)
+        cbt = torch.from_numpy(cb).to(cuda_device)
+    y = tcq.gemv(torch.from_numpy(bits.view(np.int32)).to(cuda_device),
+                 torch.from_numpy(start.view(np.int32)).to(cuda_device),
+                 None if scale is None else torch.from_numpy(scale).to(cuda_device),
+                 cbt, L, k, T, rows, cols, torch.from_numpy(x).to(cuda_device))
+    torch.cuda.synchronize()
+    _check(bits, start, scale, cb, L, k, T, rows, cols, x, y.cpu().numpy())
