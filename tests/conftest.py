@@ -19,3 +19,19 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda", 0)
+
+
+@pytest.fixture(autouse=True)
+def _device_error_word_stays_clear(request):
+    """With the bounds-checked build loaded (TCQ_LIBRARY=debug), every GPU test
+    must leave the device error word clear: no index of any instrumented kernel
+    went out of its buffer and no bounded wait gave up."""
+    yield
+    if os.environ.get("TCQ_LIBRARY") != "debug" or request.node.get_closest_marker("gpu") is None:
+        return
+    from trellis_coded_weight_tcq_b200 import tcq
+
+    if tcq._lib is None:  # the test never loaded the library
+        return
+    flags = tcq.device_errors()
+    assert flags == 0, f"device error flags {flags:#x} after {request.node.nodeid}"
