@@ -128,7 +128,9 @@ def test_dyadic_inputs_bit_exact(V, m, T, cbt, cuda_device):
 
 
 @pytest.mark.parametrize("V,m,T,n", [(4, 7, 256, 1000), (1, 0, 17, 65), (3, 8, 27, 31),
-                                     (2, 2, 1024, 33), (8, 5, 4096, 9), (1, 3, 512, 100)])
+                                     (2, 2, 1024, 33), (8, 5, 4096, 9), (1, 3, 512, 100),
+                                     (4, 7, 256, 14213),    # several groups of 32 blocks per CTA
+                                     (4, 7, 256, 100000)])  # more groups than resident warps
 def test_decode_random_streams_bit_exact(V, m, T, n, cuda_device):
     from oracle import oracle_ub8_decode
 
