@@ -27,4 +27,7 @@ def test_host_pipeline_matches_device_encode(chunks, cuda_device):
         assert torch.equal(start, ref.start_state.cpu())
         assert torch.equal(bits, ref.bits.cpu())
         assert torch.equal(cost, ref.path_cost.cpu())
-    assert len(pipe.parts) == min(chunks, wl.n_blocks)
+    # a short lead part, then `chunks` equal parts (one part when chunks is 1)
+    assert len(pipe.parts) == (1 if chunks == 1 else min(chunks + 1, wl.n_blocks))
+    assert pipe.parts[0][0] == 0 and pipe.parts[-1][1] == wl.n_blocks
+    assert all(a[1] == b[0] for a, b in zip(pipe.parts, pipe.parts[1:]))

@@ -549,10 +549,13 @@ def ub8_decode(bits, start_state, codebook, V: int, m: int, T: int, out=None, st
 class HostPipeline:
     """End-to-end encode of host arrays: pinned host -> device -> encode -> host.
 
-    Buffers are allocated once.  ``run`` splits the blocks into ``chunks`` parts:
-    a copy stream brings part i + 1's inputs in while the compute stream encodes
-    and decodes part i, and takes part i's start states, bits and costs back
-    while part i + 1 is encoded, so only the first part's input copy and the last
+    Buffers are allocated once.  ``run`` splits the blocks into a short lead
+    part (1 / (8 chunks) of them) and ``chunks`` equal parts (one part when
+    ``chunks`` is 1): a copy stream
+    brings part i + 1's inputs in while the compute stream encodes and decodes
+    part i, and takes part i's start states, bits and costs back while part i + 1
+    is encoded, so only the lead part's input copy (short, so that the encoder
+    starts early; the next part's copy hides behind its encode) and the last
     part's output copy are not hidden behind the encoder.
     """
 
@@ -565,9 +568,19 @@ class HostPipeline:
         self.x_dev = torch.empty((n_blocks, T), dtype=torch.float32, device=dev)
         self.d_dev = torch.empty((n_blocks, T), dtype=torch.float32, device=dev) if weighted else None
         self.cb_dev = codebook_host.to(dev)
-        per = -(-n_blocks // max(1, chunks))
-        self.parts = [(lo, min(n_blocks, lo + per)) for lo in range(0, n_blocks, per)]
-        self.ws = Workspace(L, k, T, per, cb_dtype_of(self.cb_dev), dev)
+        chunks = max(1, chunks)
+        # part sizes in whole waves of the encoder (every grouped configuration
+        # runs 1, 2, 4 or 8 blocks per SM at a time), so that only the last part
+        # ends on a partly filled round
+        wave = 8 * torch.cuda.get_device_properties(dev).multi_processor_count
+        lead = min(n_blocks, -(-n_blocks // (8 * chunks))) if chunks > 1 else 0  # chunks == 1: one part
+        per = max(1, -(-(n_blocks - lead) // chunks))
+        if n_blocks >= 8 * chunks * wave:
+            lead = -(-lead // wave) * wave
+            per = -(-per // wave) * wave
+        self.parts = ([(0, lead)] if lead else []) + [(lo, min(n_blocks, lo + per))
+                                                      for lo in range(lead, n_blocks, per)]
+        self.ws = Workspace(L, k, T, max(lead, per), cb_dtype_of(self.cb_dev), dev)
         self.enc = Encoded(torch.empty(n_blocks, dtype=torch.int32, device=dev),
                            torch.empty((n_blocks, W), dtype=torch.int32, device=dev),
                            torch.empty(n_blocks, dtype=torch.float32, device=dev))
