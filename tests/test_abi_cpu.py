@@ -243,3 +243,21 @@ def test_debug_build_exports_every_declared_function(lib):
                        capture_output=True, text=True, timeout=300)
     assert r.returncode == 0 and "exports ok" in r.stdout, r.stderr[-2000:]
     assert os.path.exists(path)
+
+
+@pytest.mark.parametrize("n,chunks", [(1, 8), (7, 8), (301, 1), (301, 3), (301, 8), (75775, 8),
+                                      (75776, 8), (229376, 8), (1000003, 8), (5000, 16)])
+def test_host_pipeline_parts(n, chunks):
+    """The end-to-end pipeline's parts cover the blocks once, in order; a lead
+    part then `chunks` parts (one part for chunks = 1); for large inputs every
+    part but the last is a whole number of waves (8 x 148 blocks)."""
+    parts = tcq.host_pipeline_parts(n, chunks, 148)
+    assert parts[0][0] == 0 and parts[-1][1] == n
+    assert all(hi > lo for lo, hi in parts)
+    assert all(a[1] == b[0] for a, b in zip(parts, parts[1:]))
+    assert len(parts) == (1 if chunks == 1 else min(chunks + 1, n))
+    wave = 8 * 148
+    if n >= 8 * chunks * wave:
+        assert all((hi - lo) % wave == 0 for lo, hi in parts[:-1])
+    if chunks > 1 and len(parts) > 2:  # the lead part is the short one
+        assert parts[0][1] - parts[0][0] <= min(hi - lo for lo, hi in parts[1:-1])

@@ -546,6 +546,22 @@ def ub8_decode(bits, start_state, codebook, V: int, m: int, T: int, out=None, st
     return out
 
 
+def host_pipeline_parts(n_blocks: int, chunks: int, sm_count: int):
+    """Block ranges [lo, hi) of HostPipeline: a short lead part (1 / (8 chunks)
+    of the blocks) and ``chunks`` equal parts, one part when ``chunks`` is 1.
+    For large inputs the sizes are whole waves of the encoder (8 blocks per SM:
+    every grouped configuration runs 1, 2, 4 or 8 blocks per SM at a time), so
+    that only the last part ends on a partly filled round."""
+    chunks = max(1, chunks)
+    wave = 8 * max(1, sm_count)
+    lead = min(n_blocks, -(-n_blocks // (8 * chunks))) if chunks > 1 else 0
+    per = max(1, -(-(n_blocks - lead) // chunks))
+    if n_blocks >= 8 * chunks * wave:
+        lead = -(-lead // wave) * wave
+        per = -(-per // wave) * wave
+    return ([(0, lead)] if lead else []) + [(lo, min(n_blocks, lo + per)) for lo in range(lead, n_blocks, per)]
+
+
 class HostPipeline:
     """End-to-end encode of host arrays: pinned host -> device -> encode -> host.
 
@@ -568,19 +584,9 @@ class HostPipeline:
         self.x_dev = torch.empty((n_blocks, T), dtype=torch.float32, device=dev)
         self.d_dev = torch.empty((n_blocks, T), dtype=torch.float32, device=dev) if weighted else None
         self.cb_dev = codebook_host.to(dev)
-        chunks = max(1, chunks)
-        # part sizes in whole waves of the encoder (every grouped configuration
-        # runs 1, 2, 4 or 8 blocks per SM at a time), so that only the last part
-        # ends on a partly filled round
-        wave = 8 * torch.cuda.get_device_properties(dev).multi_processor_count
-        lead = min(n_blocks, -(-n_blocks // (8 * chunks))) if chunks > 1 else 0  # chunks == 1: one part
-        per = max(1, -(-(n_blocks - lead) // chunks))
-        if n_blocks >= 8 * chunks * wave:
-            lead = -(-lead // wave) * wave
-            per = -(-per // wave) * wave
-        self.parts = ([(0, lead)] if lead else []) + [(lo, min(n_blocks, lo + per))
-                                                      for lo in range(lead, n_blocks, per)]
-        self.ws = Workspace(L, k, T, max(lead, per), cb_dtype_of(self.cb_dev), dev)
+        self.parts = host_pipeline_parts(n_blocks, chunks,
+                                         torch.cuda.get_device_properties(dev).multi_processor_count)
+        self.ws = Workspace(L, k, T, max(hi - lo for lo, hi in self.parts), cb_dtype_of(self.cb_dev), dev)
         self.enc = Encoded(torch.empty(n_blocks, dtype=torch.int32, device=dev),
                            torch.empty((n_blocks, W), dtype=torch.int32, device=dev),
                            torch.empty(n_blocks, dtype=torch.float32, device=dev))
